@@ -1,0 +1,474 @@
+"""Benchmark of the block-sparse attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload nsa64k] [--no-decode] [--no-e2e] [--no-cpu-baseline]
+
+One step = the whole hot path over one batch of synthetic input already in
+HBM: pool K/V (block keys + compressed tokens), fused block scoring + top-k,
+and the gated three-branch attention.  Each step is preceded by an L2 flush
+(a 256 MB write) outside the timed events.  Under torchrun every rank runs its
+own independent sequence (seed = rank; weak scaling, no data-path
+collective); the reported time is the max over ranks and ``value`` is the
+aggregate algorithmic TFLOP/s of all ranks.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only, a
+bounded sample of query rows per step).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS, Workload, make_inputs  # noqa
+
+METRIC = "64k-prefill sparse-attn TFLOP/s & tokens/s; decode KV GB/s (fraction of roofline)"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# FP32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (max SM clock)
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+ATTN_KERNEL = "attn_rowwise_kernel"
+ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_scoring_b200", "csrc", "attn_rowwise.cu")
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work (only causally visible keys count)
+# ---------------------------------------------------------------------------
+
+def visible_key_counts(wl: Workload):
+    t = np.arange(wl.seqlen_q, dtype=np.int64) + wl.q_pos0
+    c = t // wl.sel_block
+    out = {}
+    if wl.branches & 2:
+        out["sel"] = np.minimum(wl.top_k - 1, c) * wl.sel_block + (t - c * wl.sel_block + 1)
+    if wl.branches & 4:
+        out["win"] = np.minimum(wl.window, t + 1)
+    if wl.branches & 1:
+        n_cmp = (wl.seqlen_kv - wl.cmp_block) // wl.cmp_stride + 1 if wl.seqlen_kv >= wl.cmp_block else 0
+        nv = np.where(t >= wl.cmp_block - 1, (t - wl.cmp_block + 1) // wl.cmp_stride + 1, 0)
+        out["cmp"] = np.minimum(nv, n_cmp)
+    return out
+
+
+def algorithmic_flops(wl: Workload, rows=None) -> dict:
+    """FLOPs of the branches (2*(d_qk+d_v) per query, head and visible key) and the scoring
+    (2*d_qk per query row, selection unit and candidate block), per sequence."""
+    keys = visible_key_counts(wl)
+    sel = slice(None) if rows is None else np.asarray(rows)
+    per_key = 2 * (wl.d_qk + wl.d_v) * wl.h_q
+    f = {name: float(v[sel].sum()) * per_key for name, v in keys.items()}
+    t = np.arange(wl.seqlen_q, dtype=np.int64) + wl.q_pos0
+    cand = np.minimum(t // wl.sel_block, wl.seqlen_kv // wl.sel_block)
+    f["score"] = float(cand[sel].sum()) * 2 * wl.d_qk * wl.h_sel if wl.branches & 2 else 0.0
+    f["total"] = sum(f.values())
+    return f
+
+
+def decode_bytes(wl: Workload, idx: torch.Tensor) -> float:
+    """Bytes a decode step must read/write: pooled keys, compressed K/V, the union of
+    window and selected tokens per (sequence, KV head), q, gates and out."""
+    B, Hkv = wl.batch, wl.h_kv
+    nb_full = wl.seqlen_kv // wl.sel_block
+    n_cmp = (wl.seqlen_kv - wl.cmp_block) // wl.cmp_stride + 1
+    t = wl.q_pos0
+    kbar = B * Hkv * min(t // wl.sel_block, nb_full) * wl.d_qk * 4
+    cmpb = B * Hkv * n_cmp * (wl.d_qk + wl.d_v) * 2
+    win_lo = max(0, t - wl.window + 1)
+    tok = 0
+    idx_c = idx.cpu().numpy()
+    for b in range(B):
+        for g in range(Hkv):
+            keys = set(range(win_lo, t + 1))
+            for blk in idx_c[b, g, 0]:
+                if blk >= 0:
+                    keys.update(range(blk * wl.sel_block, min((blk + 1) * wl.sel_block, t + 1)))
+            tok += len(keys)
+    kv = tok * (wl.d_qk + wl.d_v) * 2
+    small = B * wl.h_q * (wl.d_qk * 2 + 3 * 4 + wl.d_v * 2)
+    return float(kbar + cmpb + kv + small)
+
+
+# ---------------------------------------------------------------------------
+# Clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index=0):
+        self.proc = None
+        self.path = None
+        self.dev = self._device_id(device_index)
+
+    @staticmethod
+    def _device_id(i):
+        try:
+            u = str(torch.cuda.get_device_properties(i).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return str(i)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.dev], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = float(rows[0][2])
+        loaded = [r for r in rows if float(r[1]) > 0.5 * mx] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(float(r[1]) for r in loaded), "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None,
+                "sm_mhz_min": min(sm)}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    return FALLBACK, "fallback"
+
+
+def traffic_for(kernel: str, source: str):
+    """DRAM bytes per launch recorded by ncu for `kernel`, if its source is unchanged."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    sha = hashlib.sha256(open(source, "rb").read()).hexdigest()
+    return rec["bytes_per_launch"] if rec.get("src_sha256") == sha else None
+
+
+class Prefill:
+    """Device buffers and one timed step of the prefill hot path."""
+
+    def __init__(self, wl: Workload, seed: int):
+        from dynamic_block_sparse_scoring_b200 import abi
+        self.abi, self.wl = abi, wl
+        self.cfg = abi.config(wl)
+        self.x = make_inputs(wl, device="cuda", seed=seed)
+        self.pooled = abi.alloc_pooled(self.cfg, "cuda")
+        self.idx = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, wl.top_k, dtype=torch.int32,
+                               device="cuda")
+        self.out = torch.empty(wl.batch, wl.seqlen_q, wl.h_q, wl.d_v, dtype=torch.bfloat16,
+                               device="cuda")
+        self.launches_per_step = 0
+
+    def step(self, ev=None, pool=True):
+        a, x, p = self.abi, self.x, self.pooled
+        n = 0
+        if ev:
+            ev[0].record()
+        if pool:
+            a.nsa_pool_kv(self.cfg, x["k"], x["v"], p["kbar"], p["kcmp"], p["vcmp"])
+            n += int(self.wl.branches & 2 > 0 and self.cfg.seqlen_kv >= self.cfg.sel_block) + \
+                int(self.wl.branches & 1 > 0)
+        if ev:
+            ev[1].record()
+        if self.wl.branches & 2:
+            a.nsa_topk_select(self.cfg, x["q"], p["kbar"], None, self.idx)
+            n += 1
+        if ev:
+            ev[2].record()
+        a.nsa_sparse_attn_fwd(self.cfg, x["q"], x["k"], x["v"], p["kbar"], p["kcmp"], p["vcmp"],
+                              x["gates"], self.idx if self.wl.branches & 2 else None, self.out)
+        n += 1
+        if ev:
+            ev[3].record()
+        self.launches_per_step = n
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_steps(pf: Prefill, steps: int, warmup: int, world: int, pool=True):
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        pf.step(pool=pool)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for s in range(steps):
+        flush.fill_(float(s))
+        pf.step(evs[s], pool=pool)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier(world)
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                    for e in evs])                                     # ms: pool, select, attn
+    return per, wall
+
+
+def e2e_steps(pf: Prefill, steps: int, warmup: int, world: int):
+    """Same step through the public API with pinned host inputs: H2D copies, the
+    forward (pool + select + attention) and the D2H read of the output all timed."""
+    a, wl = pf.abi, pf.wl
+    host = {k: v.cpu().pin_memory() for k, v in pf.x.items() if v is not None}
+    out_h = torch.empty(pf.out.shape, dtype=pf.out.dtype).pin_memory()
+    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    ws = a.nsa_workspace_size(pf.cfg)
+    work = torch.empty(ws, dtype=torch.uint8, device="cuda")
+
+    def one():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        a.nsa_pool_kv(pf.cfg, dev["k"], dev["v"], pf.pooled["kbar"], pf.pooled["kcmp"],
+                      pf.pooled["vcmp"])
+        a.nsa_sparse_attn_fwd(pf.cfg, dev["q"], dev["k"], dev["v"], pf.pooled["kbar"],
+                              pf.pooled["kcmp"], pf.pooled["vcmp"], dev.get("gates"), None,
+                              pf.out, work, ws)
+        out_h.copy_(pf.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def cpu_baseline(wl: Workload, x, budget_s: float = 15.0, rows_per_step=None):
+    """Time the fp64 oracle on an evenly strided sample of query rows (sequence 0)."""
+    from oracle import nsa_oracle as O
+
+    def f64(t):
+        return t.detach().to("cpu", torch.float64).numpy()
+
+    ocfg = dict(h_q=wl.h_q, h_kv=wl.h_kv, d_qk=wl.d_qk, d_v=wl.d_v, sel_block=wl.sel_block,
+                top_k=wl.top_k, window=wl.window, cmp_block=wl.cmp_block,
+                cmp_stride=wl.cmp_stride, scale=wl.scale, branches=wl.branches,
+                per_head_select=wl.per_head_select)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    K, V = f64(x["k"][0]), f64(x["v"][0])
+    T = wl.seqlen_q
+    t0 = time.perf_counter()
+    pooled = O.pooled_inputs(K, V, wl.sel_block, wl.cmp_block if wl.branches & 1 else 0,
+                             wl.cmp_stride if wl.branches & 1 else 1)
+    t_pool = time.perf_counter() - t0
+    n = 8 if rows_per_step is None else rows_per_step
+    spent, done_rows, flops = 0.0, 0, 0.0
+    rng_rows = np.linspace(0, T - 1, num=max(n, 1)).astype(np.int64)
+    while True:
+        rows = rng_rows
+        rows_t = torch.as_tensor(rows, device=x["q"].device)
+        q = f64(x["q"][0].index_select(0, rows_t))
+        g = None if x["gates"] is None else f64(x["gates"][0].index_select(0, rows_t))
+        t0 = time.perf_counter()
+        O.nsa_rows(ocfg, q, rows + wl.q_pos0, K, V, g, pooled=pooled)
+        spent += time.perf_counter() - t0
+        done_rows += len(rows)
+        flops += algorithmic_flops(wl, rows)["total"]
+        if rows_per_step is not None or spent > budget_s:
+            break
+        rng_rows = np.linspace(done_rows % 7, T - 1, num=n).astype(np.int64)
+    total = spent + t_pool
+    return {"value": flops / total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done_rows} evenly strided query rows of {wl.name} sequence 0 "
+                      f"(all selection units, all branches, K/V pooling included: "
+                      f"{t_pool:.1f} s pooling + {spent:.1f} s rows)",
+            "seconds": total, "rows": done_rows}
+
+
+def run_decode(world: int, steps: int, warmup: int):
+    wl = WORKLOADS["decode64x64k"]
+    pf = Prefill(wl, seed=1000 + (torch.distributed.get_rank() if world > 1 else 0))
+    pf.step()                        # pooled cache built once (cache maintenance, not timed)
+    torch.cuda.synchronize()
+    per, _ = timed_steps(pf, steps, warmup, world, pool=False)
+    ms = max_over_ranks(float(per[:, 1:].sum(axis=1).mean()), world)
+    nbytes = decode_bytes(wl, pf.idx)
+    pk, _ = peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9 * world
+    del pf
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
+            "bytes_per_step": nbytes, "frac": gbs / world / pk["hbm_gbs"],
+            "peak_gbs": pk["hbm_gbs"]}
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    wl = WORKLOADS[args.workload]
+    pf = Prefill(wl, seed=rank)
+    clocks = ClockSampler(torch.cuda.current_device())
+    # warm-up and timed region (clocks sampled during it)
+    clocks.start()
+    per, wall = timed_steps(pf, args.steps, args.warmup, world)
+    clk = clocks.stop()
+    step_ms = per.sum(axis=1)
+    ms = max_over_ranks(float(step_ms.mean()), world)
+    attn_ms = max_over_ranks(float(per[:, 2].mean()), world)
+    fl = algorithmic_flops(wl)
+    fl_all = fl["total"] * wl.batch * world
+    value = fl_all / (ms / 1e3) / 1e12
+    tokens = wl.seqlen_q * wl.batch * world / (ms / 1e3)
+    pk, src = peaks()
+    attn_flops = (fl["total"] - fl["score"]) * wl.batch
+    achieved = attn_flops / (attn_ms / 1e3) / 1e12
+    roof = {"kernel": ATTN_KERNEL, "bound": "alu", "achieved": achieved,
+            "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s", "frac": achieved / ALU_FP32_TFLOPS,
+            "traffic": traffic_for(ATTN_KERNEL, ATTN_SOURCE),
+            "peak_source": "FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz",
+            "flops_per_launch": attn_flops,
+            "share_of_step": float(per[:, 2].mean() / step_ms.mean())}
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_steps(pf, max(2, args.steps // 2), 1, world)
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        e2e = {"value": fl_all / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    x_cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        x_cpu = {k: (v[:1].cpu() if v is not None else None) for k, v in pf.x.items()}
+    launches = pf.launches_per_step * args.steps
+    del pf
+    torch.cuda.empty_cache()
+    decode = None if args.no_decode else run_decode(world, args.steps, args.warmup)
+    cpu = cpu_baseline(wl, x_cpu) if x_cpu is not None else None
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, sigmoid gates)",
+                "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen_q,
+                           "h_q": wl.h_q, "h_kv": wl.h_kv, "d_qk": wl.d_qk, "d_v": wl.d_v,
+                           "sel_block": wl.sel_block, "top_k": wl.top_k, "window": wl.window,
+                           "cmp": [wl.cmp_block, wl.cmp_stride],
+                           "parallelism": f"independent sequences x{world}",
+                           "l2": "256 MB flush before every step; inputs > L2"},
+                "tokens_per_s": tokens, "algorithmic_flops_per_step": fl_all,
+                "stage_ms": {"pool": float(per[:, 0].mean()), "select": float(per[:, 1].mean()),
+                             "attn": float(per[:, 2].mean())},
+                "roofline": roof, "peaks": src, "cpu_baseline": cpu, "e2e": e2e,
+                "decode": decode, "gpu_launches": launches, "clocks": clk,
+                "wall_s_timed_region": wall}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = make_inputs(wl, device=gen_dev, seed=0)
+    x = {k: (v[:1].cpu() if v is not None else None) for k, v in x.items()}
+    times, flops = [], []
+    res = None
+    for s in range(args.warmup + args.steps):
+        res = cpu_baseline(wl, x, rows_per_step=4)
+        if s >= args.warmup:
+            times.append(res["seconds"])
+            flops.append(res["value"] * res["seconds"])
+    value = sum(flops) / sum(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen_q},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"],
+                             "kind": "oracle", "sample": res["sample"] + " per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="nsa64k", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,85 @@
+// Shared device helpers for the sm_100a kernels of libnsa_b200.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nsa.h"
+
+namespace nsa {
+
+// Derived sizes of one problem, computed once on the host.
+struct Shape {
+    int B, Tq, Tk, q0, Hq, Hkv, G, dqk, dv;
+    int bs, topk, win, lc, sc;
+    int nb_full;    // complete selection blocks
+    int nb_all;     // selection blocks including a ragged tail
+    int n_cmp;      // compressed tokens
+    int Hsel;       // selection units (KV heads or query heads)
+    int heads_per_unit;
+    bool per_head;
+    float scale;
+    uint32_t flags;
+};
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    return u;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Order-preserving map of a finite fp32 score to uint32 (-0 treated as +0),
+// packed with the inverted block id so that a larger key means a higher
+// score, and for equal scores a lower block id.
+__device__ __forceinline__ unsigned long long score_key(float s, int blk) {
+    uint32_t u = __float_as_uint(s == 0.0f ? 0.0f : s);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)u << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)blk);
+}
+
+__device__ __forceinline__ int key_block(unsigned long long key) {
+    return (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+}
+
+}  // namespace nsa
+
+// Host-side launchers (defined in the kernel files, called by nsa_abi.cu).
+namespace nsa {
+cudaError_t launch_pool_kv(const Shape& s, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                           float* kbar, __nv_bfloat16* kcmp, __nv_bfloat16* vcmp,
+                           cudaStream_t st);
+cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
+                              const float* scores_in, float* scores_out, int32_t* idx,
+                              cudaStream_t st);
+cudaError_t launch_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                        const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
+                        const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
+                        __nv_bfloat16* out, cudaStream_t st);
+}  // namespace nsa

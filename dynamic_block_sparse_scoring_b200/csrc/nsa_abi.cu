@@ -1,0 +1,190 @@
+// C ABI of libnsa_b200: host-side validation and kernel launches.
+//
+// Every entry point checks its arguments before anything is enqueued and
+// returns a status code; no C++ exception crosses the boundary, nothing is
+// allocated and nothing synchronises.  The operations themselves are defined
+// in include/nsa.h.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace {
+
+using nsa::Shape;
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dqk(int d) { return d == 64 || d == 128 || d == 192 || d == 256; }
+bool supported_dv(int d) { return d == 64 || d == 128 || d == 256; }
+
+// Validates `cfg` and fills the derived sizes.
+nsa_status make_shape(const nsa_config* cfg, Shape* s) {
+    if (!cfg || !s) return NSA_ERR_INVALID_ARG;
+    const nsa_config& c = *cfg;
+    const uint32_t known = NSA_BR_CMP | NSA_BR_SEL | NSA_BR_WIN | NSA_PER_HEAD_SELECT;
+    if (c.flags & ~known) return NSA_ERR_INVALID_ARG;
+    if (!(c.flags & (NSA_BR_CMP | NSA_BR_SEL | NSA_BR_WIN))) return NSA_ERR_INVALID_ARG;
+    if (c.batch < 1 || c.seqlen_q < 0 || c.seqlen_kv < 1 || c.q_pos0 < 0) return NSA_ERR_INVALID_ARG;
+    if ((int64_t)c.q_pos0 + c.seqlen_q > c.seqlen_kv) return NSA_ERR_INVALID_ARG;
+    if (c.h_q < 1 || c.h_kv < 1 || c.h_q % c.h_kv != 0) return NSA_ERR_INVALID_ARG;
+    if (c.d_qk < 1 || c.d_v < 1) return NSA_ERR_INVALID_ARG;
+    if (!isfinite(c.scale)) return NSA_ERR_INVALID_ARG;
+    if (c.sel_block < 1) return NSA_ERR_INVALID_ARG;
+    if ((c.flags & NSA_BR_SEL) && c.top_k < 1) return NSA_ERR_INVALID_ARG;
+    if ((c.flags & NSA_BR_WIN) && c.window < 1) return NSA_ERR_INVALID_ARG;
+    if ((c.flags & NSA_BR_CMP) && (c.cmp_block < 1 || c.cmp_stride < 1)) return NSA_ERR_INVALID_ARG;
+
+    if (!supported_dqk(c.d_qk) || !supported_dv(c.d_v)) return NSA_ERR_UNSUPPORTED;
+    if (c.sel_block % 16 != 0) return NSA_ERR_UNSUPPORTED;
+    if ((c.flags & NSA_BR_SEL) && c.top_k > 32) return NSA_ERR_UNSUPPORTED;
+    if (c.flags & NSA_BR_CMP) {
+        if (c.cmp_block % c.cmp_stride != 0 || c.cmp_block / c.cmp_stride > 16)
+            return NSA_ERR_UNSUPPORTED;
+    }
+    const int G = c.h_q / c.h_kv;
+    const bool per_head = (c.flags & NSA_PER_HEAD_SELECT) != 0;
+    if (!per_head && G > 16) return NSA_ERR_UNSUPPORTED;
+
+    s->B = c.batch;
+    s->Tq = c.seqlen_q;
+    s->Tk = c.seqlen_kv;
+    s->q0 = c.q_pos0;
+    s->Hq = c.h_q;
+    s->Hkv = c.h_kv;
+    s->G = G;
+    s->dqk = c.d_qk;
+    s->dv = c.d_v;
+    s->bs = c.sel_block;
+    s->topk = (c.flags & NSA_BR_SEL) ? c.top_k : 1;
+    s->win = c.window;
+    s->lc = (c.flags & NSA_BR_CMP) ? c.cmp_block : 1;
+    s->sc = (c.flags & NSA_BR_CMP) ? c.cmp_stride : 1;
+    s->nb_full = c.seqlen_kv / c.sel_block;
+    s->nb_all = (c.seqlen_kv + c.sel_block - 1) / c.sel_block;
+    s->n_cmp = (c.flags & NSA_BR_CMP) && c.seqlen_kv >= c.cmp_block
+                   ? (c.seqlen_kv - c.cmp_block) / c.cmp_stride + 1
+                   : 0;
+    s->per_head = per_head;
+    s->Hsel = per_head ? c.h_q : c.h_kv;
+    s->heads_per_unit = per_head ? 1 : G;
+    s->scale = c.scale;
+    s->flags = c.flags;
+    return NSA_OK;
+}
+
+size_t idx_bytes(const Shape& s) {
+    return (size_t)s.B * s.Hsel * s.Tq * s.topk * sizeof(int32_t);
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+nsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nsa_status_string(nsa_status status) {
+    switch (status) {
+        case NSA_OK: return "NSA_OK";
+        case NSA_ERR_INVALID_ARG: return "NSA_ERR_INVALID_ARG: null pointer, bad shape or misaligned pointer";
+        case NSA_ERR_UNSUPPORTED: return "NSA_ERR_UNSUPPORTED: problem outside the GPU path's limits";
+        case NSA_ERR_WORKSPACE: return "NSA_ERR_WORKSPACE: workspace missing or too small";
+        case NSA_ERR_CUDA: return "NSA_ERR_CUDA: a CUDA launch or driver call failed";
+        case NSA_ERR_TIMEOUT: return "NSA_ERR_TIMEOUT: a device-side bounded wait gave up";
+    }
+    return "unknown nsa_status";
+}
+
+nsa_status nsa_workspace_size(const nsa_config* cfg, size_t* bytes) {
+    if (!bytes) return NSA_ERR_INVALID_ARG;
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    *bytes = (cfg->flags & NSA_BR_SEL) ? round_up(idx_bytes(s), 256) : 0;
+    return NSA_OK;
+}
+
+nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, float* kbar,
+                       void* kcmp, void* vcmp, void* stream) {
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    const bool need_sel = (cfg->flags & NSA_BR_SEL) != 0;
+    const bool need_cmp = (cfg->flags & NSA_BR_CMP) != 0;
+    if (!k || (need_sel && !kbar)) return NSA_ERR_INVALID_ARG;
+    if (need_cmp && (!v || !kcmp || !vcmp)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(kcmp) || !aligned16(vcmp))
+        return NSA_ERR_INVALID_ARG;
+    return cuda_status(nsa::launch_pool_kv(
+        s, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        need_sel ? kbar : nullptr, need_cmp ? static_cast<__nv_bfloat16*>(kcmp) : nullptr,
+        need_cmp ? static_cast<__nv_bfloat16*>(vcmp) : nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+nsa_status nsa_score_blocks(const nsa_config* cfg, const void* q, const float* kbar, float* scores,
+                            void* stream) {
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    if (!(cfg->flags & NSA_BR_SEL)) return NSA_ERR_INVALID_ARG;
+    if (!q || !scores || (s.nb_full > 0 && !kbar)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kbar) || !aligned16(scores)) return NSA_ERR_INVALID_ARG;
+    if (s.Tq == 0) return NSA_OK;
+    return cuda_status(nsa::launch_score_topk(s, static_cast<const __nv_bfloat16*>(q), kbar,
+                                              nullptr, scores, nullptr,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kbar,
+                           const float* scores, int32_t* idx, void* stream) {
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    if (!(cfg->flags & NSA_BR_SEL)) return NSA_ERR_INVALID_ARG;
+    if (!idx) return NSA_ERR_INVALID_ARG;
+    if (!scores && (!q || (s.nb_full > 0 && !kbar))) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kbar) || !aligned16(scores) || !aligned16(idx))
+        return NSA_ERR_INVALID_ARG;
+    if (s.Tq == 0) return NSA_OK;
+    return cuda_status(nsa::launch_score_topk(s, static_cast<const __nv_bfloat16*>(q), kbar,
+                                              scores, nullptr, idx,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void* k, const void* v,
+                               const float* kbar, const void* kcmp, const void* vcmp,
+                               const float* gates, const int32_t* idx, void* out, void* workspace,
+                               size_t ws_bytes, void* stream) {
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    const bool sel = (cfg->flags & NSA_BR_SEL) != 0;
+    const bool cmp = (cfg->flags & NSA_BR_CMP) != 0;
+    if (!q || !k || !v || !out) return NSA_ERR_INVALID_ARG;
+    if (cmp && s.n_cmp > 0 && (!kcmp || !vcmp)) return NSA_ERR_INVALID_ARG;
+    if (sel && !idx && s.nb_full > 0 && !kbar) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(kcmp) ||
+        !aligned16(vcmp) || !aligned16(gates) || !aligned16(idx) || !aligned16(out) ||
+        !aligned16(workspace))
+        return NSA_ERR_INVALID_ARG;
+    int32_t* sel_idx = const_cast<int32_t*>(idx);
+    if (sel && !idx) {
+        if (!workspace || ws_bytes < idx_bytes(s)) return NSA_ERR_WORKSPACE;
+        sel_idx = static_cast<int32_t*>(workspace);
+    }
+    if (s.Tq == 0) return NSA_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    if (sel && !idx) {
+        st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
+        if (st != NSA_OK) return st;
+    }
+    return cuda_status(nsa::launch_attn(
+        s, qb, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        static_cast<const __nv_bfloat16*>(kcmp), static_cast<const __nv_bfloat16*>(vcmp), gates,
+        sel_idx, static_cast<__nv_bfloat16*>(out), cs));
+}
+
+}  // extern "C"

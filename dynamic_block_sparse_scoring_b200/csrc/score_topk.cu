@@ -1,0 +1,224 @@
+// Block scoring and top-k block selection.
+//
+// Zhang Xiaojun #94 transcript (bidclub.ai), §4 "Inside Native Sparse
+// Attention": every query has one score per KV block; under GQA the heads of
+// a group add their scores into one selection score and take one top-k, so
+// the whole group reads the same blocks.  LateTalk #103 (zjai.club) §13: the
+// block holding the query is always selected.
+//
+// The group score is linear in the queries, so it is computed as
+// scale * (sum_h q_h) . kbar_b in fp32: one dot product per (query, group,
+// block) instead of one per head.  A CTA takes RT query rows of one
+// selection unit, stages the rows' summed queries and chunks of KC pooled
+// keys in shared memory, forms the RT x KC score tile with FFMA, and keeps a
+// running top-(k-1) per row in the registers of one warp (one key per lane,
+// sorted descending).  A key packs the order-preserving bits of the score
+// with the inverted block id, so a single 64-bit comparison orders by score
+// and then by lower block id.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace nsa {
+
+constexpr int ST_RT = 32;   // query rows per CTA
+constexpr int ST_KC = 64;   // pooled keys per chunk
+constexpr int ST_NT = 256;  // threads per CTA (8 warps x 4 rows)
+
+enum { MODE_SELECT = 0, MODE_SCORES = 1, MODE_SELECT_FROM_SCORES = 2 };
+
+template <int MODE>
+__global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
+                                                           const float* __restrict__ kbar,
+                                                           const float* __restrict__ scores_in,
+                                                           float* __restrict__ scores_out,
+                                                           int32_t* __restrict__ idx) {
+    extern __shared__ float smem[];
+    const int d = s.dqk;
+    const int ld = d + 4;
+    float* qs = smem;                       // [RT][ld]   summed queries
+    float* ks = qs + ST_RT * ld;            // [KC][ld]   pooled keys
+    float* ss = ks + ST_KC * ld;            // [RT][KC+1] score tile
+
+    const int i0 = blockIdx.x * ST_RT;
+    const int u = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int kvh = s.per_head ? u / s.G : u;
+    const int h0 = s.per_head ? u : u * s.G;
+    const int nh = s.heads_per_unit;
+    const int nrows = min(ST_RT, s.Tq - i0);
+
+    // current block of the last row bounds the candidates of the whole tile
+    const int c_last = (s.q0 + i0 + nrows - 1) / s.bs;
+    const int cmax = min(c_last, s.nb_full);
+
+    if (MODE != MODE_SELECT_FROM_SCORES) {
+        const int nvec = d / 8;
+        for (int p = tid; p < ST_RT * nvec; p += ST_NT) {
+            const int r = p / nvec, vec = p % nvec;
+            float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (r < nrows) {
+                const __nv_bfloat16* src = q + (((size_t)b * s.Tq + i0 + r) * s.Hq + h0) * d + vec * 8;
+                for (int hh = 0; hh < nh; ++hh) {
+                    float f[8];
+                    unpack8(*reinterpret_cast<const uint4*>(src + (size_t)hh * d), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qs[r * ld + vec * 8 + e] = acc[e];
+        }
+    }
+
+    const int K1 = s.topk - 1;               // past blocks kept per row
+    unsigned long long key[4] = {0ull, 0ull, 0ull, 0ull};   // lane's slot of rows 4*warp + j
+
+    for (int b0 = 0; b0 < cmax; b0 += ST_KC) {
+        const int nk = min(ST_KC, cmax - b0);
+        if (MODE != MODE_SELECT_FROM_SCORES) {
+            const float* src = kbar + ((size_t)(b * s.Hkv + kvh) * s.nb_full + b0) * d;
+            const int nf4 = d / 4;
+            for (int p = tid; p < nk * nf4; p += ST_NT) {
+                const int r = p / nf4, c4 = p % nf4;
+                *reinterpret_cast<float4*>(ks + r * ld + c4 * 4) =
+                    *reinterpret_cast<const float4*>(src + (size_t)r * d + c4 * 4);
+            }
+            __syncthreads();
+            // thread -> row r, blocks bg, bg+8, ..., bg+56 of the chunk
+            const int r = tid >> 3, bg = tid & 7;
+            float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            const float* qr = qs + r * ld;
+            for (int c = 0; c < d; c += 4) {
+                const float4 qv = *reinterpret_cast<const float4*>(qr + c);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const float4 kv = *reinterpret_cast<const float4*>(ks + (bg + 8 * m) * ld + c);
+                    acc[m] = fmaf(qv.x, kv.x, acc[m]);
+                    acc[m] = fmaf(qv.y, kv.y, acc[m]);
+                    acc[m] = fmaf(qv.z, kv.z, acc[m]);
+                    acc[m] = fmaf(qv.w, kv.w, acc[m]);
+                }
+            }
+            const int t = s.q0 + i0 + r;
+            const int cr = t / s.bs;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int jj = bg + 8 * m;
+                const int blk = b0 + jj;
+                const bool valid = (r < nrows) && (jj < nk) && (blk < cr);
+                const float val = s.scale * acc[m];
+                if (MODE == MODE_SCORES) {
+                    if (r < nrows && jj < nk) {
+                        float w = blk < cr ? val : (blk == cr ? INFINITY : -INFINITY);
+                        scores_out[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + blk] = w;
+                    }
+                } else {
+                    ss[r * (ST_KC + 1) + jj] = valid ? val : -INFINITY;
+                }
+            }
+        } else {
+            for (int p = tid; p < ST_RT * ST_KC; p += ST_NT) {
+                const int r = p / ST_KC, jj = p % ST_KC;
+                const int blk = b0 + jj;
+                float val = -INFINITY;
+                if (r < nrows && jj < nk) {
+                    const int cr = (s.q0 + i0 + r) / s.bs;
+                    if (blk < cr)
+                        val = scores_in[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + blk];
+                }
+                ss[r * (ST_KC + 1) + jj] = val;
+            }
+        }
+        __syncthreads();
+
+        if (MODE != MODE_SCORES && K1 > 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = warp * 4 + j;
+                unsigned long long thr = __shfl_sync(0xffffffffu, key[j], K1 - 1);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int jj = lane + 32 * half;
+                    const float sv = ss[r * (ST_KC + 1) + jj];
+                    const unsigned long long ck = (sv != -INFINITY) ? score_key(sv, b0 + jj) : 0ull;
+                    unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
+                    while (mask) {
+                        const int src = __ffs(mask) - 1;
+                        const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
+                        const unsigned long long mine = key[j];
+                        const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && mine > x));
+                        const unsigned long long up = __shfl_up_sync(0xffffffffu, mine, 1);
+                        if (lane < K1) {
+                            if (lane == p) key[j] = x;
+                            else if (lane > p) key[j] = up;
+                        }
+                        thr = __shfl_sync(0xffffffffu, key[j], K1 - 1);
+                        mask &= ~(1u << src);
+                        mask &= __ballot_sync(0xffffffffu, ck > thr);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    if (MODE == MODE_SCORES) {
+        // columns at and after the last chunk: +inf at the current block, -inf after it
+        for (int p = tid; p < nrows * s.nb_all; p += ST_NT) {
+            const int r = p / s.nb_all, j = p % s.nb_all;
+            if (j < cmax) continue;
+            const int cr = (s.q0 + i0 + r) / s.bs;
+            scores_out[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + j] =
+                j == cr ? INFINITY : -INFINITY;
+        }
+        return;
+    }
+
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int r = warp * 4 + j;
+        if (r >= nrows) continue;
+        const int cr = (s.q0 + i0 + r) / s.bs;
+        const bool have = lane < K1 && key[j] != 0ull;
+        const int blk = have ? key_block(key[j]) : 0x7fffffff;
+        const int npast = __popc(__ballot_sync(0xffffffffu, have));
+        int rank = 0;
+        for (int o = 0; o < 32; ++o) {
+            const int other = __shfl_sync(0xffffffffu, blk, o);
+            rank += (other < blk) ? 1 : 0;
+        }
+        int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.topk;
+        if (have) dst[rank] = blk;
+        if (lane == 0) dst[npast] = cr;
+        if (lane > npast && lane < s.topk) dst[lane] = -1;
+    }
+}
+
+cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
+                              const float* scores_in, float* scores_out, int32_t* idx,
+                              cudaStream_t st) {
+    const int ld = s.dqk + 4;
+    const size_t smem = ((size_t)ST_RT * ld + (size_t)ST_KC * ld + (size_t)ST_RT * (ST_KC + 1)) *
+                        sizeof(float);
+    dim3 grid((s.Tq + ST_RT - 1) / ST_RT, s.Hsel, s.B);
+    if (scores_out) {
+        cudaFuncSetAttribute(score_topk_kernel<MODE_SCORES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        score_topk_kernel<MODE_SCORES><<<grid, ST_NT, smem, st>>>(s, q, kbar, nullptr, scores_out,
+                                                                  nullptr);
+    } else if (scores_in) {
+        cudaFuncSetAttribute(score_topk_kernel<MODE_SELECT_FROM_SCORES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        score_topk_kernel<MODE_SELECT_FROM_SCORES><<<grid, ST_NT, smem, st>>>(
+            s, nullptr, nullptr, scores_in, nullptr, idx);
+    } else {
+        cudaFuncSetAttribute(score_topk_kernel<MODE_SELECT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        score_topk_kernel<MODE_SELECT><<<grid, ST_NT, smem, st>>>(s, q, kbar, nullptr, nullptr,
+                                                                  idx);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace nsa

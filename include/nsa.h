@@ -1,0 +1,161 @@
+/*
+ * nsa.h - C ABI of libnsa_b200.so: query-dependent top-k block-sparse causal
+ * attention forward (NSA-style group-shared selection, MoBA-style per-head
+ * selection) for NVIDIA B200 (sm_100a).
+ *
+ * Method, as described in the Zhang Xiaojun #94 transcript (bidclub.ai):
+ *   §2 "Attention From First Principles" - scaled dot products, causal mask,
+ *      softmax, weighted sum of values;
+ *   §4 "Inside Native Sparse Attention", Figure 2 - KV cut into contiguous
+ *      blocks; a compressed branch over pooled block tokens, a selected branch
+ *      over the top-k scoring blocks, a sliding-window branch, each multiplied
+ *      by a per-token gate and summed; GQA heads add their block scores so the
+ *      group shares one block set;
+ *   §7 "Kimi Simplifies The Sparse Route" - MoBA: mean-pooled block keys,
+ *      per-head selection, selected branch only;
+ * and LateTalk #103 (zjai.club) §13 - the block holding the query is always
+ * selected.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors are dense, row-major, caller-owned DEVICE memory (16-byte aligned).
+ *   q      [B, Tq, Hq, d_qk]        bf16   head h belongs to KV head h / (Hq/Hkv)
+ *   k      [B, Hkv, Tkv, d_qk]      bf16
+ *   v      [B, Hkv, Tkv, d_v]       bf16
+ *   kbar   [B, Hkv, nb_full, d_qk]  fp32   nb_full = Tkv / sel_block (complete blocks)
+ *   kcmp   [B, Hkv, n_cmp, d_qk]    bf16   n_cmp = (Tkv - cmp_block) / cmp_stride + 1
+ *   vcmp   [B, Hkv, n_cmp, d_v]     bf16
+ *   scores [B, Hsel, Tq, nb_all]    fp32   nb_all = ceil(Tkv / sel_block)
+ *   idx    [B, Hsel, Tq, top_k]     int32  ascending block ids, -1 padded
+ *   gates  [B, Tq, Hq, 3]           fp32   (compressed, selected, window)
+ *   out    [B, Tq, Hq, d_v]         bf16
+ * Hsel = Hkv (group-shared selection) or Hq (NSA_PER_HEAD_SELECT).
+ * Query i of a sequence sits at KV position t = q_pos0 + i (prefill: q_pos0 = 0
+ * and Tq = Tkv; decode: Tq = 1, q_pos0 = Tkv - 1).  Its current block is
+ * c = t / sel_block.
+ *
+ * `stream` is a cudaStream_t (NULL = legacy default stream).  Every entry
+ * point validates its arguments on the host before launching anything and
+ * returns NSA_ERR_INVALID_ARG / NSA_ERR_UNSUPPORTED without side effects;
+ * launch failures return NSA_ERR_CUDA.  Work is enqueued asynchronously on
+ * `stream`: no entry point synchronises, allocates device memory or keeps a
+ * pointer after it returns.  Calls are thread-safe; two calls that write the
+ * same buffers must be ordered by the caller.
+ *
+ * GPU-path limits (NSA_ERR_UNSUPPORTED otherwise): d_qk in {64, 128, 192, 256},
+ * d_v in {64, 128, 256}; sel_block a multiple of 16; 1 <= top_k <= 32;
+ * cmp_block a multiple of cmp_stride; Hq a multiple of Hkv, Hq/Hkv <= 16 for
+ * group-shared selection.
+ */
+#ifndef NSA_B200_NSA_H
+#define NSA_B200_NSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NSA_OK = 0,
+    NSA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misaligned pointer */
+    NSA_ERR_UNSUPPORTED = 2,   /* valid problem outside the GPU path's limits */
+    NSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than nsa_workspace_size() */
+    NSA_ERR_CUDA = 4,          /* a CUDA launch or driver call failed */
+    NSA_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up */
+} nsa_status;
+
+/* Branch and mode bits of nsa_config.flags. */
+#define NSA_BR_CMP 1u            /* compressed (coarse) branch */
+#define NSA_BR_SEL 2u            /* selected-block branch */
+#define NSA_BR_WIN 4u            /* sliding-window branch */
+#define NSA_PER_HEAD_SELECT 8u   /* MoBA: every query head selects its own blocks */
+
+typedef struct {
+    int32_t batch;       /* B: independent sequences */
+    int32_t seqlen_q;    /* Tq: queries per sequence */
+    int32_t seqlen_kv;   /* Tkv: keys/values per sequence */
+    int32_t q_pos0;      /* KV position of query 0; q_pos0 + Tq <= Tkv */
+    int32_t h_q;         /* Hq: query heads */
+    int32_t h_kv;        /* Hkv: key/value heads */
+    int32_t d_qk;        /* query/key head dimension */
+    int32_t d_v;         /* value head dimension */
+    int32_t sel_block;   /* tokens per selection block */
+    int32_t top_k;       /* blocks kept per query, the current block included */
+    int32_t window;      /* sliding window: keys [t - window + 1, t] */
+    int32_t cmp_block;   /* tokens per compressed token */
+    int32_t cmp_stride;  /* distance between compressed tokens */
+    float scale;         /* logit scale, normally 1/sqrt(d_qk) */
+    uint32_t flags;      /* NSA_BR_* | NSA_PER_HEAD_SELECT */
+} nsa_config;
+
+/*
+ * Bytes of device workspace nsa_sparse_attn_fwd needs for `cfg` when it
+ * selects the blocks itself (idx == NULL).  Writes 0 when no workspace is
+ * needed.  Pure host function.
+ */
+nsa_status nsa_workspace_size(const nsa_config* cfg, size_t* bytes);
+
+/*
+ * Block representations (transcript #94 §4 Figure 2 "compression", §7 mean
+ * pooling).  kbar[b,h,j,:] = mean of k over tokens [j*sel_block, (j+1)*sel_block)
+ * for every complete block (fp32).  When NSA_BR_CMP is set, kcmp/vcmp[b,h,j,:]
+ * = mean of k/v over [j*cmp_stride, j*cmp_stride + cmp_block), rounded to bf16;
+ * otherwise kcmp and vcmp may be NULL.  kbar may be NULL when NSA_BR_SEL is
+ * clear.  Reads k and v once.
+ */
+nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, float* kbar,
+                       void* kcmp, void* vcmp, void* stream);
+
+/*
+ * Block selection scores (transcript #94 §4: one score per query and block;
+ * group heads add theirs).  scores[b,u,i,j] =
+ *   scale * sum_{h in unit u} q[b,i,h,:] . kbar[b,kv(u),j,:]   for j < c(t),
+ *   +INFINITY for j == c(t) (always selected), -INFINITY for j > c(t).
+ * Computed in fp32 as scale * (sum_h q_h) . kbar_j (the sum is linear).
+ */
+nsa_status nsa_score_blocks(const nsa_config* cfg, const void* q, const float* kbar,
+                            float* scores, void* stream);
+
+/*
+ * Top-k block sets (transcript #94 §4 Figure 2: keep the k best blocks;
+ * LateTalk #103 §13: the current block is always kept).  For every (b, u, i):
+ * idx = {c(t)} plus the (top_k - 1) best past blocks by score, equal scores
+ * resolved to the lower block index; written ascending and padded with -1 to
+ * top_k entries (a row keeps min(top_k, c(t) + 1) blocks).  If `scores` is
+ * NULL the scores are computed on the fly from q and kbar (fused, nothing
+ * materialised); otherwise they are read from `scores` (layout above) and q,
+ * kbar may be NULL.
+ */
+nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kbar,
+                           const float* scores, int32_t* idx, void* stream);
+
+/*
+ * Gated sparse attention forward (transcript #94 §4 Figure 2).  For each
+ * query row (position t) and head h:
+ *   o_cmp = softmax attention over compressed tokens j with
+ *           j*cmp_stride + cmp_block - 1 <= t           (NSA_BR_CMP)
+ *   o_sel = softmax attention over the tokens u <= t of the blocks in idx (NSA_BR_SEL)
+ *   o_win = softmax attention over keys max(0, t-window+1) .. t           (NSA_BR_WIN)
+ *   out   = g0*o_cmp + g1*o_sel + g2*o_win   (gates NULL: weight 1 each)
+ * A branch with no visible key contributes 0.  Softmax and accumulation run in
+ * fp32; out is rounded to bf16 once.
+ * idx may be NULL, in which case the blocks are selected as nsa_topk_select
+ * does (needs q, kbar and a workspace of nsa_workspace_size() bytes);
+ * otherwise kbar may be NULL and the workspace may be NULL/0.
+ * kcmp/vcmp are read only with NSA_BR_CMP.
+ */
+nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void* k,
+                               const void* v, const float* kbar, const void* kcmp,
+                               const void* vcmp, const float* gates, const int32_t* idx,
+                               void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* nsa_status_string(nsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_B200_NSA_H */

@@ -1,0 +1,94 @@
+"""Helpers shared by the GPU parity tests: run the C-ABI path on seeded inputs and
+compare it with the fp64 oracle.
+
+Tolerances (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
+* block indices: identical, except rows whose oracle gap between the last kept
+  and the first dropped fp32-rounded score is below TIE_EPS; there the GPU set
+  must still be a valid top-k (current block kept, right size, every kept past
+  block within TIE_EPS of every dropped one);
+* outputs: max |gpu - oracle| <= OUT_MAX_ABS and mean |gpu - oracle| <= OUT_MEAN_ABS;
+* pooled keys (fp32): <= 1e-5 absolute; compressed tokens (bf16): one bf16
+  rounding of the fp64 mean (relative 2^-8) plus 1e-6.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from dynamic_block_sparse_scoring_b200 import abi
+from dynamic_block_sparse_scoring_b200.workloads import Workload, make_inputs
+from oracle import nsa_oracle as O
+
+TIE_EPS = 1e-5
+OUT_MAX_ABS = 2e-2
+OUT_MEAN_ABS = 2e-3
+SCORE_ATOL = 1e-4
+SCORE_RTOL = 1e-5
+
+
+def f64(x: torch.Tensor) -> np.ndarray:
+    return x.detach().to("cpu", torch.float64).numpy()
+
+
+def oracle_cfg(wl: Workload) -> dict:
+    return dict(h_q=wl.h_q, h_kv=wl.h_kv, d_qk=wl.d_qk, d_v=wl.d_v, sel_block=wl.sel_block,
+                top_k=wl.top_k, window=wl.window, cmp_block=wl.cmp_block,
+                cmp_stride=wl.cmp_stride, scale=wl.scale, branches=wl.branches,
+                per_head_select=wl.per_head_select, gated=wl.gated)
+
+
+class GpuRun:
+    """Inputs for a workload on cuda:0 and the library's outputs for them."""
+
+    def __init__(self, wl: Workload, seed=None):
+        self.wl = wl
+        self.cfg = abi.config(wl)
+        self.x = make_inputs(wl, device="cuda", seed=seed)
+        self.pooled = abi.alloc_pooled(self.cfg, "cuda")
+        abi.nsa_pool_kv(self.cfg, self.x["k"], self.x["v"], self.pooled["kbar"],
+                        self.pooled["kcmp"], self.pooled["vcmp"])
+        self.idx = None
+        if wl.branches & abi.NSA_BR_SEL:
+            self.idx = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, wl.top_k, dtype=torch.int32,
+                                   device="cuda")
+            abi.nsa_topk_select(self.cfg, self.x["q"], self.pooled["kbar"], None, self.idx)
+        self.out, _ = abi.forward(self.cfg, self.x["q"], self.x["k"], self.x["v"],
+                                  self.x["gates"], pooled=self.pooled)
+        torch.cuda.synchronize()
+
+    def oracle_rows(self, b: int, rows, idx=None):
+        """Oracle (out, idx, gap) for sequence b and the given query rows."""
+        wl, x = self.wl, self.x
+        rows = np.asarray(rows)
+        rows_t = torch.as_tensor(rows, device=x["q"].device)
+        q = f64(x["q"][b].index_select(0, rows_t))
+        K, V = f64(x["k"][b]), f64(x["v"][b])
+        g = None if x["gates"] is None else f64(x["gates"][b].index_select(0, rows_t))
+        pos = rows + wl.q_pos0
+        return O.nsa_rows(oracle_cfg(wl), q, pos, K, V, g, idx=idx)
+
+
+def check_idx(gpu_idx: np.ndarray, ora_idx: np.ndarray, gap: np.ndarray, scores: np.ndarray,
+              positions: np.ndarray, sel_block: int, top_k: int):
+    """gpu_idx/ora_idx [U, R, k], gap [U, R], scores [U, R, nb] (oracle, -inf non-candidates)."""
+    differ = (gpu_idx != ora_idx).any(axis=-1)
+    assert not (differ & ~(gap < TIE_EPS)).any(), \
+        f"{int((differ & ~(gap < TIE_EPS)).sum())} rows select different blocks without a near-tie"
+    for u, r in zip(*np.nonzero(differ)):
+        c = int(positions[r]) // sel_block
+        got = [int(b) for b in gpu_idx[u, r] if b >= 0]
+        assert got == sorted(got) and c in got and len(got) == min(top_k, c + 1)
+        past = [b for b in got if b != c]
+        dropped = [b for b in range(c) if b not in past]
+        if past and dropped:
+            s = scores[u, r]
+            assert min(s[past]) >= max(s[dropped]) - TIE_EPS
+    return int(differ.sum())
+
+
+def check_out(gpu: np.ndarray, ora: np.ndarray, what=""):
+    err = np.abs(gpu - ora)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite output"
+    assert err.max() <= OUT_MAX_ABS, f"{what}: max abs err {err.max():.3e}"
+    assert err.mean() <= OUT_MEAN_ABS, f"{what}: mean abs err {err.mean():.3e}"
+    return float(err.max()), float(err.mean())

@@ -1,0 +1,117 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every declared symbol,
+and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nsa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(nsa_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from dynamic_block_sparse_scoring_b200 import build
+    build.build()
+    from dynamic_block_sparse_scoring_b200 import abi as a
+    return a
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["nsa_score_blocks", "nsa_topk_select", "nsa_sparse_attn_fwd", "nsa_pool_kv",
+                 "nsa_workspace_size", "nsa_status_string"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(abi):
+    lib = ctypes.CDLL(abi._LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_config_struct_layout_matches_header(abi):
+    # 13 int32 + float + uint32, no padding
+    assert ctypes.sizeof(abi.NsaConfig) == 15 * 4
+
+
+def test_status_strings(abi):
+    for code in range(6):
+        assert abi.nsa_status_string(code).startswith(abi.STATUS[code])
+
+
+def _cfg(abi, **kw):
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
+    return abi.config(WORKLOADS["tiny"], **kw)
+
+
+def test_workspace_size_is_idx_buffer(abi):
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
+    for name, wl in WORKLOADS.items():
+        cfg = abi.config(wl)
+        n = abi.nsa_workspace_size(cfg)
+        want = wl.batch * wl.h_sel * wl.seqlen_q * wl.top_k * 4
+        assert n >= want and n % 256 == 0, name
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(h_q=3, h_kv=2), 1),          # h_q not a multiple of h_kv
+    (dict(batch=0), 1),
+    (dict(seqlen_kv=0), 1),
+    (dict(q_pos0=1), 1),               # q_pos0 + Tq > Tkv
+    (dict(flags=0), 1),
+    (dict(flags=64 | 7), 1),
+    (dict(top_k=0), 1),
+    (dict(window=0), 1),
+    (dict(cmp_stride=0), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(d_qk=96), 2),
+    (dict(d_v=32), 2),
+    (dict(sel_block=24), 2),
+    (dict(top_k=33), 2),
+    (dict(cmp_block=24, cmp_stride=16), 2),
+    (dict(h_q=32, h_kv=1), 2),         # group of 32 heads
+])
+def test_invalid_configs_rejected_on_host(abi, bad, status):
+    cfg = _cfg(abi, **bad)
+    n = ctypes.c_size_t(0)
+    assert abi.lib.nsa_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == status
+    # the compute entry points validate before launching: no device is touched
+    fake = 1 << 20
+    assert abi.lib.nsa_pool_kv(ctypes.byref(cfg), fake, fake, fake, fake, fake, None) == status
+    assert abi.lib.nsa_sparse_attn_fwd(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake,
+                                       fake, fake, fake, fake, 1 << 30, None) == status
+
+
+def test_null_and_misaligned_pointers_rejected(abi):
+    cfg = _cfg(abi)
+    L = abi.lib
+    c = ctypes.byref(cfg)
+    good, odd = 1 << 20, (1 << 20) + 8
+    assert L.nsa_pool_kv(c, None, good, good, good, good, None) == 1
+    assert L.nsa_pool_kv(c, odd, good, good, good, good, None) == 1
+    assert L.nsa_score_blocks(c, good, good, None, None) == 1
+    assert L.nsa_topk_select(c, good, good, None, None, None) == 1
+    assert L.nsa_topk_select(c, None, None, None, good, None) == 1
+    assert L.nsa_sparse_attn_fwd(c, good, good, good, good, good, good, good, good, None, None, 0,
+                                 None) == 1
+    # selecting inside needs a workspace of nsa_workspace_size() bytes
+    assert L.nsa_sparse_attn_fwd(c, good, good, good, good, good, good, good, None, good, None, 0,
+                                 None) == 3
+    assert L.nsa_sparse_attn_fwd(c, good, good, good, good, good, good, good, None, good, good, 16,
+                                 None) == 3
+    assert L.nsa_workspace_size(c, None) == 1
+    assert L.nsa_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == 1
+
+
+def test_binding_raises_on_error(abi):
+    cfg = _cfg(abi, batch=0)
+    with pytest.raises(abi.NsaError):
+        abi.nsa_workspace_size(cfg)

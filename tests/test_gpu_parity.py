@@ -1,0 +1,174 @@
+"""GPU parity: the C-ABI CUDA path against the fp64 oracle, element by element.
+
+Small problems are compared on every row; the full-size workloads on sampled
+rows (first rows, evenly strided rows, block boundaries, the last row) and,
+for decode, on sampled sequences.  Tolerances are stated in tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS, BR_CMP, BR_SEL, BR_WIN, row_sample
+from oracle import nsa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+from dynamic_block_sparse_scoring_b200 import abi
+from tests.parity import GpuRun, check_idx, check_out, f64, SCORE_ATOL, SCORE_RTOL
+
+TINY = WORKLOADS["tiny"]
+
+# Edge cases around the tiny workload: ragged lengths, degenerate branch sizes,
+# every block kept, per-head selection under GQA, chunked prefill, batch > 1,
+# other head dimensions, and scaled-down versions of the big workloads.
+EDGE = {
+    "tiny": TINY,
+    "ragged_1000": TINY.with_(name="ragged_1000", seqlen_q=1000, seqlen_kv=1000),
+    "ragged_77": TINY.with_(name="ragged_77", seqlen_q=77, seqlen_kv=77, sel_block=16, top_k=3,
+                            window=20, cmp_block=16, cmp_stride=8),
+    "every_block": TINY.with_(name="every_block", seqlen_q=512, seqlen_kv=512, top_k=32,
+                              branches=BR_SEL, gated=False),
+    "gqa_per_head": TINY.with_(name="gqa_per_head", seqlen_q=700, seqlen_kv=700, h_q=8, h_kv=2,
+                               d_qk=128, d_v=128, per_head_select=True),
+    "window_1": TINY.with_(name="window_1", seqlen_q=300, seqlen_kv=300, window=1),
+    "shorter_than_cmp_block": TINY.with_(name="short", seqlen_q=20, seqlen_kv=20),
+    "single_query": TINY.with_(name="single_query", seqlen_q=1, seqlen_kv=1),
+    "top1": TINY.with_(name="top1", seqlen_q=400, seqlen_kv=400, top_k=1),
+    "chunked_prefill": TINY.with_(name="chunked", seqlen_q=300, seqlen_kv=1000, q_pos0=700),
+    "batch3": TINY.with_(name="batch3", batch=3, seqlen_q=256, seqlen_kv=256),
+    "d256": TINY.with_(name="d256", seqlen_q=333, seqlen_kv=333, h_q=4, h_kv=2, d_qk=256,
+                       d_v=256),
+    "moba_small": WORKLOADS["moba32k"].with_(name="moba_small", seqlen_q=4096, seqlen_kv=4096,
+                                             h_q=4, h_kv=4),
+    "nsa_small": WORKLOADS["nsa64k"].with_(name="nsa_small", seqlen_q=2048, seqlen_kv=2048,
+                                           h_q=16, h_kv=1),
+    "cmp_identity": TINY.with_(name="cmp_identity", seqlen_q=200, seqlen_kv=200, cmp_block=1,
+                               cmp_stride=1),
+}
+
+
+def compare_run(run: GpuRun, rows_per_seq, seqs=None):
+    wl = run.wl
+    seqs = range(wl.batch) if seqs is None else seqs
+    for b in seqs:
+        rows = np.asarray(rows_per_seq)
+        pos = rows + wl.q_pos0
+        # selection against the oracle's own selection
+        if wl.branches & BR_SEL:
+            K = f64(run.x["k"][b])
+            rows_t = torch.as_tensor(rows, device="cuda")
+            q = f64(run.x["q"][b].index_select(0, rows_t))
+            Kbar = O.pool_block_keys(K, wl.sel_block)
+            nb_all = -(-wl.seqlen_kv // wl.sel_block)
+            s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
+                               wl.per_head_select, nb_all)
+            ora_idx, gap = O.select_blocks(s, pos, wl.sel_block, wl.top_k)
+            gpu_idx = run.idx[b].index_select(1, rows_t).cpu().numpy()
+            check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
+            idx_for_out = gpu_idx
+        else:
+            idx_for_out = None
+        # outputs, with the oracle attending over the blocks the GPU kept
+        ora_out, _, _ = run.oracle_rows(b, rows, idx=idx_for_out)
+        gpu_out = f64(run.out[b].index_select(0, torch.as_tensor(rows, device="cuda")))
+        check_out(gpu_out, ora_out, f"{wl.name} seq {b}")
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_small_problem_all_rows(name):
+    wl = EDGE[name]
+    run = GpuRun(wl)
+    compare_run(run, np.arange(wl.seqlen_q))
+
+
+def test_pool_kv_matches_oracle():
+    for wl in [TINY, EDGE["ragged_77"], WORKLOADS["nsa64k"], WORKLOADS["moba32k"]]:
+        run = GpuRun(wl) if wl.seqlen_q <= 4096 else None
+        if run is None:
+            cfg = abi.config(wl)
+            from dynamic_block_sparse_scoring_b200.workloads import make_inputs
+            x = make_inputs(wl, device="cuda")
+            pooled = abi.alloc_pooled(cfg, "cuda")
+            abi.nsa_pool_kv(cfg, x["k"], x["v"], pooled["kbar"], pooled["kcmp"], pooled["vcmp"])
+            torch.cuda.synchronize()
+        else:
+            x, pooled = run.x, run.pooled
+        K, V = f64(x["k"][0]), f64(x["v"][0])
+        if wl.branches & BR_SEL:
+            np.testing.assert_allclose(f64(pooled["kbar"][0]), O.pool_block_keys(K, wl.sel_block),
+                                       rtol=0, atol=1e-5)
+        if wl.branches & BR_CMP:
+            for got, X, d in [(pooled["kcmp"], K, wl.d_qk), (pooled["vcmp"], V, wl.d_v)]:
+                ref = O.compress(X, wl.cmp_block, wl.cmp_stride)
+                err = np.abs(f64(got[0]) - ref)
+                assert (err <= np.abs(ref) * 2.0 ** -8 + 1e-6).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_77", "gqa_per_head", "chunked_prefill",
+                                  "nsa_small"])
+def test_materialised_scores_and_select_from_scores(name):
+    wl = EDGE[name]
+    run = GpuRun(wl)
+    cfg = run.cfg
+    nb_all = -(-wl.seqlen_kv // wl.sel_block)
+    scores = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, nb_all, device="cuda")
+    abi.nsa_score_blocks(cfg, run.x["q"], run.pooled["kbar"], scores)
+    idx2 = torch.empty_like(run.idx)
+    abi.nsa_topk_select(cfg, None, None, scores, idx2)
+    torch.cuda.synchronize()
+    # selecting from the materialised scores gives the fused selection exactly
+    assert torch.equal(idx2, run.idx)
+    pos = np.arange(wl.seqlen_q) + wl.q_pos0
+    for b in range(wl.batch):
+        q = f64(run.x["q"][b])
+        Kbar = O.pool_block_keys(f64(run.x["k"][b]), wl.sel_block)
+        s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
+                           wl.per_head_select, nb_all)
+        got = scores[b].cpu().double().numpy()
+        cur = pos // wl.sel_block
+        for r in range(wl.seqlen_q):
+            c = cur[r]
+            np.testing.assert_allclose(got[:, r, :c], s[:, r, :c], rtol=SCORE_RTOL,
+                                       atol=SCORE_ATOL)
+            assert np.all(got[:, r, c] == np.inf)
+            assert np.all(got[:, r, c + 1:] == -np.inf)
+
+
+def test_every_block_kept_is_dense_causal_attention():
+    """Library SDPA (fp32) as an independent check of the special case."""
+    wl = EDGE["every_block"].with_(h_q=8, h_kv=2)
+    run = GpuRun(wl)
+    q = run.x["q"][0].float().permute(1, 0, 2)
+    k = run.x["k"][0].float().repeat_interleave(4, dim=0)
+    v = run.x["v"][0].float().repeat_interleave(4, dim=0)
+    ref = F.scaled_dot_product_attention(q, k, v, is_causal=True, scale=wl.scale).permute(1, 0, 2)
+    check_out(run.out[0].double().cpu().numpy(), ref.double().cpu().numpy(), "dense causal")
+
+
+@pytest.mark.parametrize("name", ["moba32k", "nsa64k", "nsa128k_planted"])
+def test_full_size_prefill_sampled_rows(name):
+    wl = WORKLOADS[name]
+    run = GpuRun(wl)
+    T = wl.seqlen_q
+    extra = [wl.sel_block - 1, wl.sel_block, wl.sel_block + 1, 511, 512, 513, T // 2, T - 2]
+    rows = row_sample(T, stride=max(1, T // 384), head=128, extra=extra)
+    compare_run(run, rows)
+    # every row of the selection: structural invariants
+    idx = run.idx[0]
+    t = torch.arange(T, device="cuda") + wl.q_pos0
+    c = (t // wl.sel_block).view(1, T, 1)
+    valid = idx >= 0
+    n = valid.sum(-1)
+    assert torch.equal(n, torch.clamp(c.view(1, T) + 1, max=wl.top_k).expand_as(n))
+    assert bool(((idx == c) & valid).any(-1).all())                   # current block kept
+    assert bool((idx < c + 1).all())                                   # causal blocks only
+    srt = torch.where(valid, idx, torch.full_like(idx, 1 << 30))
+    ascending = (srt[..., 1:] > srt[..., :-1]) | ~valid[..., 1:]
+    assert bool(ascending.all())                                       # ascending, no repeats
+
+
+def test_decode_sampled_sequences():
+    wl = WORKLOADS["decode64x64k"]
+    run = GpuRun(wl)
+    compare_run(run, [0], seqs=[0, 31, 63])
