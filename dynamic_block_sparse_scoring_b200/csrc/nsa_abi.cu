@@ -111,8 +111,9 @@ nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, floa
     Shape s;
     nsa_status st = make_shape(cfg, &s);
     if (st != NSA_OK) return st;
-    const bool need_sel = (cfg->flags & NSA_BR_SEL) != 0;
-    const bool need_cmp = (cfg->flags & NSA_BR_CMP) != 0;
+    // buffers of zero elements (no complete block / no compressed token) may be NULL
+    const bool need_sel = (cfg->flags & NSA_BR_SEL) != 0 && s.nb_full > 0;
+    const bool need_cmp = (cfg->flags & NSA_BR_CMP) != 0 && s.n_cmp > 0;
     if (!k || (need_sel && !kbar)) return NSA_ERR_INVALID_ARG;
     if (need_cmp && (!v || !kcmp || !vcmp)) return NSA_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(kcmp) || !aligned16(vcmp))
