@@ -41,8 +41,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # FP32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (max SM clock)
 ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-ATTN_KERNEL = "attn_rowwise_kernel"
-ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_scoring_b200", "csrc", "attn_rowwise.cu")
+ATTN_KERNEL = "attn_tc_kernel"
+ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_scoring_b200", "csrc", "attn_tc.cu")
 
 
 # ---------------------------------------------------------------------------
@@ -364,6 +364,8 @@ def run_ours(args):
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     wl = WORKLOADS[args.workload]
+    if args.seqlen:
+        wl = wl.with_(seqlen_q=args.seqlen, seqlen_kv=args.seqlen)
     pf = Prefill(wl, seed=rank)
     clocks = ClockSampler(torch.cuda.current_device())
     # warm-up and timed region (clocks sampled during it)
@@ -380,10 +382,11 @@ def run_ours(args):
     pk, src = peaks()
     attn_flops = (fl["total"] - fl["score"]) * wl.batch
     achieved = attn_flops / (attn_ms / 1e3) / 1e12
-    roof = {"kernel": ATTN_KERNEL, "bound": "alu", "achieved": achieved,
-            "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s", "frac": achieved / ALU_FP32_TFLOPS,
+    peak = pk["bf16_tflops"]
+    roof = {"kernel": ATTN_KERNEL, "bound": "tensor", "achieved": achieved,
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic_for(ATTN_KERNEL, ATTN_SOURCE),
-            "peak_source": "FP32 FFMA: 148 SMs x 128 lanes x 2 x 1.965 GHz",
+            "peak_source": f"{src} dense bf16 (burst, cuBLAS)",
             "flops_per_launch": attn_flops,
             "share_of_step": float(per[:, 2].mean() / step_ms.mean())}
     e2e = None
@@ -396,6 +399,9 @@ def run_ours(args):
     if rank == 0 and not args.no_cpu_baseline:
         x_cpu = {k: (v[:1].cpu() if v is not None else None) for k, v in pf.x.items()}
     launches = pf.launches_per_step * args.steps
+    dev_status = pf.abi.nsa_get_device_status()
+    if dev_status != 0:
+        raise SystemExit(f"device status {dev_status}: a kernel's bounded wait timed out")
     del pf
     torch.cuda.empty_cache()
     decode = None if args.no_decode else run_decode(world, args.steps, args.warmup)
@@ -461,6 +467,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=0, help="override the prefill length (profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)

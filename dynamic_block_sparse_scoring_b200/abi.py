@@ -53,6 +53,7 @@ _SIGS = {
     "nsa_score_blocks": [_cfgp, _vp, _vp, _vp, _vp],
     "nsa_topk_select": [_cfgp, _vp, _vp, _vp, _vp, _vp],
     "nsa_sparse_attn_fwd": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "nsa_get_device_status": [ctypes.POINTER(ctypes.c_int32)],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
@@ -97,6 +98,13 @@ def _check(fn: str, status: int):
 
 def nsa_status_string(status: int) -> str:
     return lib.nsa_status_string(status).decode()
+
+
+def nsa_get_device_status() -> int:
+    """Reads and clears the device status word (0 = OK, 5 = a bounded wait timed out)."""
+    v = ctypes.c_int32(0)
+    _check("nsa_get_device_status", lib.nsa_get_device_status(ctypes.byref(v)))
+    return v.value
 
 
 def nsa_workspace_size(cfg: NsaConfig) -> int:

@@ -82,4 +82,11 @@ cudaError_t launch_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloa
                         const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                         const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
                         __nv_bfloat16* out, cudaStream_t st);
+// tensor-core path (attn_tc.cu)
+bool attn_tc_supported(const Shape& s);
+cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                           const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
+                           const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
+                           __nv_bfloat16* out, cudaStream_t st);
+int read_and_clear_tc_status();
 }  // namespace nsa

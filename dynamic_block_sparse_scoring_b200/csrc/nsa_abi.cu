@@ -182,10 +182,21 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
         if (st != NSA_OK) return st;
     }
-    return cuda_status(nsa::launch_attn(
-        s, qb, static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        static_cast<const __nv_bfloat16*>(kcmp), static_cast<const __nv_bfloat16*>(vcmp), gates,
-        sel_idx, static_cast<__nv_bfloat16*>(out), cs));
+    // tensor-core kernel for the shapes it covers, the row-wise kernel otherwise
+    auto attn = nsa::attn_tc_supported(s) ? nsa::launch_attn_tc : nsa::launch_attn;
+    return cuda_status(attn(s, qb, static_cast<const __nv_bfloat16*>(k),
+                            static_cast<const __nv_bfloat16*>(v),
+                            static_cast<const __nv_bfloat16*>(kcmp),
+                            static_cast<const __nv_bfloat16*>(vcmp), gates, sel_idx,
+                            static_cast<__nv_bfloat16*>(out), cs));
+}
+
+nsa_status nsa_get_device_status(int32_t* status) {
+    if (!status) return NSA_ERR_INVALID_ARG;
+    const int v = nsa::read_and_clear_tc_status();
+    if (v < 0) return NSA_ERR_CUDA;
+    *status = v;
+    return NSA_OK;
 }
 
 }  // extern "C"

@@ -151,6 +151,14 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
                                const void* vcmp, const float* gates, const int32_t* idx,
                                void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Reads and clears the device-side status word of the tensor-core kernels:
+ * NSA_OK, or NSA_ERR_TIMEOUT when a bounded wait inside a kernel gave up (the
+ * kernel then unwound without finishing its output).  Synchronous: waits for
+ * all work on the current device first.  Not for use inside stream capture.
+ */
+nsa_status nsa_get_device_status(int32_t* status);
+
 /* Static, human-readable name of a status code. */
 const char* nsa_status_string(nsa_status status);
 

@@ -55,6 +55,7 @@ class GpuRun:
         self.out, _ = abi.forward(self.cfg, self.x["q"], self.x["k"], self.x["v"],
                                   self.x["gates"], pooled=self.pooled)
         torch.cuda.synchronize()
+        assert abi.nsa_get_device_status() == 0, "a kernel's bounded wait timed out"
 
     def oracle_rows(self, b: int, rows, idx=None):
         """Oracle (out, idx, gap) for sequence b and the given query rows."""
