@@ -53,6 +53,7 @@ _SIGS = {
     "nsa_score_blocks": [_cfgp, _vp, _vp, _vp, _vp],
     "nsa_topk_select": [_cfgp, _vp, _vp, _vp, _vp, _vp],
     "nsa_sparse_attn_fwd": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "nsa_sparse_attn_fwd_noalloc": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "nsa_get_device_status": [ctypes.POINTER(ctypes.c_int32)],
 }
 for _name, _args in _SIGS.items():
@@ -134,6 +135,14 @@ def nsa_sparse_attn_fwd(cfg, q, k, v, kbar, kcmp, vcmp, gates, idx, out, workspa
            lib.nsa_sparse_attn_fwd(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(kbar),
                                    _ptr(kcmp), _ptr(vcmp), _ptr(gates), _ptr(idx), _ptr(out),
                                    _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def nsa_sparse_attn_fwd_noalloc(cfg, q, k, v, kbar, kcmp, vcmp, gates, out, stream=None):
+    """Forward with internal selection and no workspace (the library's own scratch array)."""
+    _check("nsa_sparse_attn_fwd_noalloc",
+           lib.nsa_sparse_attn_fwd_noalloc(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(kbar), _ptr(kcmp), _ptr(vcmp), _ptr(gates),
+                                           _ptr(out), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

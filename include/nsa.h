@@ -152,6 +152,28 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
                                void* out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Same result as nsa_sparse_attn_fwd with idx == NULL (blocks selected
+ * inside), but it allocates nothing and takes no workspace: the block ids live
+ * in a 32 MiB array inside the library (a file-scope __device__ array that
+ * every GPU loading the library keeps until the process exits).  The pages
+ * describe no counterpart; this exists for callers that may not allocate
+ * device memory - plugin hosts whose execute call must not allocate because
+ * the host framework owns all device buffers, and latency-critical callers for
+ * which cudaMalloc/cudaFree are off limits because they can synchronise the
+ * device.
+ * Limit: problems with nsa_workspace_size() > 32 MiB return NSA_ERR_WORKSPACE
+ * (e.g. 65536 queries x 4 selection units x top-16 need 16 MiB).
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it.  Every call uses the same array, which keeps
+ * the previous call's contents (nothing in it needs to start at zero); calls
+ * whose GPU work overlaps race on it, so order them (e.g. one stream).
+ */
+nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, const void* k,
+                                       const void* v, const float* kbar, const void* kcmp,
+                                       const void* vcmp, const float* gates, void* out,
+                                       void* stream);
+
+/*
  * Reads and clears the device-side status word of the tensor-core kernels:
  * NSA_OK, or NSA_ERR_TIMEOUT when a bounded wait inside a kernel gave up (the
  * kernel then unwound without finishing its output).  Synchronous: waits for

@@ -1,0 +1,61 @@
+"""The allocation-free forward, nsa_sparse_attn_fwd_noalloc, against the regular
+entry point.
+
+Some callers may not allocate device memory at all (plugin hosts whose execute
+call must not allocate, latency-critical code that cannot afford cudaMalloc's
+device synchronisation), so they cannot provide the workspace that
+nsa_sparse_attn_fwd needs when it selects blocks itself.  The no-alloc variant
+keeps that scratch in a fixed array inside the library.  This file is named so
+that pytest collects it last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_scoring_b200 import abi
+from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+OUT_MAX_ABS = 2e-2
+OUT_MEAN_ABS = 2e-3
+
+
+def _forward_pair(wl, seed):
+    cfg = abi.config(wl)
+    x = make_inputs(wl, device="cuda", seed=seed)
+    pooled = abi.alloc_pooled(cfg, "cuda")
+    abi.nsa_pool_kv(cfg, x["k"], x["v"], pooled["kbar"], pooled["kcmp"], pooled["vcmp"])
+    ref, _ = abi.forward(cfg, x["q"], x["k"], x["v"], x["gates"], pooled=pooled)
+    got = torch.full_like(ref, float("nan"))
+    status = abi.lib.nsa_sparse_attn_fwd_noalloc(
+        ctypes.byref(cfg), x["q"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(),
+        pooled["kbar"].data_ptr(), pooled["kcmp"].data_ptr(), pooled["vcmp"].data_ptr(),
+        None if x["gates"] is None else x["gates"].data_ptr(), got.data_ptr(),
+        torch.cuda.current_stream().cuda_stream)
+    assert status == 0, abi.nsa_status_string(status)
+    torch.cuda.synchronize()
+    return ref.double().cpu().numpy(), got.double().cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["tiny", "nsa_small"])
+def test_noalloc_matches_regular_entry_point_twice_in_a_row(name):
+    wl = WORKLOADS["tiny"] if name == "tiny" else WORKLOADS["nsa64k"].with_(
+        name="nsa_small", seqlen_q=2048, seqlen_kv=2048, h_q=16, h_kv=1)
+    for seed in (0, 1):                  # two calls in a row on the shared scratch array
+        ref, got = _forward_pair(wl, seed)
+        assert np.isfinite(got).all()
+        err = np.abs(got - ref)
+        assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    # 131072 queries x 64 heads (per-head selection) x top-32 x 4 B = 1 GiB > 32 MiB
+    wl = WORKLOADS["nsa128k_planted"].with_(per_head_select=True, top_k=32)
+    cfg = abi.config(wl)
+    status = abi.lib.nsa_sparse_attn_fwd_noalloc(ctypes.byref(cfg), 1 << 20, 1 << 20, 1 << 20,
+                                                 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20,
+                                                 None)
+    assert status == 3                   # NSA_ERR_WORKSPACE, before anything is launched
