@@ -605,6 +605,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float mx[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+                if (hi < lo) lo = hi = SEG;    // empty: no offset 0..63 matches
                 const uint32_t span = (uint32_t)(hi - lo);
 #pragma unroll
                 for (int j = 0; j < SEG; ++j) {
