@@ -198,7 +198,18 @@ class Prefill:
                                device="cuda")
         self.out = torch.empty(wl.batch, wl.seqlen_q, wl.h_q, wl.d_v, dtype=torch.bfloat16,
                                device="cuda")
+        self.ws_bytes = abi.nsa_workspace_size(self.cfg)
+        self.ws = torch.empty(max(self.ws_bytes, 1), dtype=torch.uint8, device="cuda")
         self.launches_per_step = 0
+
+    def attn_launches(self) -> int:
+        """Kernels nsa_sparse_attn_fwd launches with an external idx: the block-major
+        selected branch adds the index build (count, scan, fill, items), its attention
+        kernel and the partial merge in front of the query-major kernel."""
+        wl = self.wl
+        minimal = self.abi.nsa_workspace_size_min(self.cfg)
+        block_major = (wl.branches & 2) and self.ws_bytes > minimal
+        return 7 if block_major else 1
 
     def step(self, ev=None, pool=True):
         a, x, p = self.abi, self.x, self.pooled
@@ -217,8 +228,9 @@ class Prefill:
         if ev:
             ev[2].record()
         a.nsa_sparse_attn_fwd(self.cfg, x["q"], x["k"], x["v"], p["kbar"], p["kcmp"], p["vcmp"],
-                              x["gates"], self.idx if self.wl.branches & 2 else None, self.out)
-        n += 1
+                              x["gates"], self.idx if self.wl.branches & 2 else None, self.out,
+                              self.ws, self.ws_bytes)
+        n += self.attn_launches()
         if ev:
             ev[3].record()
         self.launches_per_step = n
@@ -267,8 +279,8 @@ def e2e_steps(pf: Prefill, steps: int, warmup: int, world: int):
     dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_h.numel() * out_h.element_size()
-    ws = a.nsa_workspace_size(pf.cfg)
-    work = torch.empty(ws, dtype=torch.uint8, device="cuda")
+    ws = pf.ws_bytes
+    work = pf.ws
 
     def one():
         for k in host:

@@ -42,6 +42,8 @@ class NsaError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
         msg = lib.nsa_status_string(status).decode()
+        if status == 4:
+            msg += ": " + lib.nsa_last_cuda_error().decode()
         super().__init__(f"{fn} returned {status} ({msg})")
 
 
@@ -49,6 +51,7 @@ _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
 _cfgp = ctypes.POINTER(NsaConfig)
 _SIGS = {
     "nsa_workspace_size": [_cfgp, ctypes.POINTER(_sz)],
+    "nsa_workspace_size_min": [_cfgp, ctypes.POINTER(_sz)],
     "nsa_pool_kv": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp],
     "nsa_score_blocks": [_cfgp, _vp, _vp, _vp, _vp],
     "nsa_topk_select": [_cfgp, _vp, _vp, _vp, _vp, _vp],
@@ -62,8 +65,10 @@ for _name, _args in _SIGS.items():
     _f.restype = ctypes.c_int
 lib.nsa_status_string.argtypes = [ctypes.c_int]
 lib.nsa_status_string.restype = ctypes.c_char_p
+lib.nsa_last_cuda_error.argtypes = []
+lib.nsa_last_cuda_error.restype = ctypes.c_char_p
 
-EXPORTS = list(_SIGS) + ["nsa_status_string"]
+EXPORTS = list(_SIGS) + ["nsa_status_string", "nsa_last_cuda_error"]
 
 
 def config(wl: Workload, **override) -> NsaConfig:
@@ -111,6 +116,12 @@ def nsa_get_device_status() -> int:
 def nsa_workspace_size(cfg: NsaConfig) -> int:
     n = _sz(0)
     _check("nsa_workspace_size", lib.nsa_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def nsa_workspace_size_min(cfg: NsaConfig) -> int:
+    n = _sz(0)
+    _check("nsa_workspace_size_min", lib.nsa_workspace_size_min(ctypes.byref(cfg), ctypes.byref(n)))
     return n.value
 
 
@@ -183,9 +194,11 @@ def forward(cfg: NsaConfig, q, k, v, gates=None, idx=None, stream=None, pooled=N
     if out is None:
         out = torch.empty(cfg.batch, cfg.seqlen_q, cfg.h_q, cfg.d_v, dtype=torch.bfloat16,
                           device=dev)
-    ws = nsa_workspace_size(cfg) if idx is None else 0
-    if ws and workspace is None:
-        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    ws = nsa_workspace_size(cfg)
+    if workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
+    else:
+        ws = workspace.numel() * workspace.element_size()
     nsa_sparse_attn_fwd(cfg, q, k, v, pooled["kbar"], pooled["kcmp"], pooled["vcmp"], gates, idx,
                         out, workspace, ws, stream)
     return out, pooled

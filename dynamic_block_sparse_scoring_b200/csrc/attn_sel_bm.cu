@@ -1,0 +1,539 @@
+// Selected-branch attention, block-major, on tcgen05: one KV block against
+// every query that kept it.
+//
+// Zhang Xiaojun #94 transcript (bidclub.ai), §7 "Kimi Simplifies The Sparse
+// Route": MoBA gathers, for each KV block, the queries that chose it into a
+// contiguous batch and runs dense attention on it; §4 "Inside Native Sparse
+// Attention": the selected branch attends over every token of the kept
+// blocks.  With random selections neighbouring tokens rarely share blocks, so
+// a query-major tile would either re-read each block per query or compute
+// over the union of its tokens' blocks; block-major loads each 64-key block
+// once per work item of up to 128/HPT queries.
+//
+// A work item is (sequence, selection unit, block j, up to TOK queries from
+// the block's list).  Its 128 rows are the TOK queries x HPT heads, gathered
+// by TMA (one 4D box per query).  S = Q K_j^T (M=128, N=64) and O = P V_j
+// (M=128, N=d_v) run on tcgen05; the block is fully visible except for the
+// query's own block, where key u is visible iff u <= t.  Each row writes a
+// partial result for its (query, slot): o = (P V)/l in bf16 and
+// lse = m + log2(l) in the scaled-log2 domain.  The partials of a query's
+// slots are merged by sel_merge.cu.  Items come chunk by chunk (4096
+// queries); every CTA takes a contiguous share of each chunk, so the chunk's
+// queries stay in L2 while consecutive items of a CTA share their K/V block.
+//
+// Roles (320 threads): warp 0 TMA producer (K/V once per run of items on the
+// same block, Q rows per item), warp 1 MMA lane + TMEM owner, warps 2-5 and
+// 6-9 two softmax/epilogue warpgroups that take alternate items (each with
+// its own S and O in TMEM), so consecutive items overlap.  All waits are
+// bounded; a timeout records NSA_ERR_TIMEOUT in g_bm_status and unwinds.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "sel_index.cuh"
+#include "tc.cuh"
+
+namespace nsa {
+
+__device__ int g_bm_status = 0;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BLK = 64;             // keys per block (the path requires sel_block == 64)
+constexpr int NTHREADS = 320;
+constexpr int NM = 8;               // item descriptors in flight
+constexpr int CHUNK_Q = 16384;      // 128 rows x 64 columns bf16
+constexpr int CHUNK_KV = 8192;      // 64 rows x 64 columns bf16
+constexpr uint64_t WAIT_NS = 1000000000ull;
+constexpr int MAX_TOK = 16;
+
+struct ItemMeta {
+    int valid;          // 0 = end of the stream
+    int lidx;           // list id = (chunk * B * Hsel + b * Hsel + u) * nb_all + j
+    int n;              // queries in the item
+    int kvs;            // K/V stage holding block j
+    int new_block;      // first item on this K/V stage load
+    int last_of_block;  // last item using this K/V stage load
+    int pad[2];
+    int tok[MAX_TOK];   // query * 32 + slot
+};
+
+struct BmArgs {
+    Shape s;
+    const int4* items;
+    const int32_t* item_off;  // [lists + 1] first item of each list (chunk boundaries)
+    const int32_t* list;
+    __nv_bfloat16* part_o;    // [B, Hsel, Tq, topk, hpt, d_v]
+    float* part_lse;          // [B, Hsel, Tq, topk, hpt]
+    int hpt, tok;
+    int n_chunks;
+    int lists_per_chunk;
+    float scale_log2;
+};
+
+template <int DQK, int DV>
+struct BmSmem {
+    static constexpr int QC = DQK / 64, VC = DV / 64;
+    static constexpr int Q_OFF = 0;                                  // 2 stages
+    static constexpr int K_OFF = Q_OFF + 2 * QC * CHUNK_Q;            // 2 stages
+    static constexpr int V_OFF = K_OFF + 2 * QC * CHUNK_KV;           // 2 stages
+    static constexpr int META_OFF = V_OFF + 2 * VC * CHUNK_KV;
+    static constexpr int BAR_OFF = META_OFF + NM * (int)sizeof(ItemMeta);
+    // q_full[2] q_empty[2] kv_full[2] kv_empty[2] meta_full[NM] meta_empty[NM]
+    // s_full[2] p_full[2] o_full[2] o_free[2] drain
+    static constexpr int NBAR = 8 + 2 * NM + 8 + 1;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int ALLOC = MISC_OFF + 64 + 1024;
+};
+
+struct BmBars {
+    uint64_t* b;
+    __device__ __forceinline__ uint64_t* q_full(int i) const { return b + i; }
+    __device__ __forceinline__ uint64_t* q_empty(int i) const { return b + 2 + i; }
+    __device__ __forceinline__ uint64_t* kv_full(int i) const { return b + 4 + i; }
+    __device__ __forceinline__ uint64_t* kv_empty(int i) const { return b + 6 + i; }
+    __device__ __forceinline__ uint64_t* meta_full(int i) const { return b + 8 + i; }
+    __device__ __forceinline__ uint64_t* meta_empty(int i) const { return b + 8 + NM + i; }
+    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 8 + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* p_full(int i) const { return b + 10 + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* o_full(int i) const { return b + 12 + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* o_free(int i) const { return b + 14 + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* drain() const { return b + 16 + 2 * NM; }
+};
+
+__device__ __forceinline__ bool bm_warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, abort_flag, WAIT_NS));
+}
+
+__device__ __forceinline__ void bm_abort(volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicExch(&g_bm_status, (int)NSA_ERR_TIMEOUT);
+}
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    sel_bm_kernel(const __grid_constant__ CUtensorMap map_qg, const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_v, const BmArgs a) {
+    using L = BmSmem<DQK, DV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    BmBars bar{reinterpret_cast<uint64_t*>(sm + L::BAR_OFF)};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC_OFF + 8);
+    ItemMeta* metas = reinterpret_cast<ItemMeta*>(sm + L::META_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bar.q_full(i), 1);
+            tc::mbar_init(bar.q_empty(i), 1);
+            tc::mbar_init(bar.kv_full(i), 1);
+            tc::mbar_init(bar.kv_empty(i), 1);
+            tc::mbar_init(bar.s_full(i), 1);
+            tc::mbar_init(bar.p_full(i), 4);
+            tc::mbar_init(bar.o_full(i), 1);
+            tc::mbar_init(bar.o_free(i), 4);
+        }
+        for (int i = 0; i < NM; ++i) {
+            tc::mbar_init(bar.meta_full(i), 1);
+            tc::mbar_init(bar.meta_empty(i), 5);   // MMA lane + the owning warpgroup's 4 warps
+        }
+        tc::mbar_init(bar.drain(), 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    // S0 [0,64) S1 [64,128) O0 [128,128+DV) O1 [256,256+DV)
+    auto tS = [&](int i) { return tmem + 64 * i; };
+    auto tO = [&](int i) { return tmem + 128 + 128 * i; };
+
+    const int nb_all = a.s.nb_all;
+    const int bhsel = a.s.B * a.s.Hsel;
+    // This CTA's share of chunk c's items: a contiguous range, so that
+    // consecutive items mostly stay on one block (K/V loaded once for them),
+    // while all CTAs advance through the chunks together.
+    auto chunk_range = [&](int c, int& lo, int& hi) {
+        const int c0 = a.item_off[(size_t)c * a.lists_per_chunk];
+        const int c1 = a.item_off[(size_t)(c + 1) * a.lists_per_chunk];
+        const int per = (c1 - c0 + gridDim.x - 1) / gridDim.x;
+        lo = min(c1, c0 + (int)blockIdx.x * per);
+        hi = min(c1, lo + per);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        bool ok = true;
+        uint32_t kv_loads = 0, q_loads = 0;
+        int prev_lidx = -1, kvs = 0;
+        int chunk = 0, i = 0, i_end = 0, li = 0, ends = 0;
+        chunk_range(0, i, i_end);
+        while (ok && ends < 2) {
+            while (i >= i_end && chunk + 1 < a.n_chunks) chunk_range(++chunk, i, i_end);
+            ItemMeta m;
+            m.valid = i < i_end;
+            m.lidx = m.n = m.kvs = m.new_block = m.last_of_block = 0;
+            if (m.valid) {
+                const int4 it = a.items[i];
+                m.lidx = it.x;
+                m.n = it.z;
+                m.new_block = it.x != prev_lidx;
+                // the next item this CTA will take (possibly in a later chunk)
+                int nxt = i + 1, nxt_end = i_end, nchunk = chunk;
+                while (nxt >= nxt_end && nchunk + 1 < a.n_chunks) chunk_range(++nchunk, nxt, nxt_end);
+                m.last_of_block = nxt >= nxt_end || a.items[nxt].x != it.x;
+                const int bu = (it.x / nb_all) % bhsel, j = it.x % nb_all;
+                const int b = bu / a.s.Hsel, u = bu % a.s.Hsel;
+                const int kvh = a.s.per_head ? u / a.s.G : u;
+                const int h0 = a.s.per_head ? u : u * a.s.G;
+                if (m.new_block) {
+                    kvs = kv_loads & 1;
+                    if (!bm_warp_wait(bar.kv_empty(kvs), ((kv_loads >> 1) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        tc::mbar_arrive_expect_tx(bar.kv_full(kvs), (L::QC + L::VC) * CHUNK_KV);
+                        const int plane = b * a.s.Hkv + kvh;
+                        for (int c = 0; c < L::QC; ++c)
+                            tc::tma_load_3d(sm + L::K_OFF + (kvs * L::QC + c) * CHUNK_KV, &map_k,
+                                            bar.kv_full(kvs), 64 * c, j * BLK, plane);
+                        for (int c = 0; c < L::VC; ++c)
+                            tc::tma_load_3d(sm + L::V_OFF + (kvs * L::VC + c) * CHUNK_KV, &map_v,
+                                            bar.kv_full(kvs), 64 * c, j * BLK, plane);
+                    }
+                    ++kv_loads;
+                    prev_lidx = it.x;
+                }
+                m.kvs = kvs;
+                const int tokv = lane < m.n ? a.list[it.y + lane] : 0;
+                for (int tt = 0; tt < MAX_TOK; ++tt) m.tok[tt] = __shfl_sync(0xffffffffu, tokv, tt);
+                const int qs = li & 1;
+                if (!bm_warp_wait(bar.q_empty(qs), ((li >> 1) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
+                    for (int tt = 0; tt < m.n; ++tt)
+                        for (int c = 0; c < L::QC; ++c)
+                            tc::tma_load_4d(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
+                                            &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b);
+                }
+                ++q_loads;
+                ++i;
+            } else {
+                ++ends;    // two end markers, one for each softmax warpgroup
+            }
+            const int slot = li % NM;
+            if (!bm_warp_wait(bar.meta_empty(slot), ((li / NM) & 1) ^ 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                metas[slot] = m;
+                tc::mbar_arrive(bar.meta_full(slot));
+            }
+            ++li;
+        }
+        if (!ok) bm_abort(abort_flag);
+        // wait for every copy still in flight before the CTA may exit
+        volatile int never = 0;
+        for (uint32_t s = 0; s < 2; ++s) {
+            if (kv_loads > s) {
+                const uint32_t last = s + ((kv_loads - 1 - s) / 2) * 2;
+                tc::mbar_wait(bar.kv_full(s), (last >> 1) & 1, &never, WAIT_NS);
+            }
+            if (q_loads > s) {
+                const uint32_t last = s + ((q_loads - 1 - s) / 2) * 2;
+                tc::mbar_wait(bar.q_full(s), (last >> 1) & 1, &never, WAIT_NS);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            const uint32_t idesc_qk = tc::idesc_bf16_f32(BM, BLK, false, false);
+            const uint32_t idesc_pv = tc::idesc_bf16_f32(BM, DV, false, true);
+            const uint32_t q_base = tc::smem_u32(sm + L::Q_OFF);
+            const uint32_t k_base = tc::smem_u32(sm + L::K_OFF);
+            const uint32_t v_base = tc::smem_u32(sm + L::V_OFF);
+            bool ok = true, have_prev = false;
+            int prev_li = 0, prev_kvs = 0, prev_last = 0;
+            uint32_t kv_seen = 0;
+            auto issue_pv = [&](int li, int kvs, int last) -> bool {
+                const int sb = li & 1;
+                if (!tc::mbar_wait(bar.p_full(sb), (li >> 1) & 1, abort_flag, WAIT_NS) ||
+                    !tc::mbar_wait(bar.o_free(sb), ((li >> 1) & 1) ^ 1, abort_flag, WAIT_NS))
+                    return false;
+                tc::fence_after_sync();
+                const uint32_t vst = v_base + kvs * L::VC * CHUNK_KV;
+#pragma unroll
+                for (int kk = 0; kk < BLK / 16; ++kk)
+                    tc::mma_ts(tO(sb), tS(sb) + kk * 8, tc::sdesc_sw128(vst + kk * 2048, CHUNK_KV, 1024),
+                               idesc_pv, kk > 0);
+                tc::mma_commit(bar.o_full(sb));
+                if (last) tc::mma_commit(bar.kv_empty(kvs));
+                return true;
+            };
+            for (int li = 0; ok; ++li) {
+                const int slot = li % NM;
+                if (!tc::mbar_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag, WAIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                const ItemMeta& m = metas[slot];
+                const int valid = m.valid, kvs = m.kvs, new_block = m.new_block, last = m.last_of_block;
+                tc::mbar_arrive(bar.meta_empty(slot));
+                if (!valid) {
+                    if (have_prev && !issue_pv(prev_li, prev_kvs, prev_last)) ok = false;
+                    break;
+                }
+                const int qs = li & 1;
+                if (!tc::mbar_wait(bar.q_full(qs), (li >> 1) & 1, abort_flag, WAIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                if (new_block) {
+                    if (!tc::mbar_wait(bar.kv_full(kvs), (kv_seen >> 1) & 1, abort_flag, WAIT_NS)) {
+                        ok = false;
+                        break;
+                    }
+                    ++kv_seen;
+                }
+                tc::fence_after_sync();
+                const uint32_t qst = q_base + qs * L::QC * CHUNK_Q;
+                const uint32_t kst = k_base + kvs * L::QC * CHUNK_KV;
+#pragma unroll
+                for (int kk = 0; kk < DQK / 16; ++kk) {
+                    tc::mma_ss(tS(li & 1),
+                               tc::sdesc_sw128(qst + (kk >> 2) * CHUNK_Q + (kk & 3) * 32, 16, 1024),
+                               tc::sdesc_sw128(kst + (kk >> 2) * CHUNK_KV + (kk & 3) * 32, 16, 1024),
+                               idesc_qk, kk > 0);
+                }
+                tc::mma_commit(bar.s_full(li & 1));
+                tc::mma_commit(bar.q_empty(qs));
+                if (have_prev && !issue_pv(prev_li, prev_kvs, prev_last)) {
+                    ok = false;
+                    break;
+                }
+                have_prev = true;
+                prev_li = li;
+                prev_kvs = kvs;
+                prev_last = last;
+            }
+            if (!ok) bm_abort(abort_flag);
+            volatile int never = 0;
+            tc::mma_commit(bar.drain());
+            tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int wg = (warp - 2) >> 2;                  // takes items li with li % 2 == wg
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int tt = r / a.hpt, hl = r % a.hpt;
+        bool ok = true;
+        for (int li = wg; ok; li += 2) {
+            const int slot = li % NM;
+            if (!bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const ItemMeta& mref = metas[slot];
+            const int valid = mref.valid, lidx = mref.lidx, n = mref.n;
+            const int tokr = tt < MAX_TOK ? mref.tok[tt] : 0;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
+            if (!valid) break;
+            const bool row_valid = tt < n;
+            const int bu = (lidx / nb_all) % bhsel, j = lidx % nb_all;
+            const int qi = tokr >> 5, sl = tokr & 31;
+            const int t = a.s.q0 + qi;
+            const int sb = li & 1;
+            if (!bm_warp_wait(bar.s_full(sb), (li >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            uint32_t sv[BLK];
+            tc::tmem_ld32(tS(sb) + lane_off, sv);
+            tc::tmem_ld32(tS(sb) + lane_off + 32, sv + 32);
+            tc::tmem_wait_ld();
+            // visible offsets: the whole block, or u <= t inside the query's own block
+            const int hi = row_valid ? min(BLK - 1, t - j * BLK) : -1;
+            float mx[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < BLK; ++k) {
+                const float x = k <= hi ? __uint_as_float(sv[k]) : -INFINITY;
+                sv[k] = __float_as_uint(x);
+                mx[k & 7] = fmaxf(mx[k & 7], x);
+            }
+            const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m = m_raw == -INFINITY ? 0.f : m_raw * a.scale_log2;
+            float ps[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+#pragma unroll
+            for (int k = 0; k < BLK; k += 2) {
+                const float p0 = tc::ex2(fmaf(__uint_as_float(sv[k]), a.scale_log2, -m));
+                const float p1 = tc::ex2(fmaf(__uint_as_float(sv[k + 1]), a.scale_log2, -m));
+                ps[(k >> 1) & 7] += p0 + p1;
+                sv[k >> 1] = tc::pack_bf16x2(p0, p1);
+            }
+            const float l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            tc::tmem_st32(tS(sb) + lane_off, sv);
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
+
+            // epilogue: o = (P V) / l -> bf16 partial, lse = m + log2(l)
+            if (!bm_warp_wait(bar.o_full(sb), (li >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t prow = (((size_t)bu * a.s.Tq + qi) * a.s.topk + sl) * a.hpt + hl;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+                uint32_t o[32];
+                tc::tmem_ld32(tO(sb) + lane_off + c, o);
+                tc::tmem_wait_ld();
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(a.part_o + prow * DV + c);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 u4;
+                        u4.x = tc::pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+                        u4.y = tc::pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+                        u4.z = tc::pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+                        u4.w = tc::pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+                        dst[q] = u4;
+                    }
+                }
+            }
+            if (row_valid) a.part_lse[prow] = m + __log2f(l);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar.o_free(sb));
+        }
+        if (!ok) bm_abort(abort_flag);
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 bm_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box) {
+    auto enc = bm_encode_fn();
+    if (!enc) return false;
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DQK, int DV>
+cudaError_t launch_bm_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                           const __nv_bfloat16* v, const SelIndex& x, __nv_bfloat16* part_o,
+                           float* part_lse, cudaStream_t st) {
+    BmArgs a;
+    a.s = s;
+    a.items = x.items;
+    a.item_off = x.item_off;
+    a.n_chunks = sel_chunks(s);
+    a.lists_per_chunk = (int)sel_lists_per_chunk(s);
+    a.list = x.list;
+    a.part_o = part_o;
+    a.part_lse = part_lse;
+    a.hpt = s.heads_per_unit;
+    a.tok = BM / a.hpt;
+    a.scale_log2 = s.scale * 1.4426950408889634f;
+    CUtensorMap mq, mk, mv;
+    const cuuint64_t qd[4] = {(cuuint64_t)DQK, (cuuint64_t)s.Hq, (cuuint64_t)s.Tq, (cuuint64_t)s.B};
+    const cuuint64_t qs[3] = {(cuuint64_t)DQK * 2, (cuuint64_t)DQK * 2 * s.Hq,
+                              (cuuint64_t)DQK * 2 * s.Hq * s.Tq};
+    const cuuint32_t qb[4] = {64, (cuuint32_t)a.hpt, 1, 1};
+    const cuuint64_t kd[3] = {(cuuint64_t)DQK, (cuuint64_t)s.Tk, (cuuint64_t)s.B * s.Hkv};
+    const cuuint64_t ks[2] = {(cuuint64_t)DQK * 2, (cuuint64_t)DQK * 2 * s.Tk};
+    const cuuint64_t vd[3] = {(cuuint64_t)DV, (cuuint64_t)s.Tk, (cuuint64_t)s.B * s.Hkv};
+    const cuuint64_t vs[2] = {(cuuint64_t)DV * 2, (cuuint64_t)DV * 2 * s.Tk};
+    const cuuint32_t kb[3] = {64, (cuuint32_t)BLK, 1};
+    if (!encode(&mq, q, 4, qd, qs, qb) || !encode(&mk, k, 3, kd, ks, kb) ||
+        !encode(&mv, v, 3, vd, vs, kb))
+        return cudaErrorInvalidValue;
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int smem = BmSmem<DQK, DV>::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(sel_bm_kernel<DQK, DV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    sel_bm_kernel<DQK, DV><<<nsm, NTHREADS, smem, st>>>(mq, mk, mv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sel_bm_supported(const Shape& s) {
+    if (!(s.flags & NSA_BR_SEL)) return false;
+    if (s.dqk != 64 && s.dqk != 128 && s.dqk != 192) return false;
+    if (s.dv != 64 && s.dv != 128) return false;
+    if (s.bs != BLK) return false;
+    const int hpt = s.heads_per_unit;
+    return (hpt == 8 || hpt == 16) && s.topk <= 32;
+}
+
+cudaError_t launch_sel_bm(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                          const __nv_bfloat16* v, const SelIndex& x, __nv_bfloat16* part_o,
+                          float* part_lse, cudaStream_t st) {
+#define NSA_BM_CASE(A, B) \
+    if (s.dqk == A && s.dv == B) return launch_bm_impl<A, B>(s, q, k, v, x, part_o, part_lse, st);
+    NSA_BM_CASE(64, 64)
+    NSA_BM_CASE(128, 128)
+    NSA_BM_CASE(192, 128)
+    NSA_BM_CASE(64, 128)
+    NSA_BM_CASE(128, 64)
+    NSA_BM_CASE(192, 64)
+#undef NSA_BM_CASE
+    return cudaErrorInvalidValue;
+}
+
+int read_and_clear_bm_status() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_bm_status, sizeof(int)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_bm_status, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace nsa

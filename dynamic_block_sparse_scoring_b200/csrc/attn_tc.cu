@@ -74,6 +74,10 @@ struct TcArgs {
     int n_tt;             // token tiles per (sequence, unit)
     int n_work;           // total work tiles
     float scale_log2;     // scale * log2(e)
+    // selected branch computed block-major and merged: o_sel [B, Tq, Hq, d_v]
+    // bf16 (ungated); null = the selected branch runs here over the union of
+    // the tile's block sets
+    const __nv_bfloat16* o_sel;
 };
 
 template <int DQK, int DV>
@@ -95,35 +99,27 @@ struct Smem {
     static constexpr int ALLOC = BYTES + 1024;   // slack to align the base to 1024 B
 };
 
+// All barriers live at one shared-memory base; each accessor is a constant
+// offset from it, so a role keeps one pointer live instead of twelve.
 struct Bars {
-    uint64_t* q_full;
-    uint64_t* q_empty;
-    uint64_t* k_full;
-    uint64_t* k_empty;
-    uint64_t* v_full;
-    uint64_t* v_empty;
-    uint64_t* meta_full;
-    uint64_t* meta_empty;
-    uint64_t* s_full;
-    uint64_t* p_full;
-    uint64_t* pv_done;
-    uint64_t* drain;
+    uint64_t* b;
+    __device__ __forceinline__ uint64_t* q_full() const { return b; }
+    __device__ __forceinline__ uint64_t* q_empty() const { return b + 1; }
+    __device__ __forceinline__ uint64_t* k_full(int i) const { return b + 2 + i; }
+    __device__ __forceinline__ uint64_t* k_empty(int i) const { return b + 2 + NS + i; }
+    __device__ __forceinline__ uint64_t* v_full(int i) const { return b + 2 + 2 * NS + i; }
+    __device__ __forceinline__ uint64_t* v_empty(int i) const { return b + 2 + 3 * NS + i; }
+    __device__ __forceinline__ uint64_t* meta_full(int i) const { return b + 2 + 4 * NS + i; }
+    __device__ __forceinline__ uint64_t* meta_empty(int i) const { return b + 2 + 4 * NS + NM + i; }
+    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 2 + 4 * NS + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* p_full(int i) const { return b + 4 + 4 * NS + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* pv_done() const { return b + 6 + 4 * NS + 2 * NM; }
+    __device__ __forceinline__ uint64_t* drain() const { return b + 7 + 4 * NS + 2 * NM; }
 };
 
 __device__ __forceinline__ Bars make_bars(uint64_t* b) {
     Bars r;
-    r.q_full = b;
-    r.q_empty = b + 1;
-    r.k_full = b + 2;
-    r.k_empty = r.k_full + NS;
-    r.v_full = r.k_empty + NS;
-    r.v_empty = r.v_full + NS;
-    r.meta_full = r.v_empty + NS;
-    r.meta_empty = r.meta_full + NM;
-    r.s_full = r.meta_empty + NM;
-    r.p_full = r.s_full + 2;
-    r.pv_done = r.p_full + 2;
-    r.drain = r.pv_done + 1;
+    r.b = b;
     return r;
 }
 
@@ -181,10 +177,10 @@ struct Producer {
 
     __device__ bool emit(const KeyTile& kt, const WorkTile& w) {
         const int slot = gm % NM;
-        if (!warp_wait(&bar.meta_empty[slot], ((gm / NM) & 1) ^ 1, abort_flag)) return false;
+        if (!warp_wait(bar.meta_empty(slot), ((gm / NM) & 1) ^ 1, abort_flag)) return false;
         if (lane == 0) {
             reinterpret_cast<KeyTile*>(sm + L::META_OFF)[slot] = kt;
-            tc::mbar_arrive(&bar.meta_full[slot]);
+            tc::mbar_arrive(bar.meta_full(slot));
         }
         ++gm;
         if (kt.br == BR_END) return true;
@@ -195,25 +191,25 @@ struct Producer {
         const CUtensorMap* V = cmp ? mvc : mv;
         const int rows = cmp ? a.s.n_cmp : a.s.Tk;     // a segment at `rows` is fully out of
         const int plane = w.b * a.s.Hkv + w.kvh;       // bounds: TMA fills it with zeros
-        if (!warp_wait(&bar.k_empty[st], ph, abort_flag)) return false;
+        if (!warp_wait(bar.k_empty(st), ph, abort_flag)) return false;
         if (lane == 0) {
-            tc::mbar_arrive_expect_tx(&bar.k_full[st], 2 * L::QC * HALF);
+            tc::mbar_arrive_expect_tx(bar.k_full(st), 2 * L::QC * HALF);
             uint8_t* dst = sm + L::K_OFF + st * L::QC * CHUNK;
             for (int sg = 0; sg < 2; ++sg) {
                 const int row = kt.seg[sg] >= 0 ? kt.seg[sg] : rows;
                 for (int c = 0; c < L::QC; ++c)
-                    tc::tma_load_3d(dst + c * CHUNK + sg * HALF, K, &bar.k_full[st], 64 * c, row,
+                    tc::tma_load_3d(dst + c * CHUNK + sg * HALF, K, bar.k_full(st), 64 * c, row,
                                     plane);
             }
         }
-        if (!warp_wait(&bar.v_empty[st], ph, abort_flag)) return false;
+        if (!warp_wait(bar.v_empty(st), ph, abort_flag)) return false;
         if (lane == 0) {
-            tc::mbar_arrive_expect_tx(&bar.v_full[st], 2 * L::VC * HALF);
+            tc::mbar_arrive_expect_tx(bar.v_full(st), 2 * L::VC * HALF);
             uint8_t* dst = sm + L::V_OFF + st * L::VC * CHUNK;
             for (int sg = 0; sg < 2; ++sg) {
                 const int row = kt.seg[sg] >= 0 ? kt.seg[sg] : rows;
                 for (int c = 0; c < L::VC; ++c)
-                    tc::tma_load_3d(dst + c * CHUNK + sg * HALF, V, &bar.v_full[st], 64 * c, row,
+                    tc::tma_load_3d(dst + c * CHUNK + sg * HALF, V, bar.v_full(st), 64 * c, row,
                                     plane);
             }
         }
@@ -289,11 +285,14 @@ struct Producer {
         for (int work = cta; work < a.n_work; work += ncta, ++wt) {
             const WorkTile w = decode_work(a, work);
             const int t_last = w.t0 + w.ntok - 1;
-            if (!warp_wait(bar.q_empty, (wt & 1) ^ 1, abort_flag)) return false;
+            // the selected blocks' union first: the sort overlaps the pipeline drain
+            const bool sel_here = (a.s.flags & NSA_BR_SEL) && a.o_sel == nullptr;
+            const int nu = sel_here ? build_union(w, keys, members) : 0;
+            if (!warp_wait(bar.q_empty(), (wt & 1) ^ 1, abort_flag)) return false;
             if (lane == 0) {
-                tc::mbar_arrive_expect_tx(bar.q_full, L::QC * CHUNK);
+                tc::mbar_arrive_expect_tx(bar.q_full(), L::QC * CHUNK);
                 for (int c = 0; c < L::QC; ++c)
-                    tc::tma_load_4d(sm + L::Q_OFF + c * CHUNK, mq, bar.q_full, 64 * c, w.h0,
+                    tc::tma_load_4d(sm + L::Q_OFF + c * CHUNK, mq, bar.q_full(), 64 * c, w.h0,
                                     w.tt * a.tok, w.b);
             }
             ++q_loads;
@@ -311,8 +310,7 @@ struct Producer {
                     if (!emit(kt, w)) return false;
                 }
             }
-            if (a.s.flags & NSA_BR_SEL) {
-                const int nu = build_union(w, keys, members);
+            if (sel_here) {
                 const int segs_per_blk = a.s.bs / SEG;
                 const int nseg = nu * segs_per_blk;
                 for (int sgi = 0; sgi < nseg; sgi += 2) {
@@ -357,10 +355,10 @@ struct Producer {
         for (uint32_t s = 0; s < NS && s < gk; ++s) {
             const uint32_t last = s + ((gk - 1 - s) / NS) * NS;   // last key tile on stage s
             const uint32_t ph = (last / NS) & 1;
-            tc::mbar_wait(&bar.k_full[s], ph, &never, WAIT_NS);
-            tc::mbar_wait(&bar.v_full[s], ph, &never, WAIT_NS);
+            tc::mbar_wait(bar.k_full(s), ph, &never, WAIT_NS);
+            tc::mbar_wait(bar.v_full(s), ph, &never, WAIT_NS);
         }
-        if (q_loads > 0) tc::mbar_wait(bar.q_full, (q_loads - 1) & 1, &never, WAIT_NS);
+        if (q_loads > 0) tc::mbar_wait(bar.q_full(), (q_loads - 1) & 1, &never, WAIT_NS);
     }
 };
 
@@ -383,24 +381,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(bar.q_full, 1);
-        tc::mbar_init(bar.q_empty, 1);
+        tc::mbar_init(bar.q_full(), 1);
+        tc::mbar_init(bar.q_empty(), 1);
         for (int i = 0; i < NS; ++i) {
-            tc::mbar_init(&bar.k_full[i], 1);
-            tc::mbar_init(&bar.k_empty[i], 1);
-            tc::mbar_init(&bar.v_full[i], 1);
-            tc::mbar_init(&bar.v_empty[i], 1);
+            tc::mbar_init(bar.k_full(i), 1);
+            tc::mbar_init(bar.k_empty(i), 1);
+            tc::mbar_init(bar.v_full(i), 1);
+            tc::mbar_init(bar.v_empty(i), 1);
         }
         for (int i = 0; i < NM; ++i) {
-            tc::mbar_init(&bar.meta_full[i], 1);
-            tc::mbar_init(&bar.meta_empty[i], 9);   // MMA lane + 8 softmax warps
+            tc::mbar_init(bar.meta_full(i), 1);
+            tc::mbar_init(bar.meta_empty(i), 9);   // MMA lane + 8 softmax warps
         }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&bar.s_full[i], 1);
-            tc::mbar_init(&bar.p_full[i], 8);       // 8 softmax warps
+            tc::mbar_init(bar.s_full(i), 1);
+            tc::mbar_init(bar.p_full(i), 8);       // 8 softmax warps
         }
-        tc::mbar_init(bar.pv_done, 1);
-        tc::mbar_init(bar.drain, 1);
+        tc::mbar_init(bar.pv_done(), 1);
+        tc::mbar_init(bar.drain(), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -438,23 +436,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t gm = 0, gi = 0, wt = 0;
             bool ok = true;
             for (int work = blockIdx.x; ok && work < a.n_work; work += gridDim.x, ++wt) {
-                if (!tc::mbar_wait(bar.q_full, wt & 1, abort_flag, WAIT_NS)) { ok = false; break; }
+                if (!tc::mbar_wait(bar.q_full(), wt & 1, abort_flag, WAIT_NS)) { ok = false; break; }
                 bool have_prev = false;
                 uint32_t prev_gi = 0;
                 int prev_first = 0;
                 while (true) {
                     const int slot = gm % NM;
-                    if (!tc::mbar_wait(&bar.meta_full[slot], (gm / NM) & 1, abort_flag, WAIT_NS)) {
+                    if (!tc::mbar_wait(bar.meta_full(slot), (gm / NM) & 1, abort_flag, WAIT_NS)) {
                         ok = false;
                         break;
                     }
                     const int br = metas[slot].br;
                     const int first = metas[slot].first;
-                    tc::mbar_arrive(&bar.meta_empty[slot]);
+                    tc::mbar_arrive(bar.meta_empty(slot));
                     ++gm;
                     if (br != BR_END) {
                         const int st = gi % NS;
-                        if (!tc::mbar_wait(&bar.k_full[st], (gi / NS) & 1, abort_flag, WAIT_NS)) {
+                        if (!tc::mbar_wait(bar.k_full(st), (gi / NS) & 1, abort_flag, WAIT_NS)) {
                             ok = false;
                             break;
                         }
@@ -467,17 +465,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             tc::mma_ss(dS, tc::sdesc_sw128(q_base + off, 16, 1024),
                                        tc::sdesc_sw128(kst + off, 16, 1024), idesc_qk, kk > 0);
                         }
-                        tc::mma_commit(&bar.s_full[gi & 1]);
-                        tc::mma_commit(&bar.k_empty[st]);
+                        tc::mma_commit(bar.s_full(gi & 1));
+                        tc::mma_commit(bar.k_empty(st));
                     } else {
-                        tc::mma_commit(bar.q_empty);
+                        tc::mma_commit(bar.q_empty());
                     }
                     if (have_prev) {
                         // O (+)= P V for the previous key tile
                         const int pst = prev_gi % NS;
-                        if (!tc::mbar_wait(&bar.p_full[prev_gi & 1], (prev_gi >> 1) & 1, abort_flag,
+                        if (!tc::mbar_wait(bar.p_full(prev_gi & 1), (prev_gi >> 1) & 1, abort_flag,
                                            WAIT_NS) ||
-                            !tc::mbar_wait(&bar.v_full[pst], (prev_gi / NS) & 1, abort_flag,
+                            !tc::mbar_wait(bar.v_full(pst), (prev_gi / NS) & 1, abort_flag,
                                            WAIT_NS)) {
                             ok = false;
                             break;
@@ -490,8 +488,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             tc::mma_ts(tO, aP + kk * 8, tc::sdesc_sw128(vst + kk * 2048, CHUNK, 1024),
                                        idesc_pv, (prev_first && kk == 0) ? 0u : 1u);
                         }
-                        tc::mma_commit(&bar.v_empty[pst]);
-                        tc::mma_commit(bar.pv_done);
+                        tc::mma_commit(bar.v_empty(pst));
+                        tc::mma_commit(bar.pv_done());
                     }
                     if (br == BR_END) break;
                     have_prev = true;
@@ -503,8 +501,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!ok) raise_abort(abort_flag);
             // all issued MMAs must finish before TMEM is released
             volatile int never = 0;
-            tc::mma_commit(bar.drain);
-            tc::mbar_wait(bar.drain, 0, &never, WAIT_NS);
+            tc::mma_commit(bar.drain());
+            tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
         }
         __syncwarp();
     } else {
@@ -567,18 +565,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
             while (true) {
                 const int slot = gm % NM;
-                if (!warp_wait(&bar.meta_full[slot], (gm / NM) & 1, abort_flag)) {
+                if (!warp_wait(bar.meta_full(slot), (gm / NM) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 const KeyTile kt = metas[slot];
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bar.meta_empty[slot]);
+                if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
                 ++gm;
                 if (kt.br == BR_END) break;
 
                 const int sb = gi & 1;
-                if (!warp_wait(&bar.s_full[sb], (gi >> 1) & 1, abort_flag)) {
+                if (!warp_wait(bar.s_full(sb), (gi >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -654,7 +652,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
                 // O may be touched only after the previous P V has landed
                 if (have_prev) {
-                    if (!warp_wait(bar.pv_done, npv & 1, abort_flag)) {
+                    if (!warp_wait(bar.pv_done(), npv & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -682,13 +680,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 cur_br = kt.br;
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bar.p_full[sb]);
+                if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
                 have_prev = true;
                 ++gi;
             }
             if (!ok) break;
             if (have_prev) {
-                if (!warp_wait(bar.pv_done, npv & 1, abort_flag)) {
+                if (!warp_wait(bar.pv_done(), npv & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -696,7 +694,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::fence_after_sync();
                 correction(cur_br);
             }
-            // epilogue: this half of the Acc row -> bf16 -> out
+            // selected branch computed outside: out += g_sel * o_sel
+            const bool add_sel = a.o_sel != nullptr && (a.s.flags & NSA_BR_SEL) && row_valid;
+            const float g_sel = add_sel ? (a.gates ? a.gates[grow * 3 + 1] : 1.f) : 0.f;
+            // epilogue: this half of the Acc row (+ the selected branch) -> bf16 -> out
 #pragma unroll 1
             for (int c = half * DVH; c < (half + 1) * DVH; c += 32) {
                 uint32_t acc[32];
@@ -706,6 +707,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 } else {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) acc[j] = 0u;
+                }
+                if (add_sel) {
+                    const uint4* src = reinterpret_cast<const uint4*>(a.o_sel + grow * DV + c);
+                    uint4 raw[4];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) raw[q4] = src[q4];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float f[8];
+                        unpack8(raw[q4], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            acc[8 * q4 + e] = __float_as_uint(fmaf(g_sel, f[e], __uint_as_float(acc[8 * q4 + e])));
+                    }
                 }
                 if (row_valid) {
                     uint4* dst = reinterpret_cast<uint4*>(a.out + grow * DV + c);
@@ -779,9 +794,10 @@ template <int DQK, int DV>
 cudaError_t launch_tc_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                            const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
-                           __nv_bfloat16* out, cudaStream_t st) {
+                           const __nv_bfloat16* o_sel, __nv_bfloat16* out, cudaStream_t st) {
     TcArgs a;
     a.s = s;
+    a.o_sel = o_sel;
     a.idx = idx;
     a.gates = gates;
     a.out = out;
@@ -828,10 +844,10 @@ bool attn_tc_supported(const Shape& s) {
 cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                            const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
-                           __nv_bfloat16* out, cudaStream_t st) {
+                           const __nv_bfloat16* o_sel, __nv_bfloat16* out, cudaStream_t st) {
 #define NSA_TC_CASE(A, B)                                                                  \
     if (s.dqk == A && s.dv == B)                                                           \
-        return launch_tc_impl<A, B>(s, q, k, v, kcmp, vcmp, gates, idx, out, st);
+        return launch_tc_impl<A, B>(s, q, k, v, kcmp, vcmp, gates, idx, o_sel, out, st);
     NSA_TC_CASE(64, 64)
     NSA_TC_CASE(128, 128)
     NSA_TC_CASE(192, 128)

@@ -87,6 +87,15 @@ bool attn_tc_supported(const Shape& s);
 cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                            const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
-                           __nv_bfloat16* out, cudaStream_t st);
+                           const __nv_bfloat16* o_sel, __nv_bfloat16* out, cudaStream_t st);
 int read_and_clear_tc_status();
+cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
+                             const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st);
+// block-major selected branch (attn_sel_bm.cu)
+struct SelIndex;
+bool sel_bm_supported(const Shape& s);
+cudaError_t launch_sel_bm(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                          const __nv_bfloat16* v, const SelIndex& x, __nv_bfloat16* part_o,
+                          float* part_lse, cudaStream_t st);
+int read_and_clear_bm_status();
 }  // namespace nsa

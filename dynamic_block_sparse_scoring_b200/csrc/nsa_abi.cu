@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "sel_index.cuh"
 
 namespace {
 
@@ -79,7 +80,55 @@ size_t idx_bytes(const Shape& s) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-nsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA; }
+// The selected branch runs block-major (inverted index + partials) for long
+// prefills on the tensor-core path; decode and short chunks keep it inside
+// the query-major kernel.
+bool use_block_major(const Shape& s) {
+    return (s.flags & NSA_BR_SEL) && nsa::attn_tc_supported(s) && nsa::sel_bm_supported(s) &&
+           s.Tq >= 256;
+}
+
+// Workspace regions, each 256-byte aligned, in this order.
+struct WsLayout {
+    size_t idx = 0, cnt = 0, off = 0, item_off = 0, cursor = 0, list = 0, items = 0, part_o = 0,
+           part_lse = 0, o_sel = 0, total = 0, minimal = 0;
+};
+
+WsLayout ws_layout(const Shape& s) {
+    WsLayout w;
+    size_t at = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = at;
+        at = round_up(at + bytes, 256);
+        return o;
+    };
+    if (!(s.flags & NSA_BR_SEL)) return w;
+    w.idx = take(idx_bytes(s));
+    w.minimal = at;
+    if (use_block_major(s)) {
+        const size_t L = nsa::sel_lists(s);
+        const int tok = 128 / s.heads_per_unit;
+        w.cnt = take(L * 4);
+        w.off = take((L + 1) * 4);
+        w.item_off = take((L + 1) * 4);
+        w.cursor = take(L * 4);
+        w.list = take(nsa::sel_pairs_max(s) * 4);
+        w.items = take(nsa::sel_items_max(s, tok) * sizeof(int4));
+        w.part_o = take(nsa::sel_pairs_max(s) * s.heads_per_unit * s.dv * 2);
+        w.part_lse = take(nsa::sel_pairs_max(s) * s.heads_per_unit * 4);
+        w.o_sel = take((size_t)s.B * s.Tq * s.Hq * s.dv * 2);
+    }
+    w.total = at;
+    return w;
+}
+
+thread_local const char* g_last_cuda_error = "no error";
+
+nsa_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return NSA_OK;
+    g_last_cuda_error = cudaGetErrorString(e);
+    return NSA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -102,7 +151,16 @@ nsa_status nsa_workspace_size(const nsa_config* cfg, size_t* bytes) {
     Shape s;
     nsa_status st = make_shape(cfg, &s);
     if (st != NSA_OK) return st;
-    *bytes = (cfg->flags & NSA_BR_SEL) ? round_up(idx_bytes(s), 256) : 0;
+    *bytes = ws_layout(s).total;
+    return NSA_OK;
+}
+
+nsa_status nsa_workspace_size_min(const nsa_config* cfg, size_t* bytes) {
+    if (!bytes) return NSA_ERR_INVALID_ARG;
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    *bytes = ws_layout(s).minimal;
     return NSA_OK;
 }
 
@@ -170,32 +228,59 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         !aligned16(vcmp) || !aligned16(gates) || !aligned16(idx) || !aligned16(out) ||
         !aligned16(workspace))
         return NSA_ERR_INVALID_ARG;
+    const WsLayout wl = ws_layout(s);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* sel_idx = const_cast<int32_t*>(idx);
     if (sel && !idx) {
-        if (!workspace || ws_bytes < idx_bytes(s)) return NSA_ERR_WORKSPACE;
-        sel_idx = static_cast<int32_t*>(workspace);
+        if (!workspace || ws_bytes < wl.minimal) return NSA_ERR_WORKSPACE;
+        sel_idx = reinterpret_cast<int32_t*>(ws + wl.idx);
     }
     if (s.Tq == 0) return NSA_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
+    const __nv_bfloat16* kcb = static_cast<const __nv_bfloat16*>(kcmp);
+    const __nv_bfloat16* vcb = static_cast<const __nv_bfloat16*>(vcmp);
+    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out);
     if (sel && !idx) {
         st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
         if (st != NSA_OK) return st;
     }
-    // tensor-core kernel for the shapes it covers, the row-wise kernel otherwise
-    auto attn = nsa::attn_tc_supported(s) ? nsa::launch_attn_tc : nsa::launch_attn;
-    return cuda_status(attn(s, qb, static_cast<const __nv_bfloat16*>(k),
-                            static_cast<const __nv_bfloat16*>(v),
-                            static_cast<const __nv_bfloat16*>(kcmp),
-                            static_cast<const __nv_bfloat16*>(vcmp), gates, sel_idx,
-                            static_cast<__nv_bfloat16*>(out), cs));
+    if (!nsa::attn_tc_supported(s))
+        return cuda_status(nsa::launch_attn(s, qb, kb, vb, kcb, vcb, gates, sel_idx, ob, cs));
+    // block-major selected branch when the workspace holds its index and partials
+    if (use_block_major(s) && ws && ws_bytes >= wl.total) {
+        nsa::SelIndex x;
+        x.cnt = reinterpret_cast<int32_t*>(ws + wl.cnt);
+        x.off = reinterpret_cast<int32_t*>(ws + wl.off);
+        x.item_off = reinterpret_cast<int32_t*>(ws + wl.item_off);
+        x.cursor = reinterpret_cast<int32_t*>(ws + wl.cursor);
+        x.list = reinterpret_cast<int32_t*>(ws + wl.list);
+        x.items = reinterpret_cast<int4*>(ws + wl.items);
+        __nv_bfloat16* part_o = reinterpret_cast<__nv_bfloat16*>(ws + wl.part_o);
+        float* part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
+        const int tok = 128 / s.heads_per_unit;
+        st = cuda_status(nsa::launch_sel_index(s, sel_idx, x, tok, cs));
+        if (st != NSA_OK) return st;
+        st = cuda_status(nsa::launch_sel_bm(s, qb, kb, vb, x, part_o, part_lse, cs));
+        if (st != NSA_OK) return st;
+        __nv_bfloat16* o_sel = reinterpret_cast<__nv_bfloat16*>(ws + wl.o_sel);
+        st = cuda_status(nsa::launch_sel_merge(s, sel_idx, part_o, part_lse, o_sel, cs));
+        if (st != NSA_OK) return st;
+        return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, o_sel, ob, cs));
+    }
+    return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr, ob, cs));
 }
+
+const char* nsa_last_cuda_error(void) { return g_last_cuda_error; }
 
 nsa_status nsa_get_device_status(int32_t* status) {
     if (!status) return NSA_ERR_INVALID_ARG;
-    const int v = nsa::read_and_clear_tc_status();
-    if (v < 0) return NSA_ERR_CUDA;
-    *status = v;
+    const int v1 = nsa::read_and_clear_tc_status();
+    const int v2 = nsa::read_and_clear_bm_status();
+    if (v1 < 0 || v2 < 0) return NSA_ERR_CUDA;
+    *status = v1 ? v1 : v2;
     return NSA_OK;
 }
 

@@ -56,7 +56,7 @@ extern "C" nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const v
                                                   const void* kcmp, const void* vcmp,
                                                   const float* gates, void* out, void* stream) {
     size_t need = 0;
-    nsa_status st = nsa_workspace_size(cfg, &need);
+    nsa_status st = nsa_workspace_size_min(cfg, &need);
     if (st != NSA_OK) return st;
     if (need > NOALLOC_SCRATCH_BYTES) return NSA_ERR_WORKSPACE;
     void* scratch = nullptr;

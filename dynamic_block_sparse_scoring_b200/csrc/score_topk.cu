@@ -10,8 +10,8 @@
 // scale * (sum_h q_h) . kbar_b in fp32: one dot product per (query, group,
 // block) instead of one per head.  A CTA takes RT query rows of one
 // selection unit, stages the rows' summed queries and chunks of KC pooled
-// keys in shared memory, forms the RT x KC score tile with FFMA, and keeps a
-// running top-(k-1) per row in the registers of one warp (one key per lane,
+// keys in shared memory, forms the RT x KC score tile with FFMA (a 4 x 4
+// register tile per thread), and keeps a running top-(k-1) per row in the registers of one warp (one key per lane,
 // sorted descending).  A key packs the order-preserving bits of the score
 // with the inverted block id, so a single 64-bit comparison orders by score
 // and then by lower block id.
@@ -21,9 +21,10 @@
 
 namespace nsa {
 
-constexpr int ST_RT = 32;   // query rows per CTA
+constexpr int ST_RT = 64;   // query rows per CTA
 constexpr int ST_KC = 64;   // pooled keys per chunk
-constexpr int ST_NT = 256;  // threads per CTA (8 warps x 4 rows)
+constexpr int ST_NT = 256;  // threads per CTA (8 warps x 8 rows of top-k state)
+constexpr int ST_RPW = ST_RT / 8;   // rows per warp
 
 enum { MODE_SELECT = 0, MODE_SCORES = 1, MODE_SELECT_FROM_SCORES = 2 };
 
@@ -38,7 +39,8 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
     const int ld = d + 4;
     float* qs = smem;                       // [RT][ld]   summed queries
     float* ks = qs + ST_RT * ld;            // [KC][ld]   pooled keys
-    float* ss = ks + ST_KC * ld;            // [RT][KC+1] score tile
+    float* ss = ks;                         // [RT][KC+1] score tile, reuses the key buffer
+                                            // once the FFMA tile is in registers
 
     const int i0 = blockIdx.x * ST_RT;
     const int u = blockIdx.y, b = blockIdx.z;
@@ -72,7 +74,9 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
     }
 
     const int K1 = s.topk - 1;               // past blocks kept per row
-    unsigned long long key[4] = {0ull, 0ull, 0ull, 0ull};   // lane's slot of rows 4*warp + j
+    unsigned long long key[ST_RPW];      // lane's slot of rows ST_RPW*warp + j
+#pragma unroll
+    for (int j = 0; j < ST_RPW; ++j) key[j] = 0ull;
 
     for (int b0 = 0; b0 < cmax; b0 += ST_KC) {
         const int nk = min(ST_KC, cmax - b0);
@@ -85,36 +89,49 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
                     *reinterpret_cast<const float4*>(src + (size_t)r * d + c4 * 4);
             }
             __syncthreads();
-            // thread -> row r, blocks bg, bg+8, ..., bg+56 of the chunk
-            const int r = tid >> 3, bg = tid & 7;
-            float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            const float* qr = qs + r * ld;
+            // register tile: thread -> rows 4*rg .. 4*rg+3, blocks bg, bg+16, bg+32, bg+48
+            const int rg = tid >> 4, bg = tid & 15;
+            float acc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) acc[i][m] = 0.f;
             for (int c = 0; c < d; c += 4) {
-                const float4 qv = *reinterpret_cast<const float4*>(qr + c);
+                float4 qv[4], kv[4];
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const float4 kv = *reinterpret_cast<const float4*>(ks + (bg + 8 * m) * ld + c);
-                    acc[m] = fmaf(qv.x, kv.x, acc[m]);
-                    acc[m] = fmaf(qv.y, kv.y, acc[m]);
-                    acc[m] = fmaf(qv.z, kv.z, acc[m]);
-                    acc[m] = fmaf(qv.w, kv.w, acc[m]);
-                }
-            }
-            const int t = s.q0 + i0 + r;
-            const int cr = t / s.bs;
+                for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4*>(qs + (4 * rg + i) * ld + c);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int jj = bg + 8 * m;
-                const int blk = b0 + jj;
-                const bool valid = (r < nrows) && (jj < nk) && (blk < cr);
-                const float val = s.scale * acc[m];
-                if (MODE == MODE_SCORES) {
-                    if (r < nrows && jj < nk) {
-                        float w = blk < cr ? val : (blk == cr ? INFINITY : -INFINITY);
-                        scores_out[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + blk] = w;
+                for (int m = 0; m < 4; ++m) kv[m] = *reinterpret_cast<const float4*>(ks + (bg + 16 * m) * ld + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        acc[i][m] = fmaf(qv[i].x, kv[m].x, acc[i][m]);
+                        acc[i][m] = fmaf(qv[i].y, kv[m].y, acc[i][m]);
+                        acc[i][m] = fmaf(qv[i].z, kv[m].z, acc[i][m]);
+                        acc[i][m] = fmaf(qv[i].w, kv[m].w, acc[i][m]);
                     }
-                } else {
-                    ss[r * (ST_KC + 1) + jj] = valid ? val : -INFINITY;
+            }
+            __syncthreads();                 // every thread is done reading ks
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = 4 * rg + i;
+                const int t = s.q0 + i0 + r;
+                const int cr = t / s.bs;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int jj = bg + 16 * m;
+                    const int blk = b0 + jj;
+                    const bool valid = (r < nrows) && (jj < nk) && (blk < cr);
+                    const float val = s.scale * acc[i][m];
+                    if (MODE == MODE_SCORES) {
+                        if (r < nrows && jj < nk) {
+                            float w = blk < cr ? val : (blk == cr ? INFINITY : -INFINITY);
+                            scores_out[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + blk] = w;
+                        }
+                    } else {
+                        ss[r * (ST_KC + 1) + jj] = valid ? val : -INFINITY;
+                    }
                 }
             }
         } else {
@@ -134,8 +151,8 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
 
         if (MODE != MODE_SCORES && K1 > 0) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = warp * 4 + j;
+            for (int j = 0; j < ST_RPW; ++j) {
+                const int r = warp * ST_RPW + j;
                 unsigned long long thr = __shfl_sync(0xffffffffu, key[j], K1 - 1);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -176,8 +193,8 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
     }
 
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int r = warp * 4 + j;
+    for (int j = 0; j < ST_RPW; ++j) {
+        const int r = warp * ST_RPW + j;
         if (r >= nrows) continue;
         const int cr = (s.q0 + i0 + r) / s.bs;
         const bool have = lane < K1 && key[j] != 0ull;
@@ -199,8 +216,9 @@ cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const floa
                               const float* scores_in, float* scores_out, int32_t* idx,
                               cudaStream_t st) {
     const int ld = s.dqk + 4;
-    const size_t smem = ((size_t)ST_RT * ld + (size_t)ST_KC * ld + (size_t)ST_RT * (ST_KC + 1)) *
-                        sizeof(float);
+    const size_t key_buf = (size_t)ST_KC * ld > (size_t)ST_RT * (ST_KC + 1)
+                               ? (size_t)ST_KC * ld : (size_t)ST_RT * (ST_KC + 1);
+    const size_t smem = ((size_t)ST_RT * ld + key_buf) * sizeof(float);
     dim3 grid((s.Tq + ST_RT - 1) / ST_RT, s.Hsel, s.B);
     if (scores_out) {
         cudaFuncSetAttribute(score_topk_kernel<MODE_SCORES>,

@@ -1,0 +1,148 @@
+// Inverted index of the selected blocks: for every (sequence, selection unit,
+// block) the (query, slot) pairs whose top-k set holds that block.
+//
+// This is the gathering step of MoBA's execution (Zhang Xiaojun #94
+// transcript (bidclub.ai), §7 "Kimi Simplifies The Sparse Route": for each KV
+// block, collect the queries that chose it into one contiguous batch), used
+// here for group-shared NSA selection too, so that a block's keys are loaded
+// once for every query that kept it.
+//
+// Four launches: count pairs per list (atomics), one-CTA exclusive scans of
+// the counts and of the work items per list, fill the lists (atomic cursors;
+// the order inside a list does not matter because every row of an attention
+// tile is computed independently), and cut each list into work items of at
+// most `tok` queries.
+#include "common.cuh"
+#include "sel_index.cuh"
+
+namespace nsa {
+
+namespace {
+
+// list id of pair e (flat index into idx) holding block blk
+__device__ __forceinline__ size_t list_of(size_t e, int blk, int BHsel, int Tq, int topk,
+                                          int nb_all) {
+    const size_t bu = e / ((size_t)Tq * topk);                  // b * Hsel + u
+    const int qi = (int)((e % ((size_t)Tq * topk)) / topk);
+    const size_t chunk = qi / SEL_CHUNK;
+    return (chunk * BHsel + bu) * nb_all + blk;
+}
+
+__global__ void count_pairs_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
+                                   int BHsel, int Tq, int topk, int nb_all, size_t total) {
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int blk = idx[e];
+        if (blk < 0) continue;
+        atomicAdd(&cnt[list_of(e, blk, BHsel, Tq, topk, nb_all)], 1);
+    }
+}
+
+// Single CTA of 1024 threads: off = exclusive scan of cnt, item_off =
+// exclusive scan of ceil(cnt / tok); writes the totals at index L.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ cnt,
+                                                    int32_t* __restrict__ off,
+                                                    int32_t* __restrict__ item_off,
+                                                    int32_t* __restrict__ cursor, int L, int tok) {
+    __shared__ int32_t wsum_a[32], wsum_b[32];
+    __shared__ int32_t carry_a, carry_b;
+    if (threadIdx.x == 0) carry_a = carry_b = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = 0; base < L; base += 1024) {
+        const int i = base + threadIdx.x;
+        const int c = i < L ? cnt[i] : 0;
+        const int n = (c + tok - 1) / tok;
+        int a = c, b = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ya = __shfl_up_sync(0xffffffffu, a, o);
+            const int yb = __shfl_up_sync(0xffffffffu, b, o);
+            if (lane >= o) {
+                a += ya;
+                b += yb;
+            }
+        }
+        if (lane == 31) {
+            wsum_a[warp] = a;
+            wsum_b[warp] = b;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int sa = wsum_a[lane], sb = wsum_b[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int ya = __shfl_up_sync(0xffffffffu, sa, o);
+                const int yb = __shfl_up_sync(0xffffffffu, sb, o);
+                if (lane >= o) {
+                    sa += ya;
+                    sb += yb;
+                }
+            }
+            wsum_a[lane] = sa;
+            wsum_b[lane] = sb;
+        }
+        __syncthreads();
+        const int pa = (warp ? wsum_a[warp - 1] : 0) + a - c + carry_a;   // exclusive
+        const int pb = (warp ? wsum_b[warp - 1] : 0) + b - n + carry_b;
+        if (i < L) {
+            off[i] = pa;
+            cursor[i] = pa;
+            item_off[i] = pb;
+        }
+        __syncthreads();
+        if (threadIdx.x == 1023) {
+            carry_a = pa + c;
+            carry_b = pb + n;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        off[L] = carry_a;
+        item_off[L] = carry_b;
+    }
+}
+
+__global__ void fill_pairs_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ cursor,
+                                  int32_t* __restrict__ list, int BHsel, int Tq, int topk,
+                                  int nb_all, size_t total) {
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int blk = idx[e];
+        if (blk < 0) continue;
+        const int rem = (int)(e % ((size_t)Tq * topk));
+        const int qi = rem / topk, slot = rem % topk;
+        const int pos = atomicAdd(&cursor[list_of(e, blk, BHsel, Tq, topk, nb_all)], 1);
+        list[pos] = qi * 32 + slot;
+    }
+}
+
+__global__ void make_items_kernel(const int32_t* __restrict__ off,
+                                  const int32_t* __restrict__ item_off, int4* __restrict__ items,
+                                  int L, int tok) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < L; i += gridDim.x * blockDim.x) {
+        const int c = off[i + 1] - off[i];
+        int it = item_off[i];
+        for (int q = 0; q < c; q += tok, ++it) items[it] = make_int4(i, off[i] + q, min(tok, c - q), 0);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_sel_index(const Shape& s, const int32_t* idx, const SelIndex& x, int tok,
+                             cudaStream_t st) {
+    const int L = (int)sel_lists(s);
+    const int BHsel = s.B * s.Hsel;
+    const size_t total = (size_t)s.B * s.Hsel * s.Tq * s.topk;
+    cudaError_t e = cudaMemsetAsync(x.cnt, 0, sizeof(int32_t) * L, st);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
+    count_pairs_kernel<<<grid, 256, 0, st>>>(idx, x.cnt, BHsel, s.Tq, s.topk, s.nb_all, total);
+    scan_kernel<<<1, 1024, 0, st>>>(x.cnt, x.off, x.item_off, x.cursor, L, tok);
+    fill_pairs_kernel<<<grid, 256, 0, st>>>(idx, x.cursor, x.list, BHsel, s.Tq, s.topk, s.nb_all,
+                                            total);
+    make_items_kernel<<<(L + 255) / 256, 256, 0, st>>>(x.off, x.item_off, x.items, L, tok);
+    return cudaGetLastError();
+}
+
+}  // namespace nsa

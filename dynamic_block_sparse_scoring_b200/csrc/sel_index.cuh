@@ -1,0 +1,39 @@
+// Device buffers of the selected-block inverted index (see sel_index.cu).
+#pragma once
+
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace nsa {
+
+struct SelIndex {
+    int32_t* cnt;       // [L] pairs per list, L = B * Hsel * nb_all
+    int32_t* off;       // [L + 1] list offsets (exclusive scan); off[L] = pairs
+    int32_t* item_off;  // [L + 1] first work item of each list; item_off[L] = items
+    int32_t* cursor;    // [L] fill cursors
+    int32_t* list;      // [pairs] query * 32 + slot, grouped by list
+    int4* items;        // [items] (list id, first pair, pair count, 0)
+};
+
+// Lists are keyed by (query chunk, selection unit, block): list id =
+// (chunk * B * Hsel + b * Hsel + u) * nb_all + block, chunk = query / SEL_CHUNK.
+// Work items are therefore ordered chunk by chunk, which keeps the queries
+// (and the partial outputs) of one chunk hot in L2 while it is processed.
+constexpr int SEL_CHUNK = 4096;
+inline int sel_chunks(const Shape& s) { return (s.Tq + SEL_CHUNK - 1) / SEL_CHUNK; }
+inline size_t sel_lists_per_chunk(const Shape& s) { return (size_t)s.B * s.Hsel * s.nb_all; }
+
+// Upper bounds used to size the workspace.
+inline size_t sel_pairs_max(const Shape& s) { return (size_t)s.B * s.Hsel * s.Tq * s.topk; }
+inline size_t sel_lists(const Shape& s) { return (size_t)sel_chunks(s) * sel_lists_per_chunk(s); }
+inline size_t sel_items_max(const Shape& s, int tok) {
+    return sel_pairs_max(s) / tok + sel_lists(s) + 1;
+}
+
+cudaError_t launch_sel_index(const Shape& s, const int32_t* idx, const SelIndex& x, int tok,
+                             cudaStream_t st);
+
+}  // namespace nsa

@@ -91,11 +91,22 @@ typedef struct {
 } nsa_config;
 
 /*
- * Bytes of device workspace nsa_sparse_attn_fwd needs for `cfg` when it
- * selects the blocks itself (idx == NULL).  Writes 0 when no workspace is
- * needed.  Pure host function.
+ * Bytes of device workspace for nsa_sparse_attn_fwd's fastest path on `cfg`:
+ * the selected block ids (when it selects them itself) plus, for long
+ * prefills on the tensor-core path, the per-block query lists and the
+ * per-(query, slot) partial outputs of the block-major selected branch
+ * (about topk * heads * d_v * 2 bytes per query).  Writes 0 when no
+ * workspace is needed.  Pure host function.
  */
 nsa_status nsa_workspace_size(const nsa_config* cfg, size_t* bytes);
+
+/*
+ * Smallest workspace nsa_sparse_attn_fwd accepts with idx == NULL: the
+ * selected block ids only.  With a workspace smaller than
+ * nsa_workspace_size() the selected branch runs inside the query-major
+ * kernel instead (same result, slower for long prefills).  Pure host function.
+ */
+nsa_status nsa_workspace_size_min(const nsa_config* cfg, size_t* bytes);
 
 /*
  * Block representations (transcript #94 §4 Figure 2 "compression", §7 mean
@@ -142,8 +153,12 @@ nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kb
  * A branch with no visible key contributes 0.  Softmax and accumulation run in
  * fp32; out is rounded to bf16 once.
  * idx may be NULL, in which case the blocks are selected as nsa_topk_select
- * does (needs q, kbar and a workspace of nsa_workspace_size() bytes);
- * otherwise kbar may be NULL and the workspace may be NULL/0.
+ * does (needs q, kbar and at least nsa_workspace_size_min() bytes of
+ * workspace); otherwise kbar may be NULL.  A workspace of
+ * nsa_workspace_size() bytes enables the block-major selected branch (each
+ * selected KV block attended once for all the queries that kept it); a
+ * smaller one (or NULL with an external idx) computes the same result with
+ * the selected branch inside the query-major kernel.
  * kcmp/vcmp are read only with NSA_BR_CMP.
  */
 nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void* k,
@@ -161,7 +176,7 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
  * the host framework owns all device buffers, and latency-critical callers for
  * which cudaMalloc/cudaFree are off limits because they can synchronise the
  * device.
- * Limit: problems with nsa_workspace_size() > 32 MiB return NSA_ERR_WORKSPACE
+ * Limit: problems with nsa_workspace_size_min() > 32 MiB return NSA_ERR_WORKSPACE
  * (e.g. 65536 queries x 4 selection units x top-16 need 16 MiB).
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it.  Every call uses the same array, which keeps
@@ -180,6 +195,10 @@ nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, con
  * all work on the current device first.  Not for use inside stream capture.
  */
 nsa_status nsa_get_device_status(int32_t* status);
+
+/* CUDA's description of the error behind the calling thread's most recent
+ * NSA_ERR_CUDA (a static string; "no error" if there was none). */
+const char* nsa_last_cuda_error(void);
 
 /* Static, human-readable name of a status code. */
 const char* nsa_status_string(nsa_status status);

@@ -52,13 +52,22 @@ def _cfg(abi, **kw):
     return abi.config(WORKLOADS["tiny"], **kw)
 
 
-def test_workspace_size_is_idx_buffer(abi):
+def test_workspace_sizes(abi):
     from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
     for name, wl in WORKLOADS.items():
         cfg = abi.config(wl)
         n = abi.nsa_workspace_size(cfg)
+        nmin = abi.nsa_workspace_size_min(cfg)
         want = wl.batch * wl.h_sel * wl.seqlen_q * wl.top_k * 4
-        assert n >= want and n % 256 == 0, name
+        assert nmin >= want and nmin % 256 == 0 and n >= nmin, name
+    # the 64k NSA prefill runs its selected branch block-major: index + bf16 partials
+    wl = WORKLOADS["nsa64k"]
+    n = abi.nsa_workspace_size(abi.config(wl))
+    assert n >= wl.seqlen_q * wl.h_kv * wl.top_k * wl.group * wl.d_v * 2
+    # decode keeps the selected branch in the query-major kernel: ids only
+    wl = WORKLOADS["decode64x64k"]
+    cfg = abi.config(wl)
+    assert abi.nsa_workspace_size(cfg) == abi.nsa_workspace_size_min(cfg)
 
 
 @pytest.mark.parametrize("bad,status", [

@@ -45,6 +45,13 @@ EDGE = {
                                            h_q=16, h_kv=1),
     "cmp_identity": TINY.with_(name="cmp_identity", seqlen_q=200, seqlen_kv=200, cmp_block=1,
                                cmp_stride=1),
+    # block-major selected branch (groups of 8 and 16 heads, sel_block 64, >= 256 queries)
+    "bm_g8_ragged": WORKLOADS["nsa64k"].with_(name="bm_g8_ragged", seqlen_q=1000, seqlen_kv=1000,
+                                              h_q=16, h_kv=2, d_qk=128, d_v=128),
+    "bm_chunked": WORKLOADS["nsa64k"].with_(name="bm_chunked", seqlen_q=300, seqlen_kv=2000,
+                                            q_pos0=1700, h_q=16, h_kv=1),
+    "bm_batch2": WORKLOADS["nsa64k"].with_(name="bm_batch2", batch=2, seqlen_q=700, seqlen_kv=700,
+                                           h_q=32, h_kv=2, d_qk=64, d_v=64),
 }
 
 
@@ -172,3 +179,25 @@ def test_decode_sampled_sequences():
     wl = WORKLOADS["decode64x64k"]
     run = GpuRun(wl)
     compare_run(run, [0], seqs=[0, 31, 63])
+
+
+@pytest.mark.parametrize("name", ["nsa_small", "bm_g8_ragged"])
+def test_minimal_workspace_path_matches_oracle(name):
+    """With only nsa_workspace_size_min() bytes the selected branch runs query-major."""
+    wl = EDGE[name]
+    run = GpuRun(wl)
+    cfg = run.cfg
+    wmin = abi.nsa_workspace_size_min(cfg)
+    assert wmin < abi.nsa_workspace_size(cfg)
+    ws = torch.empty(wmin, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(run.out)
+    abi.nsa_sparse_attn_fwd(cfg, run.x["q"], run.x["k"], run.x["v"], run.pooled["kbar"],
+                            run.pooled["kcmp"], run.pooled["vcmp"], run.x["gates"], None, out, ws,
+                            wmin)
+    torch.cuda.synchronize()
+    assert abi.nsa_get_device_status() == 0
+    rows = np.arange(wl.seqlen_q)
+    ora, _, _ = run.oracle_rows(0, rows, idx=run.idx[0].cpu().numpy())
+    check_out(f64(out[0]), ora, f"{name} minimal workspace")
+    # the two selected-branch organisations agree with each other as well
+    check_out(f64(out[0]), f64(run.out[0]), f"{name} query-major vs block-major")
