@@ -175,6 +175,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint32_t kv_loads = 0, q_loads = 0;
         int prev_lidx = -1, kvs = 0;
         int chunk = 0, i = 0, i_end = 0, li = 0, ends = 0;
+        // register windows over the item and list arrays (both are consumed in
+        // order, so one coalesced warp load serves many items)
+        int4 iwin = make_int4(0, 0, 0, 0);
+        int ibase = -1;
+        int lwin0 = 0, lwin1 = 0, lbase = -1;
+        auto item_at = [&](int k) -> int4 {
+            if (ibase < 0 || k < ibase || k >= ibase + 32) {
+                ibase = k;
+                iwin = a.items[k + lane];          // the items array has 32 slack entries
+            }
+            int4 r;
+            r.x = __shfl_sync(0xffffffffu, iwin.x, k - ibase);
+            r.y = __shfl_sync(0xffffffffu, iwin.y, k - ibase);
+            r.z = __shfl_sync(0xffffffffu, iwin.z, k - ibase);
+            return r;
+        };
+        auto list_at = [&](int pos, int n) -> int {     // lane l < n gets list[pos + l]
+            if (lbase < 0 || pos < lbase || pos + n > lbase + 64) {
+                lbase = pos;
+                lwin0 = a.list[pos + lane];
+                lwin1 = a.list[pos + 32 + lane];       // the list array has 64 slack entries
+            }
+            const int o = pos - lbase + lane;
+            const int v0 = __shfl_sync(0xffffffffu, lwin0, o & 31);
+            const int v1 = __shfl_sync(0xffffffffu, lwin1, o & 31);
+            return o < 32 ? v0 : v1;
+        };
         chunk_range(0, i, i_end);
         while (ok && ends < 2) {
             while (i >= i_end && chunk + 1 < a.n_chunks) chunk_range(++chunk, i, i_end);
@@ -182,14 +209,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             m.valid = i < i_end;
             m.lidx = m.n = m.kvs = m.new_block = m.last_of_block = 0;
             if (m.valid) {
-                const int4 it = a.items[i];
+                const int4 it = item_at(i);
                 m.lidx = it.x;
                 m.n = it.z;
                 m.new_block = it.x != prev_lidx;
                 // the next item this CTA will take (possibly in a later chunk)
-                int nxt = i + 1, nxt_end = i_end, nchunk = chunk;
-                while (nxt >= nxt_end && nchunk + 1 < a.n_chunks) chunk_range(++nchunk, nxt, nxt_end);
-                m.last_of_block = nxt >= nxt_end || a.items[nxt].x != it.x;
+                if (i + 1 < i_end) {
+                    m.last_of_block = item_at(i + 1).x != it.x;
+                } else {
+                    int nxt = i + 1, nxt_end = i_end, nchunk = chunk;
+                    while (nxt >= nxt_end && nchunk + 1 < a.n_chunks) chunk_range(++nchunk, nxt, nxt_end);
+                    m.last_of_block = nxt >= nxt_end || a.items[nxt].x != it.x;
+                }
                 const int bu = (it.x / nb_all) % bhsel, j = it.x % nb_all;
                 const int b = bu / a.s.Hsel, u = bu % a.s.Hsel;
                 const int kvh = a.s.per_head ? u / a.s.G : u;
@@ -200,33 +231,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         ok = false;
                         break;
                     }
-                    if (lane == 0) {
-                        tc::mbar_arrive_expect_tx(bar.kv_full(kvs), (L::QC + L::VC) * CHUNK_KV);
-                        const int plane = b * a.s.Hkv + kvh;
-                        for (int c = 0; c < L::QC; ++c)
-                            tc::tma_load_3d(sm + L::K_OFF + (kvs * L::QC + c) * CHUNK_KV, &map_k,
-                                            bar.kv_full(kvs), 64 * c, j * BLK, plane);
-                        for (int c = 0; c < L::VC; ++c)
-                            tc::tma_load_3d(sm + L::V_OFF + (kvs * L::VC + c) * CHUNK_KV, &map_v,
-                                            bar.kv_full(kvs), 64 * c, j * BLK, plane);
-                    }
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.kv_full(kvs), (L::QC + L::VC) * CHUNK_KV);
+                    __syncwarp();
+                    const int plane = b * a.s.Hkv + kvh;
+                    if (lane < L::QC)
+                        tc::tma_load_3d(sm + L::K_OFF + (kvs * L::QC + lane) * CHUNK_KV, &map_k,
+                                        bar.kv_full(kvs), 64 * lane, j * BLK, plane);
+                    else if (lane < L::QC + L::VC)
+                        tc::tma_load_3d(sm + L::V_OFF + (kvs * L::VC + lane - L::QC) * CHUNK_KV, &map_v,
+                                        bar.kv_full(kvs), 64 * (lane - L::QC), j * BLK, plane);
                     ++kv_loads;
                     prev_lidx = it.x;
                 }
                 m.kvs = kvs;
-                const int tokv = lane < m.n ? a.list[it.y + lane] : 0;
+                const int tokv = list_at(it.y, m.n);
                 for (int tt = 0; tt < MAX_TOK; ++tt) m.tok[tt] = __shfl_sync(0xffffffffu, tokv, tt);
                 const int qs = li & 1;
                 if (!bm_warp_wait(bar.q_empty(qs), ((li >> 1) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                if (lane == 0) {
-                    tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
-                    for (int tt = 0; tt < m.n; ++tt)
-                        for (int c = 0; c < L::QC; ++c)
-                            tc::tma_load_4d(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
-                                            &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b);
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
+                __syncwarp();
+                // one TMA per (query, 64-column chunk), spread over the lanes
+                for (int e = lane; e < m.n * L::QC; e += 32) {
+                    const int tt = e / L::QC, c = e % L::QC;
+                    tc::tma_load_4d(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
+                                    &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b);
                 }
                 ++q_loads;
                 ++i;
@@ -511,7 +542,7 @@ bool sel_bm_supported(const Shape& s) {
     if (s.dv != 64 && s.dv != 128) return false;
     if (s.bs != BLK) return false;
     const int hpt = s.heads_per_unit;
-    return (hpt == 8 || hpt == 16) && s.topk <= 32;
+    return (hpt == 8 || hpt == 16) && s.topk <= 16;
 }
 
 cudaError_t launch_sel_bm(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,

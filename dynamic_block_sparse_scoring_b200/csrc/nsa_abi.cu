@@ -112,7 +112,7 @@ WsLayout ws_layout(const Shape& s) {
         w.off = take((L + 1) * 4);
         w.item_off = take((L + 1) * 4);
         w.cursor = take(L * 4);
-        w.list = take(nsa::sel_pairs_max(s) * 4);
+        w.list = take(nsa::sel_list_alloc(s) * 4);
         w.items = take(nsa::sel_items_max(s, tok) * sizeof(int4));
         w.part_o = take(nsa::sel_pairs_max(s) * s.heads_per_unit * s.dv * 2);
         w.part_lse = take(nsa::sel_pairs_max(s) * s.heads_per_unit * 4);

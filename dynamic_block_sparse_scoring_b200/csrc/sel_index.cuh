@@ -29,9 +29,12 @@ inline size_t sel_lists_per_chunk(const Shape& s) { return (size_t)s.B * s.Hsel 
 // Upper bounds used to size the workspace.
 inline size_t sel_pairs_max(const Shape& s) { return (size_t)s.B * s.Hsel * s.Tq * s.topk; }
 inline size_t sel_lists(const Shape& s) { return (size_t)sel_chunks(s) * sel_lists_per_chunk(s); }
+// (+32 / +64 slack entries: the block-major producer reads 32 items / 64 list
+// entries at a time past the last valid one)
 inline size_t sel_items_max(const Shape& s, int tok) {
-    return sel_pairs_max(s) / tok + sel_lists(s) + 1;
+    return sel_pairs_max(s) / tok + sel_lists(s) + 1 + 32;
 }
+inline size_t sel_list_alloc(const Shape& s) { return sel_pairs_max(s) + 64; }
 
 cudaError_t launch_sel_index(const Shape& s, const int32_t* idx, const SelIndex& x, int tok,
                              cudaStream_t st);

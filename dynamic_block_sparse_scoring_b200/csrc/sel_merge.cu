@@ -7,14 +7,15 @@
 // per-block results by their normalisers recovers that single softmax.
 //
 // HBM-bound: a thread owns 8 output columns of one (query, head) and issues
-// all of its slots' 16-byte partial loads before combining them.
+// all of its slots' 16-byte partial loads (after one read of the query's
+// block ids) before combining them.
 #include "common.cuh"
 
 namespace nsa {
 
 namespace {
 
-constexpr int MG_MAXK = 32;
+constexpr int MG_MAXK = 16;   // slots per query handled here (the block-major path needs top_k <= 16)
 
 __global__ void __launch_bounds__(256) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
                                                         const __nv_bfloat16* __restrict__ part_o,
@@ -29,24 +30,33 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(Shape s, const int32_t* 
     const int u = blockIdx.y, b = blockIdx.z;
     if (tl >= tok_per_cta || qi >= s.Tq) return;
     const size_t prow0 = ((size_t)(b * s.Hsel + u) * s.Tq + qi) * s.topk;
+    // the kept blocks fill the first slots (ascending, -1 padded)
     const int32_t* irow = idx + prow0;
+    int nvalid = 0;
+#pragma unroll
+    for (int sl = 0; sl < MG_MAXK; ++sl) nvalid += (sl < s.topk && irow[sl] >= 0) ? 1 : 0;
     float lse[MG_MAXK];
+    uint4 raw[MG_MAXK];
     float m = -INFINITY;
 #pragma unroll
-    for (int sl = 0; sl < MG_MAXK; ++sl) {
+    for (int sl = 0; sl < MG_MAXK; ++sl) {             // every load of the row issued at once
         lse[sl] = -INFINITY;
-        if (sl < s.topk && irow[sl] >= 0) lse[sl] = part_lse[(prow0 + sl) * hpt + h];
-        m = fmaxf(m, lse[sl]);
+        if (sl < nvalid) {
+            lse[sl] = part_lse[(prow0 + sl) * hpt + h];
+            raw[sl] = *reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8);
+        }
     }
+#pragma unroll
+    for (int sl = 0; sl < MG_MAXK; ++sl) m = fmaxf(m, lse[sl]);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     float wsum = 0.f;
 #pragma unroll
     for (int sl = 0; sl < MG_MAXK; ++sl) {
-        if (lse[sl] == -INFINITY) continue;
+        if (sl >= nvalid) break;
         const float w = exp2f(lse[sl] - m);
         wsum += w;
         float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8), f);
+        unpack8(raw[sl], f);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
     }
