@@ -17,17 +17,20 @@
 // query's own block, where key u is visible iff u <= t.  Each row writes a
 // partial result for its (query, slot): o = (P V)/l in bf16 and
 // lse = m + log2(l) in the scaled-log2 domain.  The partials of a query's
-// slots are merged by sel_merge.cu.  Items come chunk by chunk (4096
+// slots are merged by sel_merge.cu.  Items come chunk by chunk (2048
 // queries); every CTA takes a contiguous share of each chunk, so the chunk's
 // queries stay in L2 while consecutive items of a CTA share their K/V block.
 //
-// Roles (320 threads): warp 0 TMA producer (K/V once per run of items on the
+// Roles (448 threads): warp 0 TMA producer (K/V once per run of items on the
 // same block, Q rows per item), warp 1 MMA lane + TMEM owner, warps 2-5 and
-// 6-9 two softmax/epilogue warpgroups that take alternate items (each with
-// its own S and O in TMEM), so consecutive items overlap.  All waits are
+// 6-9 two softmax warpgroups taking alternate items (S/P double-buffered in
+// TMEM), warps 10-13 the epilogue warpgroup (O double-buffered in TMEM,
+// drained to the partial buffers while the next items' softmax runs).  All waits are
 // bounded; a timeout records NSA_ERR_TIMEOUT in g_bm_status and unwinds.
 #include <cudaTypedefs.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "sel_index.cuh"
@@ -41,12 +44,13 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BLK = 64;             // keys per block (the path requires sel_block == 64)
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 448;      // producer, MMA, 2 softmax warpgroups, epilogue warpgroup
 constexpr int NM = 8;               // item descriptors in flight
 constexpr int CHUNK_Q = 16384;      // 128 rows x 64 columns bf16
 constexpr int CHUNK_KV = 8192;      // 64 rows x 64 columns bf16
 constexpr uint64_t WAIT_NS = 1000000000ull;
 constexpr int MAX_TOK = 16;
+constexpr int NQ = 2;               // query-gather stages
 
 struct ItemMeta {
     int valid;          // 0 = end of the stream
@@ -75,31 +79,33 @@ struct BmArgs {
 template <int DQK, int DV>
 struct BmSmem {
     static constexpr int QC = DQK / 64, VC = DV / 64;
-    static constexpr int Q_OFF = 0;                                  // 2 stages
-    static constexpr int K_OFF = Q_OFF + 2 * QC * CHUNK_Q;            // 2 stages
+    static constexpr int Q_OFF = 0;                                  // NQ stages
+    static constexpr int K_OFF = Q_OFF + NQ * QC * CHUNK_Q;           // 2 stages
     static constexpr int V_OFF = K_OFF + 2 * QC * CHUNK_KV;           // 2 stages
     static constexpr int META_OFF = V_OFF + 2 * VC * CHUNK_KV;
-    static constexpr int BAR_OFF = META_OFF + NM * (int)sizeof(ItemMeta);
-    // q_full[2] q_empty[2] kv_full[2] kv_empty[2] meta_full[NM] meta_empty[NM]
+    static constexpr int ROW_OFF = META_OFF + NM * (int)sizeof(ItemMeta);   // row m, l [2][2][BM]
+    static constexpr int BAR_OFF = ROW_OFF + 4 * BM * 4;
+    // q_full[NQ] q_empty[NQ] kv_full[2] kv_empty[2] meta_full[NM] meta_empty[NM]
     // s_full[2] p_full[2] o_full[2] o_free[2] drain
-    static constexpr int NBAR = 8 + 2 * NM + 8 + 1;
+    static constexpr int NBAR = 2 * NQ + 4 + 2 * NM + 8 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int ALLOC = MISC_OFF + 64 + 1024;
 };
 
 struct BmBars {
     uint64_t* b;
+    static constexpr int KV0 = 2 * NQ, MT0 = KV0 + 4, SB0 = MT0 + 2 * NM;
     __device__ __forceinline__ uint64_t* q_full(int i) const { return b + i; }
-    __device__ __forceinline__ uint64_t* q_empty(int i) const { return b + 2 + i; }
-    __device__ __forceinline__ uint64_t* kv_full(int i) const { return b + 4 + i; }
-    __device__ __forceinline__ uint64_t* kv_empty(int i) const { return b + 6 + i; }
-    __device__ __forceinline__ uint64_t* meta_full(int i) const { return b + 8 + i; }
-    __device__ __forceinline__ uint64_t* meta_empty(int i) const { return b + 8 + NM + i; }
-    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 8 + 2 * NM + i; }
-    __device__ __forceinline__ uint64_t* p_full(int i) const { return b + 10 + 2 * NM + i; }
-    __device__ __forceinline__ uint64_t* o_full(int i) const { return b + 12 + 2 * NM + i; }
-    __device__ __forceinline__ uint64_t* o_free(int i) const { return b + 14 + 2 * NM + i; }
-    __device__ __forceinline__ uint64_t* drain() const { return b + 16 + 2 * NM; }
+    __device__ __forceinline__ uint64_t* q_empty(int i) const { return b + NQ + i; }
+    __device__ __forceinline__ uint64_t* kv_full(int i) const { return b + KV0 + i; }
+    __device__ __forceinline__ uint64_t* kv_empty(int i) const { return b + KV0 + 2 + i; }
+    __device__ __forceinline__ uint64_t* meta_full(int i) const { return b + MT0 + i; }
+    __device__ __forceinline__ uint64_t* meta_empty(int i) const { return b + MT0 + NM + i; }
+    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + SB0 + i; }
+    __device__ __forceinline__ uint64_t* p_full(int i) const { return b + SB0 + 2 + i; }
+    __device__ __forceinline__ uint64_t* o_full(int i) const { return b + SB0 + 4 + i; }
+    __device__ __forceinline__ uint64_t* o_free(int i) const { return b + SB0 + 6 + i; }
+    __device__ __forceinline__ uint64_t* drain() const { return b + SB0 + 8; }
 };
 
 __device__ __forceinline__ bool bm_warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
@@ -126,9 +132,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NQ; ++i) {
             tc::mbar_init(bar.q_full(i), 1);
             tc::mbar_init(bar.q_empty(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bar.kv_full(i), 1);
             tc::mbar_init(bar.kv_empty(i), 1);
             tc::mbar_init(bar.s_full(i), 1);
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int i = 0; i < NM; ++i) {
             tc::mbar_init(bar.meta_full(i), 1);
-            tc::mbar_init(bar.meta_empty(i), 5);   // MMA lane + the owning warpgroup's 4 warps
+            tc::mbar_init(bar.meta_empty(i), 9);   // MMA lane + owning softmax WG + epilogue WG
         }
         tc::mbar_init(bar.drain(), 1);
         *abort_flag = 0;
@@ -174,6 +182,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool ok = true;
         uint32_t kv_loads = 0, q_loads = 0;
         int prev_lidx = -1, kvs = 0;
+        const uint64_t q_policy = tc::l2_policy_evict_last();
         int chunk = 0, i = 0, i_end = 0, li = 0, ends = 0;
         // register windows over the item and list arrays (both are consumed in
         // order, so one coalesced warp load serves many items)
@@ -246,23 +255,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 m.kvs = kvs;
                 const int tokv = list_at(it.y, m.n);
                 for (int tt = 0; tt < MAX_TOK; ++tt) m.tok[tt] = __shfl_sync(0xffffffffu, tokv, tt);
-                const int qs = li & 1;
-                if (!bm_warp_wait(bar.q_empty(qs), ((li >> 1) & 1) ^ 1, abort_flag)) {
+                const int qs = li % NQ;
+                if (!bm_warp_wait(bar.q_empty(qs), ((li / NQ) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
                 __syncwarp();
-                // one TMA per (query, 64-column chunk), spread over the lanes
+                // one TMA per (query, 64-column chunk), spread over the lanes; the
+                // query rows are reused by the chunk's other blocks, so keep them in L2
                 for (int e = lane; e < m.n * L::QC; e += 32) {
                     const int tt = e / L::QC, c = e % L::QC;
-                    tc::tma_load_4d(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
-                                    &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b);
+                    tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
+                                         &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b,
+                                         q_policy);
                 }
                 ++q_loads;
                 ++i;
             } else {
-                ++ends;    // two end markers, one for each softmax warpgroup
+                ++ends;    // two end markers: each softmax warpgroup sees one
             }
             const int slot = li % NM;
             if (!bm_warp_wait(bar.meta_empty(slot), ((li / NM) & 1) ^ 1, abort_flag)) {
@@ -283,9 +294,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t last = s + ((kv_loads - 1 - s) / 2) * 2;
                 tc::mbar_wait(bar.kv_full(s), (last >> 1) & 1, &never, WAIT_NS);
             }
+        }
+        for (uint32_t s = 0; s < NQ; ++s) {
             if (q_loads > s) {
-                const uint32_t last = s + ((q_loads - 1 - s) / 2) * 2;
-                tc::mbar_wait(bar.q_full(s), (last >> 1) & 1, &never, WAIT_NS);
+                const uint32_t last = s + ((q_loads - 1 - s) / NQ) * NQ;
+                tc::mbar_wait(bar.q_full(s), (last / NQ) & 1, &never, WAIT_NS);
             }
         }
     } else if (warp == 1) {
@@ -327,8 +340,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (have_prev && !issue_pv(prev_li, prev_kvs, prev_last)) ok = false;
                     break;
                 }
-                const int qs = li & 1;
-                if (!tc::mbar_wait(bar.q_full(qs), (li >> 1) & 1, abort_flag, WAIT_NS)) {
+                const int qs = li % NQ;
+                if (!tc::mbar_wait(bar.q_full(qs), (li / NQ) & 1, abort_flag, WAIT_NS)) {
                     ok = false;
                     break;
                 }
@@ -367,14 +380,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax + epilogue
-        const int wg = (warp - 2) >> 2;                  // takes items li with li % 2 == wg
+        // ------------------------------------------------------------ softmax (warps 2-5 and
+        // 6-9, alternate items) and epilogue (warps 10-13, every item): the softmax
+        // warpgroups overlap two items while the epilogue drains finished O buffers.
+        const bool is_softmax = warp < 10;
+        const int wg = (warp - 2) >> 2;          // softmax warpgroup 0 / 1 takes items li % 2 == wg
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int tt = r / a.hpt, hl = r % a.hpt;
+        float* row_m = reinterpret_cast<float*>(sm + L::ROW_OFF);    // [2][BM] per O buffer
+        float* row_l = row_m + 2 * BM;
         bool ok = true;
-        for (int li = wg; ok; li += 2) {
+        for (int li = is_softmax ? wg : 0; ok; li += is_softmax ? 2 : 1) {
             const int slot = li % NM;
             if (!bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag)) {
                 ok = false;
@@ -391,76 +409,114 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int qi = tokr >> 5, sl = tokr & 31;
             const int t = a.s.q0 + qi;
             const int sb = li & 1;
-            if (!bm_warp_wait(bar.s_full(sb), (li >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc::fence_after_sync();
-            uint32_t sv[BLK];
-            tc::tmem_ld32(tS(sb) + lane_off, sv);
-            tc::tmem_ld32(tS(sb) + lane_off + 32, sv + 32);
-            tc::tmem_wait_ld();
-            // visible offsets: the whole block, or u <= t inside the query's own block
-            const int hi = row_valid ? min(BLK - 1, t - j * BLK) : -1;
-            float mx[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
-#pragma unroll
-            for (int k = 0; k < BLK; ++k) {
-                const float x = k <= hi ? __uint_as_float(sv[k]) : -INFINITY;
-                sv[k] = __float_as_uint(x);
-                mx[k & 7] = fmaxf(mx[k & 7], x);
-            }
-            const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            const float m = m_raw == -INFINITY ? 0.f : m_raw * a.scale_log2;
-            float ps[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) ps[q] = 0.f;
-#pragma unroll
-            for (int k = 0; k < BLK; k += 2) {
-                const float p0 = tc::ex2(fmaf(__uint_as_float(sv[k]), a.scale_log2, -m));
-                const float p1 = tc::ex2(fmaf(__uint_as_float(sv[k + 1]), a.scale_log2, -m));
-                ps[(k >> 1) & 7] += p0 + p1;
-                sv[k >> 1] = tc::pack_bf16x2(p0, p1);
-            }
-            const float l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-            tc::tmem_st32(tS(sb) + lane_off, sv);
-            tc::tmem_wait_st();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
-
-            // epilogue: o = (P V) / l -> bf16 partial, lse = m + log2(l)
-            if (!bm_warp_wait(bar.o_full(sb), (li >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc::fence_after_sync();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t prow = (((size_t)bu * a.s.Tq + qi) * a.s.topk + sl) * a.hpt + hl;
-#pragma unroll 1
-            for (int c = 0; c < DV; c += 32) {
-                uint32_t o[32];
-                tc::tmem_ld32(tO(sb) + lane_off + c, o);
+            if (is_softmax) {
+                if (!bm_warp_wait(bar.s_full(sb), (li >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                uint32_t sv[BLK];
+                tc::tmem_ld32(tS(sb) + lane_off, sv);
+                tc::tmem_ld32(tS(sb) + lane_off + 32, sv + 32);
                 tc::tmem_wait_ld();
-                if (row_valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(a.part_o + prow * DV + c);
+                // visible offsets: the whole block, or u <= t inside the query's own block
+                const int hi = row_valid ? min(BLK - 1, t - j * BLK) : -1;
+                float m = 0.f, l = 0.f;
+                // P = 2^(s*scale*log2e - m) / l, normalised before the P V product so
+                // the partial o comes out of the MMA already divided by l.  Specialised
+                // on whether any row of the warp needs the causal mask (only items on
+                // a query's own block do).
+                auto softmax_row = [&](auto masked_tag) {
+                    constexpr bool MASKED = decltype(masked_tag)::value;
+                    float mx[8];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 u4;
-                        u4.x = tc::pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-                        u4.y = tc::pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-                        u4.z = tc::pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-                        u4.w = tc::pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-                        dst[q] = u4;
+                    for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < BLK; ++k) {
+                        float x = __uint_as_float(sv[k]);
+                        if (MASKED) {
+                            x = k <= hi ? x : -INFINITY;
+                            sv[k] = __float_as_uint(x);
+                        }
+                        mx[k & 7] = fmaxf(mx[k & 7], x);
+                    }
+                    const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                    m = m_raw == -INFINITY ? 0.f : m_raw * a.scale_log2;
+                    float ps[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+#pragma unroll
+                    for (int k = 0; k < BLK; ++k) {
+                        const float pk = tc::ex2(fmaf(__uint_as_float(sv[k]), a.scale_log2, -m));
+                        ps[k & 7] += pk;
+                        sv[k] = __float_as_uint(pk);
+                    }
+                    l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+                    for (int k = 0; k < BLK; k += 2)
+                        sv[k >> 1] = tc::pack_bf16x2(__uint_as_float(sv[k]) * inv,
+                                                     __uint_as_float(sv[k + 1]) * inv);
+                };
+                if (__all_sync(0xffffffffu, hi == BLK - 1))
+                    softmax_row(std::false_type{});
+                else
+                    softmax_row(std::true_type{});
+                // (m, l) of this item's rows go to the epilogue through shared memory;
+                // buffer sb is free once the epilogue of item li - 2 has released it
+                // (o_free); the p_full arrival below orders these writes before PV(li)
+                // and hence before the epilogue reads them
+                if (li >= 2 && !bm_warp_wait(bar.o_free(sb), ((li >> 1) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                row_m[sb * BM + r] = m;
+                row_l[sb * BM + r] = l;
+                tc::tmem_st32(tS(sb) + lane_off, sv);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
+            } else {
+                // epilogue: o = P V (already divided by l) -> bf16 partial, lse = m + log2(l)
+                if (!bm_warp_wait(bar.o_full(sb), (li >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                // acquire the softmax warpgroup's (m, l) writes directly from its
+                // p_full arrival (already complete, since o_full implies it)
+                if (!bm_warp_wait(bar.p_full(sb), (li >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const float m = row_m[sb * BM + r], l = row_l[sb * BM + r];
+                const size_t prow = (((size_t)bu * a.s.Tq + qi) * a.s.topk + sl) * a.hpt + hl;
+#pragma unroll 1
+                for (int c = 0; c < DV; c += 64) {
+                    uint32_t o[64];
+                    tc::tmem_ld32(tO(sb) + lane_off + c, o);
+                    tc::tmem_ld32(tO(sb) + lane_off + c + 32, o + 32);
+                    tc::tmem_wait_ld();
+                    if (row_valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(a.part_o + prow * DV + c);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint4 u4;
+                            u4.x = tc::pack_bf16x2(__uint_as_float(o[8 * q + 0]), __uint_as_float(o[8 * q + 1]));
+                            u4.y = tc::pack_bf16x2(__uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
+                            u4.z = tc::pack_bf16x2(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]));
+                            u4.w = tc::pack_bf16x2(__uint_as_float(o[8 * q + 6]), __uint_as_float(o[8 * q + 7]));
+                            __stcs(dst + q, u4);       // streamed: read once by the merge
+                        }
                     }
                 }
+                if (row_valid) __stcs(a.part_lse + prow, m + __log2f(l));
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar.o_free(sb));
             }
-            if (row_valid) a.part_lse[prow] = m + __log2f(l);
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar.o_free(sb));
         }
         if (!ok) bm_abort(abort_flag);
     }

@@ -34,6 +34,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -581,11 +583,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                uint32_t sv[SEG];
-                tc::tmem_ld32(tS0 + sb * 128 + lane_off + half * SEG, sv);
-                tc::tmem_ld32(tS0 + sb * 128 + lane_off + half * SEG + 32, sv + 32);
-                tc::tmem_wait_ld();
-
                 // valid key offsets [lo, hi] of this thread's segment for its row
                 int lo = 0, hi = -1;
                 const int s0 = kt.seg[half];
@@ -599,54 +596,69 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         hi = min(SEG - 1, t - s0);
                     }
                 }
-                // masked max of the raw scores, 8 independent chains
-                float mx[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
                 if (hi < lo) lo = hi = SEG;    // empty: no offset 0..63 matches
-                const uint32_t span = (uint32_t)(hi - lo);
-#pragma unroll
-                for (int j = 0; j < SEG; ++j) {
-                    const bool v = (uint32_t)(j - lo) <= span;
-                    const float x = v ? __uint_as_float(sv[j]) : -INFINITY;
-                    sv[j] = __float_as_uint(x);
-                    mx[j & 7] = fmaxf(mx[j & 7], x);
-                }
-                float m_half = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                // exchange with the other half of the row; after this barrier both
-                // halves have finished reading S, so P may overwrite it
-                xmax[((gi & 1) * 2 + half) * BM + r] = m_half;
-                named_sync_softmax();
-                const float m_raw = fmaxf(m_half, xmax[((gi & 1) * 2 + (half ^ 1)) * BM + r]);
-                // scale > 0, so the scaled max is the max of the scaled scores
-                const float m_tile = m_raw * a.scale_log2;
                 const bool new_branch = kt.first != 0;
-                float m_use = new_branch ? -INFINITY : m_ref;
-                float alpha = 1.f;
+                float m_use = 0.f, alpha = 1.f, psum = 0.f;
                 bool rescale = false;
-                if (m_tile != -INFINITY) {
-                    if (m_use == -INFINITY) {
-                        m_use = m_tile;
-                    } else if (m_tile > m_use + 8.f) {
-                        alpha = tc::ex2(m_use - m_tile);
-                        rescale = true;
-                        m_use = m_tile;
+                uint32_t sv[SEG];
+                // One tile of this half-row, specialised on whether any row of the
+                // warp needs a mask (interior tiles of the compressed and window
+                // branches are fully visible).
+                auto half_row = [&](auto masked_tag) {
+                    constexpr bool MASKED = decltype(masked_tag)::value;
+                    tc::tmem_ld32(tS0 + sb * 128 + lane_off + half * SEG, sv);
+                    tc::tmem_ld32(tS0 + sb * 128 + lane_off + half * SEG + 32, sv + 32);
+                    tc::tmem_wait_ld();
+                    float mx[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+                    const uint32_t span = (uint32_t)(hi - lo);
+#pragma unroll
+                    for (int k = 0; k < SEG; ++k) {
+                        float x = __uint_as_float(sv[k]);
+                        if (MASKED) {
+                            x = (uint32_t)(k - lo) <= span ? x : -INFINITY;
+                            sv[k] = __float_as_uint(x);
+                        }
+                        mx[k & 7] = fmaxf(mx[k & 7], x);
                     }
-                }
-                // p = 2^(s*scale*log2e - m); masked scores are -inf and give 0
-                const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
-                float ps[8];
+                    const float m_half = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                    // exchange with the other half of the row; after this barrier both
+                    // halves have finished reading S, so P may overwrite it
+                    xmax[((gi & 1) * 2 + half) * BM + r] = m_half;
+                    named_sync_softmax();
+                    const float m_raw = fmaxf(m_half, xmax[((gi & 1) * 2 + (half ^ 1)) * BM + r]);
+                    // scale > 0, so the scaled max is the max of the scaled scores
+                    const float m_tile = m_raw * a.scale_log2;
+                    m_use = new_branch ? -INFINITY : m_ref;
+                    if (m_tile != -INFINITY) {
+                        if (m_use == -INFINITY) {
+                            m_use = m_tile;
+                        } else if (m_tile > m_use + 8.f) {
+                            alpha = tc::ex2(m_use - m_tile);
+                            rescale = true;
+                            m_use = m_tile;
+                        }
+                    }
+                    // p = 2^(s*scale*log2e - m); masked scores are -inf and give 0
+                    const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
+                    float ps[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+                    for (int q = 0; q < 8; ++q) ps[q] = 0.f;
 #pragma unroll
-                for (int j = 0; j < SEG; j += 2) {
-                    const float p0 = tc::ex2(fmaf(__uint_as_float(sv[j]), a.scale_log2, neg_m));
-                    const float p1 = tc::ex2(fmaf(__uint_as_float(sv[j + 1]), a.scale_log2, neg_m));
-                    ps[(j >> 1) & 7] += p0 + p1;
-                    sv[j >> 1] = tc::pack_bf16x2(p0, p1);     // packed in place: j/2 < j
-                }
-                const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                    for (int k = 0; k < SEG; k += 2) {
+                        const float p0 = tc::ex2(fmaf(__uint_as_float(sv[k]), a.scale_log2, neg_m));
+                        const float p1 = tc::ex2(fmaf(__uint_as_float(sv[k + 1]), a.scale_log2, neg_m));
+                        ps[(k >> 1) & 7] += p0 + p1;
+                        sv[k >> 1] = tc::pack_bf16x2(p0, p1);     // packed in place: k/2 < k
+                    }
+                    psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                };
+                if (__all_sync(0xffffffffu, lo == 0 && hi == SEG - 1))
+                    half_row(std::false_type{});
+                else
+                    half_row(std::true_type{});
                 tc::tmem_st32(tS0 + sb * 128 + lane_off + half * 32, sv);
                 tc::tmem_wait_st();
 

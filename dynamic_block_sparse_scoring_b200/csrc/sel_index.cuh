@@ -22,7 +22,7 @@ struct SelIndex {
 // (chunk * B * Hsel + b * Hsel + u) * nb_all + block, chunk = query / SEL_CHUNK.
 // Work items are therefore ordered chunk by chunk, which keeps the queries
 // (and the partial outputs) of one chunk hot in L2 while it is processed.
-constexpr int SEL_CHUNK = 4096;
+constexpr int SEL_CHUNK = 2048;
 inline int sel_chunks(const Shape& s) { return (s.Tq + SEL_CHUNK - 1) / SEL_CHUNK; }
 inline size_t sel_lists_per_chunk(const Shape& s) { return (size_t)s.B * s.Hsel * s.nb_all; }
 

@@ -42,8 +42,8 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(Shape s, const int32_t* 
     for (int sl = 0; sl < MG_MAXK; ++sl) {             // every load of the row issued at once
         lse[sl] = -INFINITY;
         if (sl < nvalid) {
-            lse[sl] = part_lse[(prow0 + sl) * hpt + h];
-            raw[sl] = *reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8);
+            lse[sl] = __ldcs(part_lse + (prow0 + sl) * hpt + h);
+            raw[sl] = __ldcs(reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8));
         }
     }
 #pragma unroll

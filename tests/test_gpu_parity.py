@@ -15,7 +15,8 @@ from oracle import nsa_oracle as O
 pytestmark = pytest.mark.gpu
 
 from dynamic_block_sparse_scoring_b200 import abi
-from tests.parity import GpuRun, check_idx, check_out, f64, SCORE_ATOL, SCORE_RTOL
+from tests.parity import (GpuRun, check_idx, check_out, f64, OUT_MAX_ABS, OUT_MEAN_ABS,
+                          SCORE_ATOL, SCORE_RTOL)
 
 TINY = WORKLOADS["tiny"]
 
@@ -199,5 +200,8 @@ def test_minimal_workspace_path_matches_oracle(name):
     rows = np.arange(wl.seqlen_q)
     ora, _, _ = run.oracle_rows(0, rows, idx=run.idx[0].cpu().numpy())
     check_out(f64(out[0]), ora, f"{name} minimal workspace")
-    # the two selected-branch organisations agree with each other as well
-    check_out(f64(out[0]), f64(run.out[0]), f"{name} query-major vs block-major")
+    # the two selected-branch organisations agree with each other as well; each is
+    # within the output tolerance of the oracle, so they are within twice it of
+    # each other (a bf16 output of magnitude 2-4 can round one ulp = 0.0156 apart)
+    err = np.abs(f64(out[0]) - f64(run.out[0]))
+    assert err.max() <= 2 * OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS

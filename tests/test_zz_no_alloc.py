@@ -40,10 +40,13 @@ def _forward_pair(wl, seed):
     return ref.double().cpu().numpy(), got.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("name", ["tiny", "nsa_small"])
+# The regular entry point uses the same kernels as the no-alloc one on these
+# problems (16 heads per group over 192 queries of a 2048-token cache, and the
+# tiny single-group problem), so the two results are compared directly.
+@pytest.mark.parametrize("name", ["tiny", "nsa_chunk"])
 def test_noalloc_matches_regular_entry_point_twice_in_a_row(name):
     wl = WORKLOADS["tiny"] if name == "tiny" else WORKLOADS["nsa64k"].with_(
-        name="nsa_small", seqlen_q=2048, seqlen_kv=2048, h_q=16, h_kv=1)
+        name="nsa_chunk", seqlen_q=192, seqlen_kv=2048, q_pos0=2048 - 192, h_q=16, h_kv=1)
     for seed in (0, 1):                  # two calls in a row on the shared scratch array
         ref, got = _forward_pair(wl, seed)
         assert np.isfinite(got).all()
