@@ -203,13 +203,11 @@ class Prefill:
         self.launches_per_step = 0
 
     def attn_launches(self) -> int:
-        """Kernels nsa_sparse_attn_fwd launches with an external idx: the block-major
-        selected branch adds the index build (count, scan, fill, items), its attention
-        kernel and the partial merge in front of the query-major kernel."""
-        wl = self.wl
-        minimal = self.abi.nsa_workspace_size_min(self.cfg)
-        block_major = (wl.branches & 2) and self.ws_bytes > minimal
-        return 7 if block_major else 1
+        """Kernels nsa_sparse_attn_fwd launches with an external idx (the library reports
+        its own plan: block-major adds the index build, its attention kernel and the
+        partial merge; split-K adds the split merge)."""
+        self.path, n = self.abi.nsa_attn_plan(self.cfg, False, self.ws_bytes)
+        return n
 
     def step(self, ev=None, pool=True):
         a, x, p = self.abi, self.x, self.pooled

@@ -58,6 +58,8 @@ _SIGS = {
     "nsa_sparse_attn_fwd": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "nsa_sparse_attn_fwd_noalloc": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "nsa_get_device_status": [ctypes.POINTER(ctypes.c_int32)],
+    "nsa_attn_plan": [_cfgp, ctypes.c_int, _sz, ctypes.POINTER(ctypes.c_int32),
+                      ctypes.POINTER(ctypes.c_int32)],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
@@ -104,6 +106,17 @@ def _check(fn: str, status: int):
 
 def nsa_status_string(status: int) -> str:
     return lib.nsa_status_string(status).decode()
+
+
+PATHS = {0: "rowwise", 1: "query-major", 2: "block-major", 3: "split-k"}
+
+
+def nsa_attn_plan(cfg: NsaConfig, select_inside: bool, ws_bytes: int):
+    """(path name, kernels launched) nsa_sparse_attn_fwd uses for this call shape."""
+    path, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("nsa_attn_plan", lib.nsa_attn_plan(ctypes.byref(cfg), int(select_inside), ws_bytes,
+                                              ctypes.byref(path), ctypes.byref(n)))
+    return PATHS[path.value], n.value
 
 
 def nsa_get_device_status() -> int:

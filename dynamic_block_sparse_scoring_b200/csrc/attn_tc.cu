@@ -34,6 +34,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -80,6 +81,15 @@ struct TcArgs {
     // bf16 (ungated); null = the selected branch runs here over the union of
     // the tile's block sets
     const __nv_bfloat16* o_sel;
+    // split-K (few work tiles, e.g. decode): each tile's key tiles are cut into
+    // n_split contiguous shares processed by different CTAs; each writes, per row
+    // and branch, o = O/l (fp32) and lse = m + log2(l) (scaled log2 units) to
+    // split_o [B, Tq, Hq, 3, n_split, d_v] / split_lse [B, Tq, Hq, 3, n_split]
+    // (lse = -inf: no key of that branch in this share), merged by
+    // split_merge_kernel.  n_split = 1: no split, the gated output is written here.
+    int n_split;
+    float* split_o;
+    float* split_lse;
 };
 
 template <int DQK, int DV>
@@ -284,8 +294,9 @@ struct Producer {
         uint32_t wt = 0;
         uint32_t* keys = reinterpret_cast<uint32_t*>(sm + L::UNION_OFF);
         uint32_t* members = keys + MAX_UNION / 2;
-        for (int work = cta; work < a.n_work; work += ncta, ++wt) {
-            const WorkTile w = decode_work(a, work);
+        for (int work = cta; work < a.n_work * a.n_split; work += ncta, ++wt) {
+            const WorkTile w = decode_work(a, work % a.n_work);
+            const int split = work / a.n_work;
             const int t_last = w.t0 + w.ntok - 1;
             // the selected blocks' union first: the sort overlaps the pipeline drain
             const bool sel_here = (a.s.flags & NSA_BR_SEL) && a.o_sel == nullptr;
@@ -300,12 +311,26 @@ struct Producer {
             ++q_loads;
             KeyTile kt;
             kt.pad[0] = kt.pad[1] = 0;
+            // key tiles of the three branches, numbered 0..n_total-1 in emission
+            // order; this work item emits the tiles of its split share only
+            int nvis = 0;
             if (a.s.flags & NSA_BR_CMP) {
-                int nvis = t_last - a.s.lc + 1 < 0 ? 0 : (t_last - a.s.lc + 1) / a.s.sc + 1;
+                nvis = t_last - a.s.lc + 1 < 0 ? 0 : (t_last - a.s.lc + 1) / a.s.sc + 1;
                 nvis = min(nvis, a.s.n_cmp);
-                for (int j0 = 0; j0 < nvis; j0 += BN) {
+            }
+            const int nseg_sel = sel_here ? nu * (a.s.bs / SEG) : 0;
+            const int win_lo = max(0, w.t0 - a.s.win + 1);
+            const int n_tiles = (nvis + BN - 1) / BN + (nseg_sel + 1) / 2 +
+                                ((a.s.flags & NSA_BR_WIN) ? (t_last - win_lo + BN) / BN : 0);
+            const int g_lo = (int)((long long)split * n_tiles / a.n_split);
+            const int g_hi = (int)((long long)(split + 1) * n_tiles / a.n_split);
+            int g = 0;
+            if (a.s.flags & NSA_BR_CMP) {
+                const int g_br = max(g, g_lo);      // first tile of this branch in the share
+                for (int j0 = 0; j0 < nvis; j0 += BN, ++g) {
+                    if (g < g_lo || g >= g_hi) continue;
                     kt.br = BR_CMP;
-                    kt.first = j0 == 0;
+                    kt.first = g == g_br;
                     kt.seg[0] = j0;
                     kt.seg[1] = j0 + SEG < nvis ? j0 + SEG : -1;
                     kt.member[0] = kt.member[1] = 0xFFFFFFFFu;
@@ -314,10 +339,12 @@ struct Producer {
             }
             if (sel_here) {
                 const int segs_per_blk = a.s.bs / SEG;
-                const int nseg = nu * segs_per_blk;
-                for (int sgi = 0; sgi < nseg; sgi += 2) {
+                const int nseg = nseg_sel;
+                const int g_br = max(g, g_lo);
+                for (int sgi = 0; sgi < nseg; sgi += 2, ++g) {
+                    if (g < g_lo || g >= g_hi) continue;
                     kt.br = BR_SEL;
-                    kt.first = sgi == 0;
+                    kt.first = g == g_br;
                     for (int h = 0; h < 2; ++h) {
                         const int q = sgi + h;
                         if (q < nseg) {
@@ -333,10 +360,12 @@ struct Producer {
                 }
             }
             if (a.s.flags & NSA_BR_WIN) {
-                const int lo = max(0, w.t0 - a.s.win + 1);
-                for (int u0 = lo; u0 <= t_last; u0 += BN) {
+                const int lo = win_lo;
+                const int g_br = max(g, g_lo);
+                for (int u0 = lo; u0 <= t_last; u0 += BN, ++g) {
+                    if (g < g_lo || g >= g_hi) continue;
                     kt.br = BR_WIN;
-                    kt.first = u0 == lo;
+                    kt.first = g == g_br;
                     kt.seg[0] = u0;
                     kt.seg[1] = u0 + SEG <= t_last ? u0 + SEG : -1;
                     kt.member[0] = kt.member[1] = 0xFFFFFFFFu;
@@ -437,7 +466,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t v_base = tc::smem_u32(sm + L::V_OFF);
             uint32_t gm = 0, gi = 0, wt = 0;
             bool ok = true;
-            for (int work = blockIdx.x; ok && work < a.n_work; work += gridDim.x, ++wt) {
+            for (int work = blockIdx.x; ok && work < a.n_work * a.n_split; work += gridDim.x, ++wt) {
                 if (!tc::mbar_wait(bar.q_full(), wt & 1, abort_flag, WAIT_NS)) { ok = false; break; }
                 bool have_prev = false;
                 uint32_t prev_gi = 0;
@@ -523,8 +552,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         constexpr int DVH = DV / 2;
         uint32_t gm = 0, gi = 0, npv = 0;
         bool ok = true;
-        for (int work = blockIdx.x; ok && work < a.n_work; work += gridDim.x) {
-            const WorkTile w = decode_work(a, work);
+        for (int work = blockIdx.x; ok && work < a.n_work * a.n_split; work += gridDim.x) {
+            const WorkTile w = decode_work(a, work % a.n_work);
+            const int split = work / a.n_work;
+            const bool split_mode = a.n_split > 1;
+            uint32_t visited = 0;                  // branches with at least one tile here
             const int tt = r / a.hpt;
             const int h = w.h0 + r % a.hpt;
             const bool row_valid = tt < w.ntok;
@@ -537,12 +569,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bool acc_has = false, have_prev = false;
             float m_ref = -INFINITY, l = 0.f;      // l: this half's share of the row sum
 
-            // folds gate * O / l of the finished branch into Acc (warp-uniform)
+            // folds gate * O / l of the finished branch into Acc (warp-uniform); in
+            // split mode writes this share's O / l and lse for the row instead
             auto correction = [&](int br) {
                 xsum[half * BM + r] = l;
                 named_sync_softmax();
                 const float lrow = l + xsum[(half ^ 1) * BM + r];
                 named_sync_softmax();
+                if (split_mode) {
+                    const size_t pr = (grow * 3 + br) * a.n_split + split;
+                    const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
+#pragma unroll 1
+                    for (int c = half * DVH; c < (half + 1) * DVH; c += 32) {
+                        uint32_t o[32];
+                        tc::tmem_ld32(tO + lane_off + c, o);
+                        tc::tmem_wait_ld();
+                        if (row_valid) {
+                            float4* dst = reinterpret_cast<float4*>(a.split_o + pr * DV + c);
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4)
+                                dst[q4] = make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
+                                                      __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
+                        }
+                    }
+                    if (row_valid && half == 0)
+                        a.split_lse[pr] = lrow > 0.f ? m_ref + __log2f(lrow) : -INFINITY;
+                    visited |= 1u << br;
+                    return;
+                }
                 float wgt = 0.f;
                 if (row_valid && lrow > 0.f) {
                     const float g = a.gates ? a.gates[grow * 3 + br] : 1.f;
@@ -706,6 +760,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::fence_after_sync();
                 correction(cur_br);
             }
+            if (split_mode) {
+                if (row_valid && half == 0)
+                    for (int br = 0; br < 3; ++br)
+                        if (!(visited & (1u << br)))
+                            a.split_lse[(grow * 3 + br) * a.n_split + split] = -INFINITY;
+                tc::fence_before_sync();
+                continue;
+            }
             // selected branch computed outside: out += g_sel * o_sel
             const bool add_sel = a.o_sel != nullptr && (a.s.flags & NSA_BR_SEL) && row_valid;
             const float g_sel = add_sel ? (a.gates ? a.gates[grow * 3 + 1] : 1.f) : 0.f;
@@ -806,10 +868,14 @@ template <int DQK, int DV>
 cudaError_t launch_tc_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                            const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
-                           const __nv_bfloat16* o_sel, __nv_bfloat16* out, cudaStream_t st) {
+                           const __nv_bfloat16* o_sel, int n_split, float* split_o,
+                           float* split_lse, __nv_bfloat16* out, cudaStream_t st) {
     TcArgs a;
     a.s = s;
     a.o_sel = o_sel;
+    a.n_split = n_split;
+    a.split_o = split_o;
+    a.split_lse = split_lse;
     a.idx = idx;
     a.gates = gates;
     a.out = out;
@@ -835,7 +901,7 @@ cudaError_t launch_tc_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bf
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DQK, DV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int grid = min(a.n_work, nsm);
+    const int grid = min(a.n_work * a.n_split, nsm);
     if (grid <= 0) return cudaSuccess;
     attn_tc_kernel<DQK, DV><<<grid, NTHREADS, smem, st>>>(mq, mk, mv, mkc, mvc, a);
     return cudaGetLastError();
@@ -856,10 +922,12 @@ bool attn_tc_supported(const Shape& s) {
 cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                            const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
-                           const __nv_bfloat16* o_sel, __nv_bfloat16* out, cudaStream_t st) {
+                           const __nv_bfloat16* o_sel, int n_split, float* split_o,
+                           float* split_lse, __nv_bfloat16* out, cudaStream_t st) {
 #define NSA_TC_CASE(A, B)                                                                  \
     if (s.dqk == A && s.dv == B)                                                           \
-        return launch_tc_impl<A, B>(s, q, k, v, kcmp, vcmp, gates, idx, o_sel, out, st);
+        return launch_tc_impl<A, B>(s, q, k, v, kcmp, vcmp, gates, idx, o_sel, n_split,   \
+                                    split_o, split_lse, out, st);
     NSA_TC_CASE(64, 64)
     NSA_TC_CASE(128, 128)
     NSA_TC_CASE(192, 128)
@@ -868,6 +936,73 @@ cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bf
     NSA_TC_CASE(192, 64)
 #undef NSA_TC_CASE
     return cudaErrorInvalidValue;
+}
+
+namespace {
+
+// out[row] = sum_br g_br * (sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M)) over the
+// split shares of each branch (empty branches contribute 0).  One thread per
+// 4 output columns of a (query, head) row.
+__global__ void __launch_bounds__(256) split_merge_kernel(Shape s, int n_split,
+                                                          const float* __restrict__ split_o,
+                                                          const float* __restrict__ split_lse,
+                                                          const float* __restrict__ gates,
+                                                          __nv_bfloat16* __restrict__ out) {
+    const int c4n = s.dv / 4;
+    const size_t nrows = (size_t)s.B * s.Tq * s.Hq;
+    const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= nrows * c4n) return;
+    const size_t row = e / c4n;
+    const int c4 = (int)(e % c4n);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int br = 0; br < 3; ++br) {
+        const uint32_t bit = br == 0 ? NSA_BR_CMP : br == 1 ? NSA_BR_SEL : NSA_BR_WIN;
+        if (!(s.flags & bit)) continue;
+        const float* lse = split_lse + (row * 3 + br) * n_split;
+        float m = -INFINITY;
+        for (int sp = 0; sp < n_split; ++sp) m = fmaxf(m, lse[sp]);
+        if (m == -INFINITY) continue;
+        float wsum = 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < n_split; ++sp) {
+            if (lse[sp] == -INFINITY) continue;
+            const float w = exp2f(lse[sp] - m);
+            wsum += w;
+            const float4 v = reinterpret_cast<const float4*>(split_o + ((row * 3 + br) * n_split + sp) * s.dv)[c4];
+            o.x = fmaf(w, v.x, o.x);
+            o.y = fmaf(w, v.y, o.y);
+            o.z = fmaf(w, v.z, o.z);
+            o.w = fmaf(w, v.w, o.w);
+        }
+        const float g = (gates ? gates[row * 3 + br] : 1.f) / wsum;
+        acc.x = fmaf(g, o.x, acc.x);
+        acc.y = fmaf(g, o.y, acc.y);
+        acc.z = fmaf(g, o.z, acc.z);
+        acc.w = fmaf(g, o.w, acc.w);
+    }
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + row * s.dv + 4 * c4);
+    dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+    dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+}
+
+}  // namespace
+
+int attn_tc_split_count(const Shape& s) {
+    const int hpt = s.heads_per_unit;
+    const int tok = BM / hpt;
+    const int n_work = (s.Tq + tok - 1) / tok * s.B * s.Hsel;
+    // enough work items to cover the SMs about four times over
+    if (n_work >= 2 * 148) return 1;
+    return std::min(16, (4 * 148 + n_work - 1) / n_work);
+}
+
+cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o,
+                               const float* split_lse, const float* gates, __nv_bfloat16* out,
+                               cudaStream_t st) {
+    const size_t n = (size_t)s.B * s.Tq * s.Hq * (s.dv / 4);
+    split_merge_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(s, n_split, split_o, split_lse,
+                                                                     gates, out);
+    return cudaGetLastError();
 }
 
 int read_and_clear_tc_status() {

@@ -87,7 +87,12 @@ bool attn_tc_supported(const Shape& s);
 cudaError_t launch_attn_tc(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                            const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
-                           const __nv_bfloat16* o_sel, __nv_bfloat16* out, cudaStream_t st);
+                           const __nv_bfloat16* o_sel, int n_split, float* split_o,
+                           float* split_lse, __nv_bfloat16* out, cudaStream_t st);
+int attn_tc_split_count(const Shape& s);
+cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o,
+                               const float* split_lse, const float* gates, __nv_bfloat16* out,
+                               cudaStream_t st);
 int read_and_clear_tc_status();
 cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
                              const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st);

@@ -91,7 +91,8 @@ bool use_block_major(const Shape& s) {
 // Workspace regions, each 256-byte aligned, in this order.
 struct WsLayout {
     size_t idx = 0, cnt = 0, off = 0, item_off = 0, cursor = 0, list = 0, items = 0, part_o = 0,
-           part_lse = 0, o_sel = 0, total = 0, minimal = 0;
+           part_lse = 0, o_sel = 0, split_o = 0, split_lse = 0, total = 0, minimal = 0;
+    int n_split = 1;
 };
 
 WsLayout ws_layout(const Shape& s) {
@@ -102,9 +103,17 @@ WsLayout ws_layout(const Shape& s) {
         at = round_up(at + bytes, 256);
         return o;
     };
-    if (!(s.flags & NSA_BR_SEL)) return w;
-    w.idx = take(idx_bytes(s));
+    if (s.flags & NSA_BR_SEL) w.idx = take(idx_bytes(s));
     w.minimal = at;
+    // split-K partials for problems with few work tiles (decode)
+    if (nsa::attn_tc_supported(s) && !use_block_major(s)) {
+        w.n_split = nsa::attn_tc_split_count(s);
+        if (w.n_split > 1) {
+            const size_t rows = (size_t)s.B * s.Tq * s.Hq * 3 * w.n_split;
+            w.split_o = take(rows * s.dv * 4);
+            w.split_lse = take(rows * 4);
+        }
+    }
     if (use_block_major(s)) {
         const size_t L = nsa::sel_lists(s);
         const int tok = 128 / s.heads_per_unit;
@@ -152,6 +161,36 @@ nsa_status nsa_workspace_size(const nsa_config* cfg, size_t* bytes) {
     nsa_status st = make_shape(cfg, &s);
     if (st != NSA_OK) return st;
     *bytes = ws_layout(s).total;
+    return NSA_OK;
+}
+
+// Which organisation nsa_sparse_attn_fwd uses for a call, and how many
+// kernels it launches (shared by the dispatch below and nsa_attn_plan).
+struct Plan {
+    int path;       // NSA_PATH_*
+    int kernels;
+};
+
+Plan make_plan(const Shape& s, bool select_inside, size_t ws_bytes, const WsLayout& wl) {
+    Plan p{NSA_PATH_ROWWISE, 1};
+    if (nsa::attn_tc_supported(s)) {
+        if (use_block_major(s) && ws_bytes >= wl.total) p = {NSA_PATH_BLOCK_MAJOR, 7};
+        else if (wl.n_split > 1 && ws_bytes >= wl.total) p = {NSA_PATH_SPLIT_K, 2};
+        else p = {NSA_PATH_QUERY_MAJOR, 1};
+    }
+    if (select_inside) p.kernels += 1;
+    return p;
+}
+
+nsa_status nsa_attn_plan(const nsa_config* cfg, int select_inside, size_t ws_bytes, int32_t* path,
+                         int32_t* kernels) {
+    if (!path || !kernels) return NSA_ERR_INVALID_ARG;
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    const Plan p = make_plan(s, select_inside && (cfg->flags & NSA_BR_SEL), ws_bytes, ws_layout(s));
+    *path = p.path;
+    *kernels = p.kernels;
     return NSA_OK;
 }
 
@@ -247,10 +286,11 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
         if (st != NSA_OK) return st;
     }
-    if (!nsa::attn_tc_supported(s))
+    const Plan plan = make_plan(s, false, ws ? ws_bytes : 0, wl);
+    if (plan.path == NSA_PATH_ROWWISE)
         return cuda_status(nsa::launch_attn(s, qb, kb, vb, kcb, vcb, gates, sel_idx, ob, cs));
     // block-major selected branch when the workspace holds its index and partials
-    if (use_block_major(s) && ws && ws_bytes >= wl.total) {
+    if (plan.path == NSA_PATH_BLOCK_MAJOR) {
         nsa::SelIndex x;
         x.cnt = reinterpret_cast<int32_t*>(ws + wl.cnt);
         x.off = reinterpret_cast<int32_t*>(ws + wl.off);
@@ -268,9 +308,19 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         __nv_bfloat16* o_sel = reinterpret_cast<__nv_bfloat16*>(ws + wl.o_sel);
         st = cuda_status(nsa::launch_sel_merge(s, sel_idx, part_o, part_lse, o_sel, cs));
         if (st != NSA_OK) return st;
-        return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, o_sel, ob, cs));
+        return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, o_sel, 1,
+                                               nullptr, nullptr, ob, cs));
     }
-    return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr, ob, cs));
+    if (plan.path == NSA_PATH_SPLIT_K) {
+        float* split_o = reinterpret_cast<float*>(ws + wl.split_o);
+        float* split_lse = reinterpret_cast<float*>(ws + wl.split_lse);
+        st = cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr,
+                                             wl.n_split, split_o, split_lse, ob, cs));
+        if (st != NSA_OK) return st;
+        return cuda_status(nsa::launch_split_merge(s, wl.n_split, split_o, split_lse, gates, ob, cs));
+    }
+    return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr, 1,
+                                           nullptr, nullptr, ob, cs));
 }
 
 const char* nsa_last_cuda_error(void) { return g_last_cuda_error; }

@@ -196,6 +196,20 @@ nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, con
  */
 nsa_status nsa_get_device_status(int32_t* status);
 
+/* Organisations of nsa_sparse_attn_fwd (same results, different speed). */
+#define NSA_PATH_ROWWISE 0       /* shapes outside the tensor-core kernels' limits */
+#define NSA_PATH_QUERY_MAJOR 1   /* tensor cores; selected branch over each tile's block union */
+#define NSA_PATH_BLOCK_MAJOR 2   /* + selected branch block-major (long prefills, full workspace) */
+#define NSA_PATH_SPLIT_K 3       /* + each tile's keys split over several CTAs (few tiles, e.g. decode) */
+
+/*
+ * The organisation nsa_sparse_attn_fwd picks for `cfg` with a workspace of
+ * `ws_bytes` bytes, and the number of kernels it launches (select_inside != 0:
+ * idx == NULL, the selection kernel included).  Pure host function.
+ */
+nsa_status nsa_attn_plan(const nsa_config* cfg, int select_inside, size_t ws_bytes,
+                         int32_t* path, int32_t* kernels);
+
 /* CUDA's description of the error behind the calling thread's most recent
  * NSA_ERR_CUDA (a static string; "no error" if there was none). */
 const char* nsa_last_cuda_error(void);

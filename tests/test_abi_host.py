@@ -64,10 +64,15 @@ def test_workspace_sizes(abi):
     wl = WORKLOADS["nsa64k"]
     n = abi.nsa_workspace_size(abi.config(wl))
     assert n >= wl.seqlen_q * wl.h_kv * wl.top_k * wl.group * wl.d_v * 2
-    # decode keeps the selected branch in the query-major kernel: ids only
+    # decode keeps the selected branch in the query-major kernel and splits each
+    # tile's keys over several CTAs (partials + merge)
     wl = WORKLOADS["decode64x64k"]
     cfg = abi.config(wl)
-    assert abi.nsa_workspace_size(cfg) == abi.nsa_workspace_size_min(cfg)
+    assert abi.nsa_attn_plan(cfg, True, abi.nsa_workspace_size(cfg))[0] == "split-k"
+    assert abi.nsa_attn_plan(cfg, True, abi.nsa_workspace_size_min(cfg))[0] == "query-major"
+    assert abi.nsa_attn_plan(abi.config(WORKLOADS["nsa64k"]), True,
+                             abi.nsa_workspace_size(abi.config(WORKLOADS["nsa64k"])))[0] == "block-major"
+    assert abi.nsa_attn_plan(abi.config(WORKLOADS["moba32k"]), True, 0)[0] == "rowwise"
 
 
 @pytest.mark.parametrize("bad,status", [
