@@ -187,7 +187,24 @@ struct Producer {
     uint32_t gm = 0, gk = 0;   // descriptors / key tiles issued so far
     int lane;
 
+    bool prefetch_only = false;     // set for the L2 prefetch pass of a split share
+
     __device__ bool emit(const KeyTile& kt, const WorkTile& w) {
+        if (prefetch_only) {
+            if (kt.br == BR_END) return true;
+            const bool cmp = kt.br == BR_CMP;
+            const int plane = w.b * a.s.Hkv + w.kvh;
+            const int e = lane;                   // one box per lane: 2 segments x (QC + VC) chunks
+            const int per_seg = L::QC + L::VC;
+            if (e < 2 * per_seg) {
+                const int sg = e / per_seg, c = e % per_seg;
+                if (kt.seg[sg] >= 0) {
+                    if (c < L::QC) tc::tma_prefetch_l2_3d(cmp ? mkc : mk, 64 * c, kt.seg[sg], plane);
+                    else tc::tma_prefetch_l2_3d(cmp ? mvc : mv, 64 * (c - L::QC), kt.seg[sg], plane);
+                }
+            }
+            return true;
+        }
         const int slot = gm % NM;
         if (!warp_wait(bar.meta_empty(slot), ((gm / NM) & 1) ^ 1, abort_flag)) return false;
         if (lane == 0) {
@@ -324,6 +341,10 @@ struct Producer {
                                 ((a.s.flags & NSA_BR_WIN) ? (t_last - win_lo + BN) / BN : 0);
             const int g_lo = (int)((long long)split * n_tiles / a.n_split);
             const int g_hi = (int)((long long)(split + 1) * n_tiles / a.n_split);
+            // split shares stream from HBM: first prefetch the share's K/V into L2,
+            // then emit the tiles (two passes over the same enumeration)
+            for (int pass = a.n_split > 1 ? 0 : 1; pass < 2; ++pass) {
+            prefetch_only = pass == 0;
             int g = 0;
             if (a.s.flags & NSA_BR_CMP) {
                 const int g_br = max(g, g_lo);      // first tile of this branch in the share
@@ -372,6 +393,8 @@ struct Producer {
                     if (!emit(kt, w)) return false;
                 }
             }
+            }                                   // pass
+            prefetch_only = false;
             kt.br = BR_END;
             kt.first = 0;
             kt.seg[0] = kt.seg[1] = -1;
@@ -991,9 +1014,9 @@ int attn_tc_split_count(const Shape& s) {
     const int hpt = s.heads_per_unit;
     const int tok = BM / hpt;
     const int n_work = (s.Tq + tok - 1) / tok * s.B * s.Hsel;
-    // enough work items to cover the SMs about four times over
+    // enough work items to cover the SMs about eight times over
     if (n_work >= 2 * 148) return 1;
-    return std::min(16, (4 * 148 + n_work - 1) / n_work);
+    return std::min(16, (8 * 148 + n_work - 1) / n_work);
 }
 
 cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o,

@@ -212,6 +212,113 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
     }
 }
 
+// Few query rows (decode): one CTA per (query, unit, sequence).  Each of its
+// 32 warps scores a contiguous range of past blocks (the lanes split the d_qk
+// dot product, so a pooled key row is one coalesced read) and keeps its own
+// running top-(k-1); the warp lists are then merged by warp 0.
+constexpr int SR_NT = 1024;             // 32 warps: more pooled rows in flight per CTA
+constexpr int SR_NW = SR_NT / 32;
+
+__global__ void __launch_bounds__(SR_NT, 1) select_rows_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
+                                                            const float* __restrict__ kbar,
+                                                            int32_t* __restrict__ idx) {
+    __shared__ float qs[256];
+    __shared__ unsigned long long lists[SR_NW][32];
+    const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int d = s.dqk;
+    const int kvh = s.per_head ? u / s.G : u;
+    const int h0 = s.per_head ? u : u * s.G;
+    const int t = s.q0 + i;
+    const int cr = t / s.bs;
+    const int ncand = min(cr, s.nb_full);
+    const int K1 = s.topk - 1;
+    for (int c = tid; c < d; c += SR_NT) {
+        float acc = 0.f;
+        const __nv_bfloat16* src = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d + c;
+        for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += bf2f(src[(size_t)hh * d]);
+        qs[c] = acc;
+    }
+    __syncthreads();
+    unsigned long long key = 0ull;               // this lane's slot of the warp's list
+    unsigned long long thr = 0ull;
+    const int per = (ncand + SR_NW - 1) / SR_NW;
+    const int j0 = warp * per, j1 = min(ncand, j0 + per);
+    const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * d;
+    for (int jb = j0; jb < j1; jb += 32) {
+        // 32 blocks per round: every lane ends up holding the score of block jb + lane
+        float mine = -INFINITY;
+        for (int jj = 0; jj < 32 && jb + jj < j1; jj += 8) {
+            // eight pooled rows in flight at once
+            float part[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                part[e] = 0.f;
+                if (jb + jj + e < j1) {
+                    const float* row = kb + (size_t)(jb + jj + e) * d;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {      // d <= 256: all loads issued together
+                        const int c = lane + 32 * cc;
+                        if (c < d) part[e] = fmaf(qs[c], row[c], part[e]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float tot = warp_sum(part[e]);
+                if (lane == jj + e) mine = s.scale * tot;
+            }
+        }
+        if (K1 > 0) {
+            const unsigned long long ck = (jb + lane < j1) ? score_key(mine, jb + lane) : 0ull;
+            unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
+            while (mask) {
+                const int src = __ffs(mask) - 1;
+                const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
+                const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && key > x));
+                const unsigned long long up = __shfl_up_sync(0xffffffffu, key, 1);
+                if (lane < K1) {
+                    if (lane == p) key = x;
+                    else if (lane > p) key = up;
+                }
+                thr = __shfl_sync(0xffffffffu, key, K1 - 1);
+                mask &= ~(1u << src);
+                mask &= __ballot_sync(0xffffffffu, ck > thr);
+            }
+        }
+    }
+    lists[warp][lane] = key;
+    __syncthreads();
+    if (warp != 0) return;
+    // merge the other warps' lists into warp 0's
+    for (int w = 1; w < SR_NW && K1 > 0; ++w) {
+        const unsigned long long ck = lists[w][lane];
+        unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
+        while (mask) {
+            const int src = __ffs(mask) - 1;
+            const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
+            const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && key > x));
+            const unsigned long long up = __shfl_up_sync(0xffffffffu, key, 1);
+            if (lane < K1) {
+                if (lane == p) key = x;
+                else if (lane > p) key = up;
+            }
+            thr = __shfl_sync(0xffffffffu, key, K1 - 1);
+            mask &= ~(1u << src);
+            mask &= __ballot_sync(0xffffffffu, ck > thr);
+        }
+    }
+    const bool have = lane < K1 && key != 0ull;
+    const int blk = have ? key_block(key) : 0x7fffffff;
+    const int npast = __popc(__ballot_sync(0xffffffffu, have));
+    int rank = 0;
+    for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, blk, o) < blk) ? 1 : 0;
+    int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
+    if (have) dst[rank] = blk;
+    if (lane == 0) dst[npast] = cr;
+    if (lane > npast && lane < s.topk) dst[lane] = -1;
+}
+
 cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
                               const float* scores_in, float* scores_out, int32_t* idx,
                               cudaStream_t st) {
@@ -230,6 +337,9 @@ cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const floa
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         score_topk_kernel<MODE_SELECT_FROM_SCORES><<<grid, ST_NT, smem, st>>>(
             s, nullptr, nullptr, scores_in, nullptr, idx);
+    } else if (s.Tq <= 16) {
+        // few query rows: a 64-row score tile would be mostly empty
+        select_rows_kernel<<<dim3(s.Tq, s.Hsel, s.B), SR_NT, 0, st>>>(s, q, kbar, idx);
     } else {
         cudaFuncSetAttribute(score_topk_kernel<MODE_SELECT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

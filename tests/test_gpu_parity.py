@@ -46,6 +46,10 @@ EDGE = {
                                            h_q=16, h_kv=1),
     "cmp_identity": TINY.with_(name="cmp_identity", seqlen_q=200, seqlen_kv=200, cmp_block=1,
                                cmp_stride=1),
+    # a few queries at the end of a cache (the few-row selection kernel; split-K)
+    "few_queries": TINY.with_(name="few_queries", seqlen_q=5, seqlen_kv=900, q_pos0=895),
+    "decode_small": WORKLOADS["decode64x64k"].with_(name="decode_small", batch=3, seqlen_kv=3000,
+                                                     q_pos0=2999),
     # block-major selected branch (groups of 8 and 16 heads, sel_block 64, >= 256 queries)
     "bm_g8_ragged": WORKLOADS["nsa64k"].with_(name="bm_g8_ragged", seqlen_q=1000, seqlen_kv=1000,
                                               h_q=16, h_kv=2, d_qk=128, d_v=128),
