@@ -82,7 +82,8 @@ struct BmSmem {
     static constexpr int Q_OFF = 0;                                  // NQ stages
     static constexpr int K_OFF = Q_OFF + NQ * QC * CHUNK_Q;           // 2 stages
     static constexpr int V_OFF = K_OFF + 2 * QC * CHUNK_KV;           // 2 stages
-    static constexpr int META_OFF = V_OFF + 2 * VC * CHUNK_KV;
+    static constexpr int STG_OFF = V_OFF + 2 * VC * CHUNK_KV;        // 2 x [BM rows x 128 B]
+    static constexpr int META_OFF = STG_OFF + 2 * BM * 128;
     static constexpr int ROW_OFF = META_OFF + NM * (int)sizeof(ItemMeta);   // row m, l [2][2][BM]
     static constexpr int BAR_OFF = ROW_OFF + 4 * BM * 4;
     // q_full[NQ] q_empty[NQ] kv_full[2] kv_empty[2] meta_full[NM] meta_empty[NM]
@@ -120,7 +121,8 @@ __device__ __forceinline__ void bm_abort(volatile int* abort_flag) {
 template <int DQK, int DV>
 __global__ void __launch_bounds__(NTHREADS, 1)
     sel_bm_kernel(const __grid_constant__ CUtensorMap map_qg, const __grid_constant__ CUtensorMap map_k,
-                  const __grid_constant__ CUtensorMap map_v, const BmArgs a) {
+                  const __grid_constant__ CUtensorMap map_v,
+                  const __grid_constant__ CUtensorMap map_po, const BmArgs a) {
     using L = BmSmem<DQK, DV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -379,20 +381,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 10) {
         // ------------------------------------------------------------ softmax (warps 2-5 and
-        // 6-9, alternate items) and epilogue (warps 10-13, every item): the softmax
-        // warpgroups overlap two items while the epilogue drains finished O buffers.
-        const bool is_softmax = warp < 10;
+        // 6-9, alternate items; S/P double-buffered in TMEM)
         const int wg = (warp - 2) >> 2;          // softmax warpgroup 0 / 1 takes items li % 2 == wg
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const int tt = r / a.hpt, hl = r % a.hpt;
+        const int tt = r / a.hpt;
         float* row_m = reinterpret_cast<float*>(sm + L::ROW_OFF);    // [2][BM] per O buffer
         float* row_l = row_m + 2 * BM;
         bool ok = true;
-        for (int li = is_softmax ? wg : 0; ok; li += is_softmax ? 2 : 1) {
+        for (int li = wg; ok; li += 2) {
             const int slot = li % NM;
             if (!bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag)) {
                 ok = false;
@@ -405,119 +405,171 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
             if (!valid) break;
             const bool row_valid = tt < n;
-            const int bu = (lidx / nb_all) % bhsel, j = lidx % nb_all;
-            const int qi = tokr >> 5, sl = tokr & 31;
-            const int t = a.s.q0 + qi;
+            const int j = lidx % nb_all;
+            const int t = a.s.q0 + (tokr >> 5);
             const int sb = li & 1;
-            if (is_softmax) {
-                if (!bm_warp_wait(bar.s_full(sb), (li >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                uint32_t sv[BLK];
-                tc::tmem_ld32(tS(sb) + lane_off, sv);
-                tc::tmem_ld32(tS(sb) + lane_off + 32, sv + 32);
-                tc::tmem_wait_ld();
-                // visible offsets: the whole block, or u <= t inside the query's own block
-                const int hi = row_valid ? min(BLK - 1, t - j * BLK) : -1;
-                float m = 0.f, l = 0.f;
-                // P = 2^(s*scale*log2e - m) / l, normalised before the P V product so
-                // the partial o comes out of the MMA already divided by l.  Specialised
-                // on whether any row of the warp needs the causal mask (only items on
-                // a query's own block do).
-                auto softmax_row = [&](auto masked_tag) {
-                    constexpr bool MASKED = decltype(masked_tag)::value;
-                    float mx[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
-#pragma unroll
-                    for (int k = 0; k < BLK; ++k) {
-                        float x = __uint_as_float(sv[k]);
-                        if (MASKED) {
-                            x = k <= hi ? x : -INFINITY;
-                            sv[k] = __float_as_uint(x);
-                        }
-                        mx[k & 7] = fmaxf(mx[k & 7], x);
-                    }
-                    const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                    m = m_raw == -INFINITY ? 0.f : m_raw * a.scale_log2;
-                    float ps[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) ps[q] = 0.f;
-#pragma unroll
-                    for (int k = 0; k < BLK; ++k) {
-                        const float pk = tc::ex2(fmaf(__uint_as_float(sv[k]), a.scale_log2, -m));
-                        ps[k & 7] += pk;
-                        sv[k] = __float_as_uint(pk);
-                    }
-                    l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-                    for (int k = 0; k < BLK; k += 2)
-                        sv[k >> 1] = tc::pack_bf16x2(__uint_as_float(sv[k]) * inv,
-                                                     __uint_as_float(sv[k + 1]) * inv);
-                };
-                if (__all_sync(0xffffffffu, hi == BLK - 1))
-                    softmax_row(std::false_type{});
-                else
-                    softmax_row(std::true_type{});
-                // (m, l) of this item's rows go to the epilogue through shared memory;
-                // buffer sb is free once the epilogue of item li - 2 has released it
-                // (o_free); the p_full arrival below orders these writes before PV(li)
-                // and hence before the epilogue reads them
-                if (li >= 2 && !bm_warp_wait(bar.o_free(sb), ((li >> 1) & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                row_m[sb * BM + r] = m;
-                row_l[sb * BM + r] = l;
-                tc::tmem_st32(tS(sb) + lane_off, sv);
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
-            } else {
-                // epilogue: o = P V (already divided by l) -> bf16 partial, lse = m + log2(l)
-                if (!bm_warp_wait(bar.o_full(sb), (li >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                // acquire the softmax warpgroup's (m, l) writes directly from its
-                // p_full arrival (already complete, since o_full implies it)
-                if (!bm_warp_wait(bar.p_full(sb), (li >> 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const float m = row_m[sb * BM + r], l = row_l[sb * BM + r];
-                const size_t prow = (((size_t)bu * a.s.Tq + qi) * a.s.topk + sl) * a.hpt + hl;
-#pragma unroll 1
-                for (int c = 0; c < DV; c += 64) {
-                    uint32_t o[64];
-                    tc::tmem_ld32(tO(sb) + lane_off + c, o);
-                    tc::tmem_ld32(tO(sb) + lane_off + c + 32, o + 32);
-                    tc::tmem_wait_ld();
-                    if (row_valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(a.part_o + prow * DV + c);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            uint4 u4;
-                            u4.x = tc::pack_bf16x2(__uint_as_float(o[8 * q + 0]), __uint_as_float(o[8 * q + 1]));
-                            u4.y = tc::pack_bf16x2(__uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
-                            u4.z = tc::pack_bf16x2(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]));
-                            u4.w = tc::pack_bf16x2(__uint_as_float(o[8 * q + 6]), __uint_as_float(o[8 * q + 7]));
-                            __stcs(dst + q, u4);       // streamed: read once by the merge
-                        }
-                    }
-                }
-                if (row_valid) __stcs(a.part_lse + prow, m + __log2f(l));
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar.o_free(sb));
+            if (!bm_warp_wait(bar.s_full(sb), (li >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
             }
+            tc::fence_after_sync();
+            uint32_t sv[BLK];
+            tc::tmem_ld32(tS(sb) + lane_off, sv);
+            tc::tmem_ld32(tS(sb) + lane_off + 32, sv + 32);
+            tc::tmem_wait_ld();
+            // visible offsets: the whole block, or u <= t inside the query's own block
+            const int hi = row_valid ? min(BLK - 1, t - j * BLK) : -1;
+            float m = 0.f, l = 0.f;
+            // P = 2^(s*scale*log2e - m) / l, normalised before the P V product so
+            // the partial o comes out of the MMA already divided by l.  Specialised
+            // on whether any row of the warp needs the causal mask (only items on
+            // a query's own block do).
+            auto softmax_row = [&](auto masked_tag) {
+                constexpr bool MASKED = decltype(masked_tag)::value;
+                float mx[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < BLK; ++k) {
+                    float x = __uint_as_float(sv[k]);
+                    if (MASKED) {
+                        x = k <= hi ? x : -INFINITY;
+                        sv[k] = __float_as_uint(x);
+                    }
+                    mx[k & 7] = fmaxf(mx[k & 7], x);
+                }
+                const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                m = m_raw == -INFINITY ? 0.f : m_raw * a.scale_log2;
+                float ps[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+#pragma unroll
+                for (int k = 0; k < BLK; ++k) {
+                    const float pk = tc::ex2(fmaf(__uint_as_float(sv[k]), a.scale_log2, -m));
+                    ps[k & 7] += pk;
+                    sv[k] = __float_as_uint(pk);
+                }
+                l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+                for (int k = 0; k < BLK; k += 2)
+                    sv[k >> 1] = tc::pack_bf16x2(__uint_as_float(sv[k]) * inv,
+                                                 __uint_as_float(sv[k + 1]) * inv);
+            };
+            if (__all_sync(0xffffffffu, hi == BLK - 1))
+                softmax_row(std::false_type{});
+            else
+                softmax_row(std::true_type{});
+            // (m, l) of this item's rows go to the epilogue through shared memory;
+            // buffer sb is free once the epilogue of item li - 2 has released it
+            // (o_free); the p_full arrival below orders these writes before PV(li)
+            // and hence before the epilogue reads them
+            if (li >= 2 && !bm_warp_wait(bar.o_free(sb), ((li >> 1) & 1) ^ 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            row_m[sb * BM + r] = m;
+            row_l[sb * BM + r] = l;
+            tc::tmem_st32(tS(sb) + lane_off, sv);
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
         }
+        if (!ok) bm_abort(abort_flag);
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 10-13,
+        // every item): o = P V (already divided by l) -> bf16 partial rows, staged in
+        // shared memory in the 128-byte-swizzled layout and written by TMA stores
+        // (one {64 columns x hpt rows} box per query and column half, whole lines
+        // instead of a 256-byte row per lane); lse = m + log2(l) per row.  The four
+        // warps decide every wait together (barrier reduction), so none of them can
+        // be left alone at a named barrier.
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int tt = r / a.hpt, hl = r % a.hpt;
+        const float* row_m = reinterpret_cast<const float*>(sm + L::ROW_OFF);
+        const float* row_l = row_m + 2 * BM;
+        const bool issuer = warp == 10;           // lane q issues the stores of the item's query q
+        const uint64_t st_policy = tc::l2_policy_evict_first();
+        uint32_t halves = 0;
+        bool ok = true;
+        for (int li = 0;; ++li) {
+            const int slot = li % NM;
+            bool okw = bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag);
+            int valid = 0, lidx = 0, n = 0, tokr = 0, tok_lane = 0;
+            if (okw) {
+                const ItemMeta& mref = metas[slot];
+                valid = mref.valid;
+                lidx = mref.lidx;
+                n = mref.n;
+                tokr = tt < MAX_TOK ? mref.tok[tt] : 0;
+                tok_lane = lane < MAX_TOK ? mref.tok[lane] : 0;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
+            }
+            if (!tc::named_bar_and(1, 128, okw)) {
+                ok = false;
+                break;
+            }
+            if (!valid) break;
+            const int sb = li & 1;
+            okw = bm_warp_wait(bar.o_full(sb), (li >> 1) & 1, abort_flag) &&
+                  // acquire the softmax warpgroup's (m, l) writes directly from its
+                  // p_full arrival (already complete, since o_full implies it)
+                  bm_warp_wait(bar.p_full(sb), (li >> 1) & 1, abort_flag);
+            if (!tc::named_bar_and(1, 128, okw)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const bool row_valid = tt < n;
+            const int bu = (lidx / nb_all) % bhsel;
+            const float m = row_m[sb * BM + r], l = row_l[sb * BM + r];
+            const size_t prow = (((size_t)bu * a.s.Tq + (tokr >> 5)) * a.s.topk + (tokr & 31)) * a.hpt + hl;
+            // first partial row of the query this lane stores (issuer warp)
+            const int prow_q = (int)((((size_t)bu * a.s.Tq + (tok_lane >> 5)) * a.s.topk + (tok_lane & 31)) * a.hpt);
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 64, ++halves) {
+                uint32_t o[64];
+                tc::tmem_ld32(tO(sb) + lane_off + c, o);
+                tc::tmem_ld32(tO(sb) + lane_off + c + 32, o + 32);
+                tc::tmem_wait_ld();
+                if (c + 64 == DV) {
+                    // every column of O(sb) is in registers: MMA may reuse the buffer
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar.o_free(sb));
+                }
+                // staging buffer (halves & 1) was last read by the stores issued two
+                // halves ago; at most the latest group may still be reading
+                if (issuer) tc::bulk_wait_read<1>();
+                tc::named_bar_sync(1, 128);
+                uint8_t* rowp = sm + L::STG_OFF + (halves & 1) * (BM * 128) + r * 128;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    uint4 u4;
+                    u4.x = tc::pack_bf16x2(__uint_as_float(o[8 * q + 0]), __uint_as_float(o[8 * q + 1]));
+                    u4.y = tc::pack_bf16x2(__uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
+                    u4.z = tc::pack_bf16x2(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]));
+                    u4.w = tc::pack_bf16x2(__uint_as_float(o[8 * q + 6]), __uint_as_float(o[8 * q + 7]));
+                    *reinterpret_cast<uint4*>(rowp + ((q ^ (r & 7)) << 4)) = u4;
+                }
+                tc::fence_proxy_async_smem();
+                tc::named_bar_sync(1, 128);
+                if (issuer) {
+                    if (lane < n)
+                        tc::tma_store_2d_hint(&map_po,
+                                              sm + L::STG_OFF + (halves & 1) * (BM * 128) + lane * a.hpt * 128,
+                                              c, prow_q, st_policy);
+                    tc::bulk_commit();
+                }
+            }
+            if (row_valid) __stcs(a.part_lse + prow, m + __log2f(l));
+        }
+        if (issuer) tc::bulk_wait<0>();
         if (!ok) bm_abort(abort_flag);
     }
 
@@ -576,8 +628,13 @@ cudaError_t launch_bm_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bf
     const cuuint64_t vd[3] = {(cuuint64_t)DV, (cuuint64_t)s.Tk, (cuuint64_t)s.B * s.Hkv};
     const cuuint64_t vs[2] = {(cuuint64_t)DV * 2, (cuuint64_t)DV * 2 * s.Tk};
     const cuuint32_t kb[3] = {64, (cuuint32_t)BLK, 1};
+    // partial rows [B * Hsel * Tq * topk * hpt, DV] written in {64, hpt} boxes
+    CUtensorMap mpo;
+    const cuuint64_t pd[2] = {(cuuint64_t)DV, (cuuint64_t)sel_partial_rows(s)};
+    const cuuint64_t ps[1] = {(cuuint64_t)DV * 2};
+    const cuuint32_t pb[2] = {64, (cuuint32_t)a.hpt};
     if (!encode(&mq, q, 4, qd, qs, qb) || !encode(&mk, k, 3, kd, ks, kb) ||
-        !encode(&mv, v, 3, vd, vs, kb))
+        !encode(&mv, v, 3, vd, vs, kb) || !encode(&mpo, part_o, 2, pd, ps, pb))
         return cudaErrorInvalidValue;
     int dev = 0, nsm = 148;
     cudaGetDevice(&dev);
@@ -586,7 +643,7 @@ cudaError_t launch_bm_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bf
     cudaError_t e = cudaFuncSetAttribute(sel_bm_kernel<DQK, DV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    sel_bm_kernel<DQK, DV><<<nsm, NTHREADS, smem, st>>>(mq, mk, mv, a);
+    sel_bm_kernel<DQK, DV><<<nsm, NTHREADS, smem, st>>>(mq, mk, mv, mpo, a);
     return cudaGetLastError();
 }
 
@@ -598,7 +655,8 @@ bool sel_bm_supported(const Shape& s) {
     if (s.dv != 64 && s.dv != 128) return false;
     if (s.bs != BLK) return false;
     const int hpt = s.heads_per_unit;
-    return (hpt == 8 || hpt == 16) && s.topk <= 16;
+    // partial rows are addressed by 32-bit TMA coordinates
+    return (hpt == 8 || hpt == 16) && s.topk <= 16 && sel_partial_rows(s) < (size_t(1) << 31);
 }
 
 cudaError_t launch_sel_bm(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,

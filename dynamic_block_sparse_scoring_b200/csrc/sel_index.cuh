@@ -28,6 +28,8 @@ inline size_t sel_lists_per_chunk(const Shape& s) { return (size_t)s.B * s.Hsel 
 
 // Upper bounds used to size the workspace.
 inline size_t sel_pairs_max(const Shape& s) { return (size_t)s.B * s.Hsel * s.Tq * s.topk; }
+// rows of the selected-branch partial buffers: one per (pair, head of the unit)
+inline size_t sel_partial_rows(const Shape& s) { return sel_pairs_max(s) * s.heads_per_unit; }
 inline size_t sel_lists(const Shape& s) { return (size_t)sel_chunks(s) * sel_lists_per_chunk(s); }
 // (+32 / +64 slack entries: the block-major producer reads 32 items / 64 list
 // entries at a time past the last valid one)
