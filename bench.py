@@ -41,8 +41,16 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # FP32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (max SM clock)
 ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-ATTN_KERNEL = "attn_tc_kernel"
-ATTN_SOURCE = os.path.join(ROOT, "dynamic_block_sparse_scoring_b200", "csrc", "attn_tc.cu")
+CSRC = os.path.join(ROOT, "dynamic_block_sparse_scoring_b200", "csrc")
+# stage name reported by nsa_timing_read -> (kernel, source file) for the ncu traffic record
+STAGE_KERNELS = {
+    "attn_tc": ("attn_tc_kernel", os.path.join(CSRC, "attn_tc.cu")),
+    "sel_bm": ("sel_bm_kernel", os.path.join(CSRC, "attn_sel_bm.cu")),
+    "sel_merge": ("sel_merge_kernel", os.path.join(CSRC, "sel_merge.cu")),
+    "index": ("sel_index", os.path.join(CSRC, "sel_index.cu")),
+    "split_merge": ("split_merge_kernel", os.path.join(CSRC, "attn_tc.cu")),
+    "rowwise": ("attn_rowwise_kernel", os.path.join(CSRC, "attn_rowwise.cu")),
+}
 
 
 # ---------------------------------------------------------------------------
@@ -248,24 +256,70 @@ def max_over_ranks(v: float, world: int) -> float:
 
 
 def timed_steps(pf: Prefill, steps: int, warmup: int, world: int, pool=True):
+    """Per-step device times (pool, select, attention) and the mean time of every stage
+    inside the attention call (the library's stage events on the launching stream; the
+    host reads them between steps, outside the steps' own events)."""
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     for _ in range(warmup):
         flush.fill_(1.0)
         pf.step(pool=pool)
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    stages = {}
     barrier(world)
     torch.cuda.synchronize()
+    pf.abi.nsa_timing_enable(True)
     wall0 = time.perf_counter()
     for s in range(steps):
         flush.fill_(float(s))
         pf.step(evs[s], pool=pool)
+        for name, ms in pf.abi.nsa_timing_read():
+            stages.setdefault(name, []).append(ms)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    pf.abi.nsa_timing_enable(False)
     barrier(world)
     per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
                     for e in evs])                                     # ms: pool, select, attn
-    return per, wall
+    return per, wall, {k: float(np.mean(v)) for k, v in stages.items()}
+
+
+def stage_rooflines(wl: Workload, path: str, stage_ms: dict, idx: torch.Tensor, pk: dict) -> dict:
+    """Algorithmic work of every attention stage over its measured mean duration.
+
+    Tensor-core stages count the branch FLOPs they compute (block-major: the selected
+    branch in sel_bm, window + compressed in attn_tc; otherwise attn_tc does all three).
+    The index and merge stages are HBM-bound: they count the bytes they must move."""
+    fl = algorithmic_flops(wl)
+    B = wl.batch
+    idx_bytes = idx.numel() * 4
+    n_valid = int((idx >= 0).sum().item()) if wl.branches & 2 else 0
+    out = {}
+    for name, ms in stage_ms.items():
+        if ms <= 0:
+            continue
+        if name in ("attn_tc", "sel_bm", "rowwise"):
+            if name == "sel_bm":
+                work = fl.get("sel", 0.0) * B
+            elif path == "block-major":
+                work = (fl.get("win", 0.0) + fl.get("cmp", 0.0)) * B
+            else:
+                work = (fl["total"] - fl["score"]) * B
+            ach = work / (ms / 1e3) / 1e12
+            out[name] = {"ms": ms, "bound": "tensor", "unit": "TFLOP/s", "work": work,
+                         "achieved": ach, "peak": pk["bf16_tflops"], "frac": ach / pk["bf16_tflops"]}
+        else:
+            hpt = wl.h_q // wl.h_sel
+            if name == "sel_merge":      # read every valid partial (o bf16 + lse), write o_sel
+                work = n_valid * hpt * (2 * wl.d_v + 4) + B * wl.seqlen_q * wl.h_q * wl.d_v * 2 + idx_bytes
+            elif name == "index":        # read idx twice, write the pair lists
+                work = 2 * idx_bytes + n_valid * 4
+            else:                        # split merge: fp32 (o, l, m) per split, branch and row
+                work = 0.0
+            ach = work / (ms / 1e3) / 1e9
+            out[name] = {"ms": ms, "bound": "hbm", "unit": "GB/s", "work": work,
+                         "achieved": ach, "peak": pk["hbm_gbs"], "frac": ach / pk["hbm_gbs"]}
+    return out
 
 
 def e2e_steps(pf: Prefill, steps: int, warmup: int, world: int):
@@ -355,7 +409,7 @@ def run_decode(world: int, steps: int, warmup: int):
     pf = Prefill(wl, seed=1000 + (torch.distributed.get_rank() if world > 1 else 0))
     pf.step()                        # pooled cache built once (cache maintenance, not timed)
     torch.cuda.synchronize()
-    per, _ = timed_steps(pf, steps, warmup, world, pool=False)
+    per, _, _ = timed_steps(pf, steps, warmup, world, pool=False)
     ms = max_over_ranks(float(per[:, 1:].sum(axis=1).mean()), world)
     nbytes = decode_bytes(wl, pf.idx)
     pk, _ = peaks()
@@ -380,25 +434,34 @@ def run_ours(args):
     clocks = ClockSampler(torch.cuda.current_device())
     # warm-up and timed region (clocks sampled during it)
     clocks.start()
-    per, wall = timed_steps(pf, args.steps, args.warmup, world)
+    per, wall, stage_ms = timed_steps(pf, args.steps, args.warmup, world)
     clk = clocks.stop()
     step_ms = per.sum(axis=1)
     ms = max_over_ranks(float(step_ms.mean()), world)
-    attn_ms = max_over_ranks(float(per[:, 2].mean()), world)
     fl = algorithmic_flops(wl)
     fl_all = fl["total"] * wl.batch * world
     value = fl_all / (ms / 1e3) / 1e12
     tokens = wl.seqlen_q * wl.batch * world / (ms / 1e3)
     pk, src = peaks()
-    attn_flops = (fl["total"] - fl["score"]) * wl.batch
-    achieved = attn_flops / (attn_ms / 1e3) / 1e12
-    peak = pk["bf16_tflops"]
-    roof = {"kernel": ATTN_KERNEL, "bound": "tensor", "achieved": achieved,
-            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": traffic_for(ATTN_KERNEL, ATTN_SOURCE),
-            "peak_source": f"{src} dense bf16 (burst, cuBLAS)",
-            "flops_per_launch": attn_flops,
-            "share_of_step": float(per[:, 2].mean() / step_ms.mean())}
+    pf.attn_launches()
+    stages = stage_rooflines(wl, pf.path, stage_ms, pf.idx, pk)
+    stage_ms_all = {k: max_over_ranks(v["ms"], world) for k, v in stages.items()}
+    dom = max(stages, key=lambda k: stages[k]["ms"])
+    d = dict(stages[dom])
+    d["achieved"] *= d["ms"] / stage_ms_all[dom]       # slowest rank
+    d["frac"] = d["achieved"] / d["peak"]
+    kernel, source = STAGE_KERNELS[dom]
+    roof = {"kernel": kernel, "stage": dom, "bound": d["bound"], "achieved": d["achieved"],
+            "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+            "traffic": traffic_for(kernel, source),
+            "peak_source": f"{src} " + ("dense bf16 (burst, cuBLAS)" if d["bound"] == "tensor"
+                                        else "HBM copy"),
+            ("flops_per_launch" if d["bound"] == "tensor" else "bytes_per_launch"): d["work"],
+            "launch_ms": stage_ms_all[dom],
+            "share_of_step": float(stage_ms[dom] / step_ms.mean()),
+            "path": pf.path,
+            "stages": {k: {"ms": v["ms"], "achieved": v["achieved"], "unit": v["unit"],
+                           "frac": v["frac"], "bound": v["bound"]} for k, v in stages.items()}}
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_steps(pf, max(2, args.steps // 2), 1, world)

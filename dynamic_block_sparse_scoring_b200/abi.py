@@ -60,6 +60,9 @@ _SIGS = {
     "nsa_get_device_status": [ctypes.POINTER(ctypes.c_int32)],
     "nsa_attn_plan": [_cfgp, ctypes.c_int, _sz, ctypes.POINTER(ctypes.c_int32),
                       ctypes.POINTER(ctypes.c_int32)],
+    "nsa_timing_enable": [ctypes.c_int32],
+    "nsa_timing_read": [ctypes.c_int32, ctypes.POINTER(ctypes.c_float),
+                        ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_int32)],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
@@ -124,6 +127,23 @@ def nsa_get_device_status() -> int:
     v = ctypes.c_int32(0)
     _check("nsa_get_device_status", lib.nsa_get_device_status(ctypes.byref(v)))
     return v.value
+
+
+TIMING_MAX_STAGES = 8
+
+
+def nsa_timing_enable(on: bool):
+    """Start / stop recording stage events in this thread's nsa_sparse_attn_fwd calls."""
+    _check("nsa_timing_enable", lib.nsa_timing_enable(int(bool(on))))
+
+
+def nsa_timing_read():
+    """[(stage name, ms)] of this thread's most recent timed nsa_sparse_attn_fwd call."""
+    ms = (ctypes.c_float * TIMING_MAX_STAGES)()
+    names = (ctypes.c_char_p * TIMING_MAX_STAGES)()
+    n = ctypes.c_int32(0)
+    _check("nsa_timing_read", lib.nsa_timing_read(TIMING_MAX_STAGES, ms, names, ctypes.byref(n)))
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n.value, TIMING_MAX_STAGES))]
 
 
 def nsa_workspace_size(cfg: NsaConfig) -> int:

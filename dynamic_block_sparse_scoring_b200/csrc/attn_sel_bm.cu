@@ -17,9 +17,9 @@
 // query's own block, where key u is visible iff u <= t.  Each row writes a
 // partial result for its (query, slot): o = (P V)/l in bf16 and
 // lse = m + log2(l) in the scaled-log2 domain.  The partials of a query's
-// slots are merged by sel_merge.cu.  Items come chunk by chunk (2048
-// queries); every CTA takes a contiguous share of each chunk, so the chunk's
-// queries stay in L2 while consecutive items of a CTA share their K/V block.
+// slots are merged by sel_merge.cu.  Items come chunk by chunk (SEL_CHUNK
+// queries); every CTA takes a contiguous share of each chunk, so consecutive
+// items of a CTA share their K/V block.
 //
 // Roles (448 threads): warp 0 TMA producer (K/V once per run of items on the
 // same block, Q rows per item), warp 1 MMA lane + TMEM owner, warps 2-5 and

@@ -139,6 +139,50 @@ nsa_status cuda_status(cudaError_t e) {
     return NSA_ERR_CUDA;
 }
 
+// Per-host-thread stage events for nsa_timing_enable / nsa_timing_read.
+struct StageTiming {
+    bool on = false;
+    bool created = false;
+    int dev = -1;
+    cudaEvent_t ev[NSA_TIMING_MAX_STAGES + 1];
+    const char* names[NSA_TIMING_MAX_STAGES];
+    int n = 0;             // stages recorded by the current / most recent call
+    bool closed = false;   // the most recent call recorded its final event
+    bool active = false;   // the current call records
+
+    void begin() {
+        n = 0;
+        closed = false;
+        active = false;
+        if (!on || !created) return;
+        int d = -1;
+        active = cudaGetDevice(&d) == cudaSuccess && d == dev;
+    }
+    void mark(const char* name, cudaStream_t st) {
+        if (!active || n >= NSA_TIMING_MAX_STAGES) return;
+        if (cudaEventRecord(ev[n], st) != cudaSuccess) {
+            active = false;
+            n = 0;
+            return;
+        }
+        names[n++] = name;
+    }
+    void end(cudaStream_t st) {
+        if (!active) return;
+        closed = n > 0 && cudaEventRecord(ev[n], st) == cudaSuccess;
+        if (!closed) n = 0;
+        active = false;
+    }
+};
+thread_local StageTiming g_timing;
+
+// Records the end of the timed call on every return path of nsa_sparse_attn_fwd.
+struct TimingScope {
+    cudaStream_t st;
+    explicit TimingScope(cudaStream_t s) : st(s) { g_timing.begin(); }
+    ~TimingScope() { g_timing.end(st); }
+};
+
 }  // namespace
 
 extern "C" {
@@ -282,13 +326,17 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
     const __nv_bfloat16* kcb = static_cast<const __nv_bfloat16*>(kcmp);
     const __nv_bfloat16* vcb = static_cast<const __nv_bfloat16*>(vcmp);
     __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out);
+    TimingScope timing(cs);
     if (sel && !idx) {
+        g_timing.mark("select", cs);
         st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
         if (st != NSA_OK) return st;
     }
     const Plan plan = make_plan(s, false, ws ? ws_bytes : 0, wl);
-    if (plan.path == NSA_PATH_ROWWISE)
+    if (plan.path == NSA_PATH_ROWWISE) {
+        g_timing.mark("rowwise", cs);
         return cuda_status(nsa::launch_attn(s, qb, kb, vb, kcb, vcb, gates, sel_idx, ob, cs));
+    }
     // block-major selected branch when the workspace holds its index and partials
     if (plan.path == NSA_PATH_BLOCK_MAJOR) {
         nsa::SelIndex x;
@@ -301,26 +349,71 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         __nv_bfloat16* part_o = reinterpret_cast<__nv_bfloat16*>(ws + wl.part_o);
         float* part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
         const int tok = 128 / s.heads_per_unit;
+        g_timing.mark("index", cs);
         st = cuda_status(nsa::launch_sel_index(s, sel_idx, x, tok, cs));
         if (st != NSA_OK) return st;
+        g_timing.mark("sel_bm", cs);
         st = cuda_status(nsa::launch_sel_bm(s, qb, kb, vb, x, part_o, part_lse, cs));
         if (st != NSA_OK) return st;
         __nv_bfloat16* o_sel = reinterpret_cast<__nv_bfloat16*>(ws + wl.o_sel);
+        g_timing.mark("sel_merge", cs);
         st = cuda_status(nsa::launch_sel_merge(s, sel_idx, part_o, part_lse, o_sel, cs));
         if (st != NSA_OK) return st;
+        g_timing.mark("attn_tc", cs);
         return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, o_sel, 1,
                                                nullptr, nullptr, ob, cs));
     }
     if (plan.path == NSA_PATH_SPLIT_K) {
         float* split_o = reinterpret_cast<float*>(ws + wl.split_o);
         float* split_lse = reinterpret_cast<float*>(ws + wl.split_lse);
+        g_timing.mark("attn_tc", cs);
         st = cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr,
                                              wl.n_split, split_o, split_lse, ob, cs));
         if (st != NSA_OK) return st;
+        g_timing.mark("split_merge", cs);
         return cuda_status(nsa::launch_split_merge(s, wl.n_split, split_o, split_lse, gates, ob, cs));
     }
+    g_timing.mark("attn_tc", cs);
     return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr, 1,
                                            nullptr, nullptr, ob, cs));
+}
+
+nsa_status nsa_timing_enable(int32_t on) {
+    StageTiming& t = g_timing;
+    if (on && !t.created) {
+        int d = -1;
+        if (cudaGetDevice(&d) != cudaSuccess) return NSA_ERR_CUDA;
+        int made = 0;
+        for (; made <= NSA_TIMING_MAX_STAGES; ++made) {
+            const cudaError_t e = cudaEventCreate(&t.ev[made]);
+            if (e != cudaSuccess) {
+                for (int i = 0; i < made; ++i) cudaEventDestroy(t.ev[i]);
+                return cuda_status(e);
+            }
+        }
+        t.created = true;
+        t.dev = d;
+    }
+    t.on = on != 0;
+    return NSA_OK;
+}
+
+nsa_status nsa_timing_read(int32_t max_stages, float* ms, const char** names, int32_t* n_stages) {
+    if (!n_stages || max_stages < 0 || (max_stages > 0 && (!ms || !names))) return NSA_ERR_INVALID_ARG;
+    StageTiming& t = g_timing;
+    *n_stages = 0;
+    if (!t.created || !t.closed || t.n == 0) return NSA_OK;
+    nsa_status st = cuda_status(cudaEventSynchronize(t.ev[t.n]));
+    if (st != NSA_OK) return st;
+    for (int i = 0; i < t.n && i < max_stages; ++i) {
+        float v = 0.f;
+        st = cuda_status(cudaEventElapsedTime(&v, t.ev[i], t.ev[i + 1]));
+        if (st != NSA_OK) return st;
+        ms[i] = v;
+        names[i] = t.names[i];
+    }
+    *n_stages = t.n;
+    return NSA_OK;
 }
 
 const char* nsa_last_cuda_error(void) { return g_last_cuda_error; }

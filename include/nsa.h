@@ -210,6 +210,30 @@ nsa_status nsa_get_device_status(int32_t* status);
 nsa_status nsa_attn_plan(const nsa_config* cfg, int select_inside, size_t ws_bytes,
                          int32_t* path, int32_t* kernels);
 
+/*
+ * Stage timing, a measurement aid (the pages have no counterpart).
+ *
+ * nsa_timing_enable(1) makes the calling host thread's later
+ * nsa_sparse_attn_fwd calls record a CUDA event on the call's stream before
+ * each stage and one after the last.  The events (NSA_TIMING_MAX_STAGES + 1
+ * per host thread) are created with cudaEventCreate on first use, on the
+ * device current then; calls made while another device is current record
+ * nothing.  No device memory is allocated.  nsa_timing_enable(0) stops the
+ * recording (the events are kept).
+ *
+ * nsa_timing_read waits for the last event of the thread's most recent timed
+ * call and writes up to `max_stages` stage names (static strings) and
+ * durations in milliseconds; *n_stages receives the number of stages (0 if
+ * no call was timed).  Stage names: "select" (score + top-k when idx is
+ * NULL), "index" (block-major inverted index), "sel_bm" (block-major selected
+ * branch), "sel_merge", "attn_tc" (tensor-core branches + gated merge),
+ * "split_merge", "rowwise".  Each stage's time runs from its first launch to
+ * the next stage's first launch on the same stream.
+ */
+#define NSA_TIMING_MAX_STAGES 8
+nsa_status nsa_timing_enable(int32_t on);
+nsa_status nsa_timing_read(int32_t max_stages, float* ms, const char** names, int32_t* n_stages);
+
 /* CUDA's description of the error behind the calling thread's most recent
  * NSA_ERR_CUDA (a static string; "no error" if there was none). */
 const char* nsa_last_cuda_error(void);

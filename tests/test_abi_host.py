@@ -129,3 +129,15 @@ def test_binding_raises_on_error(abi):
     cfg = _cfg(abi, batch=0)
     with pytest.raises(abi.NsaError):
         abi.nsa_workspace_size(cfg)
+
+
+def test_timing_read_without_a_timed_call(abi):
+    L = abi.lib
+    n = ctypes.c_int32(7)
+    assert L.nsa_timing_read(0, None, None, ctypes.byref(n)) == 0
+    assert n.value == 0
+    assert L.nsa_timing_read(-1, None, None, ctypes.byref(n)) == 1
+    assert L.nsa_timing_read(4, None, None, ctypes.byref(n)) == 1
+    assert L.nsa_timing_read(0, None, None, None) == 1
+    assert L.nsa_timing_enable(0) == 0
+    assert abi.nsa_timing_read() == []

@@ -158,12 +158,19 @@ def test_every_block_kept_is_dense_causal_attention():
     check_out(run.out[0].double().cpu().numpy(), ref.double().cpu().numpy(), "dense causal")
 
 
-@pytest.mark.parametrize("name", ["moba32k", "nsa64k", "nsa128k_planted"])
+SAMPLED = {name: WORKLOADS[name] for name in ["moba32k", "nsa64k", "nsa128k_planted"]}
+# block-major work items cross the 8192-query chunk boundary (ragged second chunk)
+SAMPLED["bm_two_chunks"] = WORKLOADS["nsa64k"].with_(name="bm_two_chunks", seqlen_q=9000,
+                                                     seqlen_kv=9000, h_q=16, h_kv=1)
+
+
+@pytest.mark.parametrize("name", sorted(SAMPLED))
 def test_full_size_prefill_sampled_rows(name):
-    wl = WORKLOADS[name]
+    wl = SAMPLED[name]
     run = GpuRun(wl)
     T = wl.seqlen_q
     extra = [wl.sel_block - 1, wl.sel_block, wl.sel_block + 1, 511, 512, 513, T // 2, T - 2]
+    extra += [r for r in (8190, 8191, 8192, 8193) if r < T]
     rows = row_sample(T, stride=max(1, T // 384), head=128, extra=extra)
     compare_run(run, rows)
     # every row of the selection: structural invariants
