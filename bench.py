@@ -50,6 +50,8 @@ STAGE_KERNELS = {
     "index": ("sel_index", os.path.join(CSRC, "sel_index.cu")),
     "split_merge": ("split_merge_kernel", os.path.join(CSRC, "attn_tc.cu")),
     "rowwise": ("attn_rowwise_kernel", os.path.join(CSRC, "attn_rowwise.cu")),
+    "attn_dec": ("dec_kernel", os.path.join(CSRC, "attn_decode.cu")),
+    "dec_merge": ("dec_merge_kernel", os.path.join(CSRC, "attn_decode.cu")),
 }
 
 
@@ -409,7 +411,9 @@ def run_decode(world: int, steps: int, warmup: int):
     pf = Prefill(wl, seed=1000 + (torch.distributed.get_rank() if world > 1 else 0))
     pf.step()                        # pooled cache built once (cache maintenance, not timed)
     torch.cuda.synchronize()
-    per, _, _ = timed_steps(pf, steps, warmup, world, pool=False)
+    per, _, dec_stages = timed_steps(pf, steps, warmup, world, pool=False)
+    pf.attn_launches()
+    path = pf.path
     ms = max_over_ranks(float(per[:, 1:].sum(axis=1).mean()), world)
     nbytes = decode_bytes(wl, pf.idx)
     pk, _ = peaks()
@@ -418,7 +422,8 @@ def run_decode(world: int, steps: int, warmup: int):
     torch.cuda.empty_cache()
     return {"workload": wl.name, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
             "bytes_per_step": nbytes, "frac": gbs / world / pk["hbm_gbs"],
-            "peak_gbs": pk["hbm_gbs"]}
+            "peak_gbs": pk["hbm_gbs"], "path": path,
+            "stage_ms": {"select": float(per[:, 1].mean()), **dec_stages}}
 
 
 def run_ours(args):
@@ -430,6 +435,8 @@ def run_ours(args):
     wl = WORKLOADS[args.workload]
     if args.seqlen:
         wl = wl.with_(seqlen_q=args.seqlen, seqlen_kv=args.seqlen)
+    if args.batch:
+        wl = wl.with_(batch=args.batch)
     pf = Prefill(wl, seed=rank)
     clocks = ClockSampler(torch.cuda.current_device())
     # warm-up and timed region (clocks sampled during it)
@@ -541,6 +548,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqlen", type=int, default=0, help="override the prefill length (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)

@@ -111,7 +111,7 @@ def nsa_status_string(status: int) -> str:
     return lib.nsa_status_string(status).decode()
 
 
-PATHS = {0: "rowwise", 1: "query-major", 2: "block-major", 3: "split-k"}
+PATHS = {0: "rowwise", 1: "query-major", 2: "block-major", 3: "split-k", 4: "decode"}
 
 
 def nsa_attn_plan(cfg: NsaConfig, select_inside: bool, ws_bytes: int):

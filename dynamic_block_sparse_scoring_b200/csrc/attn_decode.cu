@@ -1,0 +1,687 @@
+// Few-query attention (decode) on tcgen05 with the keys as the MMA M dimension.
+//
+// Zhang Xiaojun #94 transcript (bidclub.ai), §4 "Inside Native Sparse
+// Attention": a query attends over the compressed tokens, the tokens of its
+// kept blocks and its sliding window, one softmax per branch, and the three
+// outputs are summed with per-head gates; §5 "Hardware Makes Sparsity Work":
+// the heads of a GQA group share those keys.  At decode a (sequence, group)
+// has one query token, i.e. G query rows.  A query-major tile would stack them
+// as 16 of 128 MMA rows and pay the softmax of all 128; here the roles are
+// transposed instead:
+//
+//   S^T = K Q^T     M = 128 keys of a tile, N = 16 (the group's heads), K = d_qk
+//   O^T += V^T P^T  M = d_v = 128,          N = 16,                    K = 128 keys
+//
+// so a softmax thread owns one key and sees its 16 head scores, and a tile
+// costs 16 exponentials per thread.  The per-head maxima are reduced across
+// the 128 key threads; the running sums stay per thread (scaled on the rare
+// rescale) and are reduced once per work item.
+//
+// Work item = (sequence, unit, query, branch, range of 128-key tiles).
+// Compressed and window tiles are contiguous key ranges; a selected tile is
+// two 64-key segments of the kept blocks.  Each item writes a partial result
+// per head (o = O/l in fp32, lse = m + log2 l); dec_merge_kernel combines the
+// items of a branch with the log-sum-exp rule and sums the branches with the
+// gates.  CTAs are persistent and take items round-robin.
+//
+// Roles (192 threads): warp 0 TMA producer, warp 1 MMA lane + TMEM owner,
+// warps 2-5 softmax and epilogue (TMEM lane quarter = warp % 4).  Every wait
+// is bounded; a timeout records NSA_ERR_TIMEOUT in g_dec_status and unwinds.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace nsa {
+
+__device__ int g_dec_status = 0;
+
+namespace {
+
+constexpr int DT = 128;             // keys per tile
+constexpr int NH = 16;              // MMA N: query rows (heads of one token), padded to 16
+constexpr int DV = 128;             // value width = MMA M of O^T
+constexpr int NTHREADS = 192;
+constexpr int CH = DT * 128;        // one 64-column chunk of a 128-key tile (16 KB)
+constexpr int QCH = NH * 128;       // one 64-column chunk of the 16 query rows (2 KB)
+constexpr int PCH = NH * 128;       // one 64-key chunk of P^T (2 KB)
+constexpr uint64_t WAIT_NS = 1000000000ull;
+
+enum { B_CMP = 0, B_SEL = 1, B_WIN = 2 };
+
+struct DecArgs {
+    Shape s;
+    const int32_t* idx;
+    float* part_o;      // [items][NH][DV]
+    float* part_lse;    // [items][NH]
+    int hpt;
+    int tpi;            // tiles per item
+    int ni[3];          // items per unit and branch (0 = branch off)
+    int ni_all;
+    int n_items;
+    int spb;            // 64-key segments per selection block
+    float scale_log2;
+};
+
+template <int DQK>
+struct DecSmem {
+    static constexpr int QC = DQK / 64;
+    static constexpr int K_OFF = 0;                             // 2 stages x QC chunks
+    static constexpr int V_OFF = K_OFF + 2 * QC * CH;           // 2 stages x 2 chunks
+    static constexpr int Q_OFF = V_OFF + 2 * 2 * CH;            // 2 buffers x QC chunks
+    static constexpr int P_OFF = Q_OFF + 2 * QC * QCH;          // 2 buffers x 2 chunks
+    static constexpr int RED_OFF = P_OFF + 2 * 2 * PCH;         // [4 warps][NH] fp32
+    static constexpr int BAR_OFF = RED_OFF + 4 * NH * 4;
+    // q_full[2] q_empty[2] kv_full[2] kv_empty[2] s_full[2] s_free[2] p_full[2] pv_done[2]
+    // o_full o_free
+    static constexpr int NBAR = 18;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int ALLOC = MISC_OFF + 64 + 1024;
+};
+
+struct DecBars {
+    uint64_t* b;
+    __device__ __forceinline__ uint64_t* q_full(int i) const { return b + i; }
+    __device__ __forceinline__ uint64_t* q_empty(int i) const { return b + 2 + i; }
+    __device__ __forceinline__ uint64_t* kv_full(int i) const { return b + 4 + i; }
+    __device__ __forceinline__ uint64_t* kv_empty(int i) const { return b + 6 + i; }
+    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 8 + i; }
+    __device__ __forceinline__ uint64_t* s_free(int i) const { return b + 10 + i; }
+    __device__ __forceinline__ uint64_t* p_full(int i) const { return b + 12 + i; }
+    __device__ __forceinline__ uint64_t* pv_done(int i) const { return b + 14 + i; }
+    __device__ __forceinline__ uint64_t* o_full() const { return b + 16; }
+    __device__ __forceinline__ uint64_t* o_free() const { return b + 17; }
+};
+
+// What one work item covers; every role derives it the same way.
+struct Item {
+    int b, u, i, t;     // sequence, selection unit, query row, query position
+    int br;             // B_CMP / B_SEL / B_WIN
+    int t0, t1;         // tile range [t0, t1) (empty when t0 >= t1)
+    int n_vis;          // compressed: visible tokens
+    int win_lo;         // window: first key
+    int nseg;           // selected: 64-key segments of the kept blocks
+    const int32_t* irow;
+};
+
+__device__ __forceinline__ Item item_info(const DecArgs& a, int item) {
+    const Shape& s = a.s;
+    Item it;
+    const int unit = item / a.ni_all;
+    int k = item % a.ni_all;
+    it.i = unit % s.Tq;
+    const int bu = unit / s.Tq;
+    it.u = bu % s.Hsel;
+    it.b = bu / s.Hsel;
+    it.t = s.q0 + it.i;
+    it.br = k < a.ni[0] ? B_CMP : (k < a.ni[0] + a.ni[1] ? B_SEL : B_WIN);
+    const int sub = it.br == B_CMP ? k : (it.br == B_SEL ? k - a.ni[0] : k - a.ni[0] - a.ni[1]);
+    it.n_vis = 0;
+    it.win_lo = 0;
+    it.nseg = 0;
+    it.irow = nullptr;
+    int ntiles = 0;
+    if (it.br == B_CMP) {
+        it.n_vis = it.t >= s.lc - 1 ? min((it.t - s.lc + 1) / s.sc + 1, s.n_cmp) : 0;
+        ntiles = (it.n_vis + DT - 1) / DT;
+    } else if (it.br == B_SEL) {
+        it.irow = a.idx + (((size_t)it.b * s.Hsel + it.u) * s.Tq + it.i) * s.topk;
+        int nv = 0;
+        for (int e = 0; e < s.topk; ++e) nv += it.irow[e] >= 0 ? 1 : 0;
+        it.nseg = nv * a.spb;
+        ntiles = (it.nseg + 1) / 2;
+    } else {
+        it.win_lo = max(0, it.t - s.win + 1);
+        ntiles = (it.t - it.win_lo + 1 + DT - 1) / DT;
+    }
+    it.t0 = sub * a.tpi;
+    it.t1 = min(ntiles, it.t0 + a.tpi);
+    return it;
+}
+
+// First key of 64-key segment e of a selected item (kept blocks ascending, -1 padded last).
+__device__ __forceinline__ int seg_start(const DecArgs& a, const Item& it, int e) {
+    const int blk = it.irow[e / a.spb];
+    return blk * a.s.bs + (e % a.spb) * 64;
+}
+
+__device__ __forceinline__ bool dec_warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, abort_flag, WAIT_NS));
+}
+
+__device__ __forceinline__ void dec_abort(volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicExch(&g_dec_status, (int)NSA_ERR_TIMEOUT);
+}
+
+// order-preserving int image of a float (for redux.sync.max)
+__device__ __forceinline__ int f2ord(float x) {
+    const int i = __float_as_int(x);
+    return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
+
+__device__ __forceinline__ int warp_max_i(int v) {
+    int r;
+    asm volatile("redux.sync.max.s32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+    return r;
+}
+
+template <int DQK>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    dec_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k128,
+               const __grid_constant__ CUtensorMap map_v128, const __grid_constant__ CUtensorMap map_k64,
+               const __grid_constant__ CUtensorMap map_v64, const __grid_constant__ CUtensorMap map_kc,
+               const __grid_constant__ CUtensorMap map_vc, const DecArgs a) {
+    using L = DecSmem<DQK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    DecBars bar{reinterpret_cast<uint64_t*>(sm + L::BAR_OFF)};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC_OFF + 8);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Shape& s = a.s;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bar.q_full(i), 1);
+            tc::mbar_init(bar.q_empty(i), 1);
+            tc::mbar_init(bar.kv_full(i), 1);
+            tc::mbar_init(bar.kv_empty(i), 1);
+            tc::mbar_init(bar.s_full(i), 1);
+            tc::mbar_init(bar.s_free(i), 4);
+            tc::mbar_init(bar.p_full(i), 4);
+            tc::mbar_init(bar.pv_done(i), 1);
+        }
+        tc::mbar_init(bar.o_full(), 1);
+        tc::mbar_init(bar.o_free(), 4);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 64);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto tS = [&](int i) { return tmem + 16 * i; };   // S^T buffers: columns [0,16) [16,32)
+    const uint32_t tO = tmem + 32;                      // O^T: columns [32,48)
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        bool ok = true;
+        uint32_t tcount = 0, qcount = 0;
+        for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+            const Item it = item_info(a, item);
+            if (it.t0 >= it.t1) continue;
+            const int kvh = it.u;                    // group-shared selection: unit = KV head
+            const int plane = it.b * s.Hkv + kvh;
+            const int qb = qcount & 1;
+            if (!dec_warp_wait(bar.q_empty(qb), ((qcount >> 1) & 1) ^ 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qb), L::QC * a.hpt * 128);
+            __syncwarp();
+            if (lane < L::QC)
+                tc::tma_load_4d(sm + L::Q_OFF + (qb * L::QC + lane) * QCH, &map_q, bar.q_full(qb),
+                                64 * lane, it.u * a.hpt, it.i, it.b);
+            ++qcount;
+            for (int j = it.t0; j < it.t1; ++j, ++tcount) {
+                const int st = tcount & 1;
+                if (!dec_warp_wait(bar.kv_empty(st), ((tcount >> 1) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* kst = sm + L::K_OFF + st * L::QC * CH;
+                uint8_t* vst = sm + L::V_OFF + st * 2 * CH;
+                if (it.br == B_SEL) {
+                    // an odd last segment is paired with itself (masked by the softmax),
+                    // so that the stage never holds stale or uninitialised V rows
+                    const int e0 = 2 * j, e1 = 2 * j + 1;
+                    const int r0 = seg_start(a, it, e0);
+                    const int r1 = e1 < it.nseg ? seg_start(a, it, e1) : r0;
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.kv_full(st), 2 * (L::QC + 2) * (CH / 2));
+                    __syncwarp();
+                    // lanes [0, QC) K chunks, [QC, QC+2) V chunks; second segment on lanes +8
+                    const int h = lane >> 3, c = lane & 7;
+                    if (h < 2 && c < L::QC + 2) {
+                        const int row = h ? r1 : r0;
+                        if (c < L::QC)
+                            tc::tma_load_3d(kst + c * CH + h * (CH / 2), &map_k64, bar.kv_full(st), 64 * c, row, plane);
+                        else
+                            tc::tma_load_3d(vst + (c - L::QC) * CH + h * (CH / 2), &map_v64, bar.kv_full(st),
+                                            64 * (c - L::QC), row, plane);
+                    }
+                } else {
+                    const bool cmp = it.br == B_CMP;
+                    const int row = cmp ? j * DT : it.win_lo + j * DT;
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.kv_full(st), (L::QC + 2) * CH);
+                    __syncwarp();
+                    if (lane < L::QC)
+                        tc::tma_load_3d(kst + lane * CH, cmp ? &map_kc : &map_k128, bar.kv_full(st), 64 * lane, row, plane);
+                    else if (lane < L::QC + 2)
+                        tc::tma_load_3d(vst + (lane - L::QC) * CH, cmp ? &map_vc : &map_v128, bar.kv_full(st),
+                                        64 * (lane - L::QC), row, plane);
+                }
+            }
+        }
+        if (!ok) dec_abort(abort_flag);
+        // wait for every copy still in flight before the CTA may exit
+        volatile int never = 0;
+        for (uint32_t st = 0; st < 2; ++st) {
+            if (tcount > st) {
+                const uint32_t last = st + ((tcount - 1 - st) / 2) * 2;
+                tc::mbar_wait(bar.kv_full(st), (last >> 1) & 1, &never, WAIT_NS);
+            }
+            if (qcount > st) {
+                const uint32_t last = st + ((qcount - 1 - st) / 2) * 2;
+                tc::mbar_wait(bar.q_full(st), (last >> 1) & 1, &never, WAIT_NS);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            const uint32_t idesc_qk = tc::idesc_bf16_f32(DT, NH, false, false);
+            const uint32_t idesc_pv = tc::idesc_bf16_f32(DV, NH, true, false);
+            const uint32_t k_base = tc::smem_u32(sm + L::K_OFF);
+            const uint32_t v_base = tc::smem_u32(sm + L::V_OFF);
+            const uint32_t q_base = tc::smem_u32(sm + L::Q_OFF);
+            const uint32_t p_base = tc::smem_u32(sm + L::P_OFF);
+            bool ok = true;
+            uint32_t tcount = 0, qcount = 0, ocount = 0;
+            auto issue_pv = [&](uint32_t n, bool first) -> bool {
+                const int pb = n & 1;
+                if (!tc::mbar_wait(bar.p_full(pb), (n >> 1) & 1, abort_flag, WAIT_NS)) return false;
+                // the first PV of an item overwrites O: the previous item's epilogue must have read it
+                if (first && ocount > 0 && !tc::mbar_wait(bar.o_free(), (ocount - 1) & 1, abort_flag, WAIT_NS))
+                    return false;
+                tc::fence_after_sync();
+                const uint32_t vst = v_base + pb * 2 * CH;
+                const uint32_t pst = p_base + pb * 2 * PCH;
+#pragma unroll
+                for (int kk = 0; kk < DT / 16; ++kk)
+                    tc::mma_ss(tO, tc::sdesc_sw128(vst + kk * 2048, CH, 1024),
+                               tc::sdesc_sw128(pst + (kk >> 2) * PCH + (kk & 3) * 32, 16, 1024), idesc_pv,
+                               (first && kk == 0) ? 0u : 1u);
+                tc::mma_commit(bar.kv_empty(pb));
+                tc::mma_commit(bar.pv_done(pb));
+                return true;
+            };
+            for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+                const Item it = item_info(a, item);
+                if (it.t0 >= it.t1) continue;
+                const int qb = qcount & 1;
+                if (!tc::mbar_wait(bar.q_full(qb), (qcount >> 1) & 1, abort_flag, WAIT_NS)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t qst = q_base + qb * L::QC * QCH;
+                for (int j = it.t0; j < it.t1; ++j, ++tcount) {
+                    const int st = tcount & 1;
+                    if (!tc::mbar_wait(bar.kv_full(st), (tcount >> 1) & 1, abort_flag, WAIT_NS) ||
+                        (tcount >= 2 && !tc::mbar_wait(bar.s_free(st), ((tcount >> 1) & 1) ^ 1, abort_flag, WAIT_NS))) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t kst = k_base + st * L::QC * CH;
+#pragma unroll
+                    for (int kk = 0; kk < DQK / 16; ++kk)
+                        tc::mma_ss(tS(st), tc::sdesc_sw128(kst + (kk >> 2) * CH + (kk & 3) * 32, 16, 1024),
+                                   tc::sdesc_sw128(qst + (kk >> 2) * QCH + (kk & 3) * 32, 16, 1024), idesc_qk,
+                                   kk > 0 ? 1u : 0u);
+                    tc::mma_commit(bar.s_full(st));
+                    if (j == it.t1 - 1) tc::mma_commit(bar.q_empty(qb));
+                    if (j > it.t0 && !issue_pv(tcount - 1, j - 1 == it.t0)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok) break;
+                if (!issue_pv(tcount - 1, it.t1 - 1 == it.t0)) {
+                    ok = false;
+                    break;
+                }
+                tc::mma_commit(bar.o_full());
+                ++qcount;
+                ++ocount;
+            }
+            if (!ok) dec_abort(abort_flag);
+            volatile int never = 0;
+            // the last commit arrives once everything issued before it completed
+            if (ocount > 0) tc::mbar_wait(bar.o_free(), (ocount - 1) & 1, &never, WAIT_NS);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;            // key of the tile; d_v lane of O^T
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float* red = reinterpret_cast<float*>(sm + L::RED_OFF);     // [4][NH]
+        uint8_t* pbuf = sm + L::P_OFF;
+        const int wq = warp - 2;                      // 0..3, slot in red
+        bool ok = true;
+        uint32_t tcount = 0, ocount = 0;
+        for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+            const Item it = item_info(a, item);
+            float* po = a.part_o + (size_t)item * NH * DV;
+            float* pl = a.part_lse + (size_t)item * NH;
+            if (it.t0 >= it.t1) {
+                for (int h = 0; h < a.hpt; ++h) po[h * DV + r] = 0.f;
+                if (r < NH) pl[r] = -INFINITY;
+                continue;
+            }
+            float mrun[NH], lsum[NH];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                mrun[h] = -INFINITY;
+                lsum[h] = 0.f;
+            }
+            for (int j = it.t0; j < it.t1; ++j, ++tcount) {
+                const int sb = tcount & 1;
+                // key of this thread and whether the query sees it
+                bool valid;
+                if (it.br == B_CMP) {
+                    valid = j * DT + r < it.n_vis;
+                } else if (it.br == B_SEL) {
+                    const int e = 2 * j + (r >> 6);
+                    valid = e < it.nseg && seg_start(a, it, e) + (r & 63) <= it.t;
+                } else {
+                    valid = it.win_lo + j * DT + r <= it.t;
+                }
+                bool okw = dec_warp_wait(bar.s_full(sb), (tcount >> 1) & 1, abort_flag);
+                float x[NH];
+                if (okw) {
+                    tc::fence_after_sync();
+                    uint32_t sv[NH];
+                    tc::tmem_ld16(tS(sb) + lane_off, sv);
+                    tc::tmem_wait_ld();
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar.s_free(sb));
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        x[h] = (valid && h < a.hpt) ? __uint_as_float(sv[h]) * a.scale_log2 : -INFINITY;
+                        const int m = warp_max_i(f2ord(x[h]));
+                        if (lane == h) red[wq * NH + h] = ord2f(m);
+                    }
+                }
+                if (!tc::named_bar_and(1, 128, okw)) {
+                    ok = false;
+                    break;
+                }
+                // tile maxima; lazy rescale (only when a head's maximum grows by > 2^8)
+                bool rescale = false;
+                float alpha[NH];
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const float tm = fmaxf(fmaxf(red[h], red[NH + h]), fmaxf(red[2 * NH + h], red[3 * NH + h]));
+                    alpha[h] = 1.f;
+                    if (tm > mrun[h] + 8.f) {
+                        alpha[h] = tc::ex2(mrun[h] - tm);      // 0 when mrun = -inf
+                        mrun[h] = tm;
+                        lsum[h] *= alpha[h];
+                        rescale = true;
+                    }
+                }
+                bool ok2 = true;
+                if (rescale && j > it.t0) {
+                    // O^T holds tiles < j: wait for PV(j - 1), then scale its head columns
+                    ok2 = dec_warp_wait(bar.pv_done((tcount - 1) & 1), ((tcount - 1) >> 1) & 1, abort_flag);
+                    if (ok2) {
+                        tc::fence_after_sync();
+                        uint32_t ov[NH];
+                        tc::tmem_ld16(tO + lane_off, ov);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
+                        tc::tmem_st16(tO + lane_off, ov);
+                        tc::tmem_wait_st();
+                    }
+                }
+                // P^T buffer sb was last read by PV(tcount - 2)
+                if (ok2 && tcount >= 2)
+                    ok2 = dec_warp_wait(bar.pv_done(sb), ((tcount >> 1) & 1) ^ 1, abort_flag);
+                if (ok2) {
+                    uint8_t* pb = pbuf + sb * 2 * PCH + (r >> 6) * PCH;
+                    const int unit16 = (r & 63) >> 3;
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const float p = x[h] == -INFINITY ? 0.f : tc::ex2(x[h] - mrun[h]);
+                        lsum[h] += p;
+                        *reinterpret_cast<__nv_bfloat16*>(pb + h * 128 + ((unit16 ^ (h & 7)) << 4) + (r & 7) * 2) =
+                            __float2bfloat16_rn(p);
+                    }
+                    tc::fence_before_sync();
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
+                }
+                if (!tc::named_bar_and(1, 128, ok2)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (!ok) break;
+            // epilogue: o = O^T / l per head, lse = m + log2 l
+            bool okw = dec_warp_wait(bar.o_full(), ocount & 1, abort_flag);
+            uint32_t ov[NH];
+            if (okw) {
+                tc::fence_after_sync();
+                tc::tmem_ld16(tO + lane_off, ov);
+                tc::tmem_wait_ld();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar.o_free());
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const float v = warp_sum(lsum[h]);
+                    if (lane == h) red[wq * NH + h] = v;
+                }
+            }
+            if (!tc::named_bar_and(1, 128, okw)) {
+                ok = false;
+                break;
+            }
+            ++ocount;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const float l = (red[h] + red[NH + h]) + (red[2 * NH + h] + red[3 * NH + h]);
+                if (h < a.hpt) po[h * DV + r] = l > 0.f ? __uint_as_float(ov[h]) / l : 0.f;
+                if (r == h) pl[h] = l > 0.f ? mrun[h] + __log2f(l) : -INFINITY;
+            }
+            // red is rewritten by the next tile only after everyone has read it
+            tc::named_bar_sync(1, 128);
+        }
+        if (!ok) dec_abort(abort_flag);
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, 64);
+}
+
+// out[b, i, h] = sum over branches of gate * (log-sum-exp merge of the branch's items)
+__global__ void __launch_bounds__(256) dec_merge_kernel(Shape s, DecArgs a, const float* __restrict__ gates,
+                                                        __nv_bfloat16* __restrict__ out) {
+    const int c8n = DV / 8;
+    const size_t total = (size_t)s.B * s.Tq * s.Hq * c8n;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int c8 = (int)(e % c8n);
+        const size_t row = e / c8n;                  // (b, i, hq)
+        const int hq = (int)(row % s.Hq);
+        const int i = (int)((row / s.Hq) % s.Tq);
+        const int b = (int)(row / ((size_t)s.Hq * s.Tq));
+        const int u = hq / a.hpt, hl = hq % a.hpt;
+        const size_t unit = ((size_t)b * s.Hsel + u) * s.Tq + i;
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int k0 = 0;
+        for (int br = 0; br < 3; ++br) {
+            const int n = a.ni[br];
+            if (n == 0) continue;
+            const size_t it0 = unit * a.ni_all + k0;
+            k0 += n;
+            float m = -INFINITY;
+            for (int k = 0; k < n; ++k) m = fmaxf(m, a.part_lse[(it0 + k) * NH + hl]);
+            if (m == -INFINITY) continue;                // empty branch: o = 0
+            float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f;
+            for (int k = 0; k < n; ++k) {
+                const float w = exp2f(a.part_lse[(it0 + k) * NH + hl] - m);
+                wsum += w;
+                const float4* src = reinterpret_cast<const float4*>(a.part_o + ((it0 + k) * NH + hl) * DV + c8 * 8);
+                const float4 x0 = src[0], x1 = src[1];
+                o[0] = fmaf(w, x0.x, o[0]); o[1] = fmaf(w, x0.y, o[1]);
+                o[2] = fmaf(w, x0.z, o[2]); o[3] = fmaf(w, x0.w, o[3]);
+                o[4] = fmaf(w, x1.x, o[4]); o[5] = fmaf(w, x1.y, o[5]);
+                o[6] = fmaf(w, x1.z, o[6]); o[7] = fmaf(w, x1.w, o[7]);
+            }
+            const float g = gates ? gates[row * 3 + br] : 1.f;
+            const float f = g / wsum;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = fmaf(f, o[q], acc[q]);
+        }
+        *reinterpret_cast<uint4*>(out + row * DV + c8 * 8) = pack8(acc);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 dec_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool dec_encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                const cuuint64_t* strides, const cuuint32_t* box) {
+    auto enc = dec_encode_fn();
+    if (!enc) return false;
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+DecArgs make_args(const Shape& s, const int32_t* idx, float* part_o, float* part_lse) {
+    DecArgs a;
+    a.s = s;
+    a.idx = idx;
+    a.part_o = part_o;
+    a.part_lse = part_lse;
+    a.hpt = s.heads_per_unit;
+    a.spb = s.bs / 64;
+    a.scale_log2 = s.scale * 1.4426950408889634f;
+    // most tiles any query of the problem has, per branch
+    const int t_last = s.q0 + s.Tq - 1;
+    const int cmp_tiles = (s.flags & NSA_BR_CMP) ? (s.n_cmp + DT - 1) / DT : 0;
+    const int sel_tiles = (s.flags & NSA_BR_SEL) ? (s.topk * a.spb + 1) / 2 : 0;
+    const int win_tiles = (s.flags & NSA_BR_WIN) ? (min(s.win, t_last + 1) + DT - 1) / DT : 0;
+    const long units = (long)s.B * s.Hsel * s.Tq;
+    const long tiles = units * (cmp_tiles + sel_tiles + win_tiles);
+    // about ten items per SM
+    a.tpi = (int)std::max<long>(1, std::min<long>(64, (tiles + 10 * 148 - 1) / (10 * 148)));
+    a.ni[0] = (cmp_tiles + a.tpi - 1) / a.tpi;
+    a.ni[1] = (sel_tiles + a.tpi - 1) / a.tpi;
+    a.ni[2] = (win_tiles + a.tpi - 1) / a.tpi;
+    a.ni_all = a.ni[0] + a.ni[1] + a.ni[2];
+    a.n_items = (int)(units * a.ni_all);
+    return a;
+}
+
+template <int DQK>
+cudaError_t launch_dec_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp, const __nv_bfloat16* vcmp,
+                            const DecArgs& a, cudaStream_t st) {
+    CUtensorMap mq, mk128, mv128, mk64, mv64, mkc, mvc;
+    const cuuint64_t qd[4] = {(cuuint64_t)DQK, (cuuint64_t)s.Hq, (cuuint64_t)s.Tq, (cuuint64_t)s.B};
+    const cuuint64_t qs[3] = {(cuuint64_t)DQK * 2, (cuuint64_t)DQK * 2 * s.Hq,
+                              (cuuint64_t)DQK * 2 * s.Hq * s.Tq};
+    const cuuint32_t qb[4] = {64, (cuuint32_t)a.hpt, 1, 1};
+    const cuuint64_t kd[3] = {(cuuint64_t)DQK, (cuuint64_t)s.Tk, (cuuint64_t)s.B * s.Hkv};
+    const cuuint64_t ks[2] = {(cuuint64_t)DQK * 2, (cuuint64_t)DQK * 2 * s.Tk};
+    const cuuint64_t vd[3] = {(cuuint64_t)DV, (cuuint64_t)s.Tk, (cuuint64_t)s.B * s.Hkv};
+    const cuuint64_t vs[2] = {(cuuint64_t)DV * 2, (cuuint64_t)DV * 2 * s.Tk};
+    const cuuint32_t b128[3] = {64, (cuuint32_t)DT, 1};
+    const cuuint32_t b64[3] = {64, 64, 1};
+    if (!dec_encode(&mq, q, 4, qd, qs, qb) || !dec_encode(&mk128, k, 3, kd, ks, b128) ||
+        !dec_encode(&mv128, v, 3, vd, vs, b128) || !dec_encode(&mk64, k, 3, kd, ks, b64) ||
+        !dec_encode(&mv64, v, 3, vd, vs, b64))
+        return cudaErrorInvalidValue;
+    if ((s.flags & NSA_BR_CMP) && s.n_cmp > 0) {
+        const cuuint64_t cd[3] = {(cuuint64_t)DQK, (cuuint64_t)s.n_cmp, (cuuint64_t)s.B * s.Hkv};
+        const cuuint64_t cs[2] = {(cuuint64_t)DQK * 2, (cuuint64_t)DQK * 2 * s.n_cmp};
+        const cuuint64_t cvd[3] = {(cuuint64_t)DV, (cuuint64_t)s.n_cmp, (cuuint64_t)s.B * s.Hkv};
+        const cuuint64_t cvs[2] = {(cuuint64_t)DV * 2, (cuuint64_t)DV * 2 * s.n_cmp};
+        if (!dec_encode(&mkc, kcmp, 3, cd, cs, b128) || !dec_encode(&mvc, vcmp, 3, cvd, cvs, b128))
+            return cudaErrorInvalidValue;
+    } else {
+        mkc = mk128;      // never used: no compressed tile is enumerated
+        mvc = mv128;
+    }
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int smem = DecSmem<DQK>::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(dec_kernel<DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = std::min(nsm, a.n_items);
+    dec_kernel<DQK><<<grid, NTHREADS, smem, st>>>(mq, mk128, mv128, mk64, mv64, mkc, mvc, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_dec_supported(const Shape& s) {
+    if (s.per_head) return false;
+    if (s.dqk != 64 && s.dqk != 128 && s.dqk != 192) return false;
+    if (s.dv != DV) return false;
+    const int hpt = s.heads_per_unit;
+    if (hpt != 8 && hpt != 16) return false;
+    if ((s.flags & NSA_BR_SEL) && s.bs % 64 != 0) return false;
+    return s.Tq >= 1 && s.Tq <= 4;
+}
+
+size_t attn_dec_items(const Shape& s) { return (size_t)make_args(s, nullptr, nullptr, nullptr).n_items; }
+size_t attn_dec_part_floats() { return (size_t)NH * DV; }
+
+cudaError_t launch_attn_dec(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp, const __nv_bfloat16* vcmp,
+                            const int32_t* idx, float* part_o, float* part_lse, cudaStream_t st) {
+    const DecArgs a = make_args(s, idx, part_o, part_lse);
+    if (a.n_items == 0) return cudaSuccess;
+    if (s.dqk == 64) return launch_dec_impl<64>(s, q, k, v, kcmp, vcmp, a, st);
+    if (s.dqk == 128) return launch_dec_impl<128>(s, q, k, v, kcmp, vcmp, a, st);
+    if (s.dqk == 192) return launch_dec_impl<192>(s, q, k, v, kcmp, vcmp, a, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_dec_merge(const Shape& s, const float* part_o, const float* part_lse,
+                             const float* gates, __nv_bfloat16* out, cudaStream_t st) {
+    DecArgs a = make_args(s, nullptr, const_cast<float*>(part_o), const_cast<float*>(part_lse));
+    const size_t total = (size_t)s.B * s.Tq * s.Hq * (DV / 8);
+    if (total == 0) return cudaSuccess;
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 8);
+    dec_merge_kernel<<<grid, 256, 0, st>>>(s, a, gates, out);
+    return cudaGetLastError();
+}
+
+int read_and_clear_dec_status() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dec_status, sizeof(int)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_dec_status, &zero, sizeof(int));
+    return v;
+}
+
+}  // namespace nsa

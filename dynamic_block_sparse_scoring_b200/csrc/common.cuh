@@ -103,4 +103,14 @@ cudaError_t launch_sel_bm(const Shape& s, const __nv_bfloat16* q, const __nv_bfl
                           const __nv_bfloat16* v, const SelIndex& x, __nv_bfloat16* part_o,
                           float* part_lse, cudaStream_t st);
 int read_and_clear_bm_status();
+// few-query attention with the keys as the MMA M dimension (attn_decode.cu)
+bool attn_dec_supported(const Shape& s);
+size_t attn_dec_items(const Shape& s);
+size_t attn_dec_part_floats();   // fp32 values of one item's partial output (16 rows x 128)
+cudaError_t launch_attn_dec(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp, const __nv_bfloat16* vcmp,
+                            const int32_t* idx, float* part_o, float* part_lse, cudaStream_t st);
+cudaError_t launch_dec_merge(const Shape& s, const float* part_o, const float* part_lse,
+                             const float* gates, __nv_bfloat16* out, cudaStream_t st);
+int read_and_clear_dec_status();
 }  // namespace nsa

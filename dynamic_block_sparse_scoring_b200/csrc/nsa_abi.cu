@@ -88,10 +88,14 @@ bool use_block_major(const Shape& s) {
            s.Tq >= 256;
 }
 
+// Few query rows per sequence (decode): keys as the MMA M dimension.
+bool use_decode(const Shape& s) { return nsa::attn_dec_supported(s); }
+
 // Workspace regions, each 256-byte aligned, in this order.
 struct WsLayout {
     size_t idx = 0, cnt = 0, off = 0, item_off = 0, cursor = 0, list = 0, items = 0, part_o = 0,
-           part_lse = 0, o_sel = 0, split_o = 0, split_lse = 0, total = 0, minimal = 0;
+           part_lse = 0, o_sel = 0, split_o = 0, split_lse = 0, dec_o = 0, dec_lse = 0, total = 0,
+           minimal = 0;
     int n_split = 1;
 };
 
@@ -106,7 +110,11 @@ WsLayout ws_layout(const Shape& s) {
     if (s.flags & NSA_BR_SEL) w.idx = take(idx_bytes(s));
     w.minimal = at;
     // split-K partials for problems with few work tiles (decode)
-    if (nsa::attn_tc_supported(s) && !use_block_major(s)) {
+    if (use_decode(s)) {
+        const size_t items = nsa::attn_dec_items(s);
+        w.dec_o = take(items * nsa::attn_dec_part_floats() * 4);
+        w.dec_lse = take(items * 16 * 4);
+    } else if (nsa::attn_tc_supported(s) && !use_block_major(s)) {
         w.n_split = nsa::attn_tc_split_count(s);
         if (w.n_split > 1) {
             const size_t rows = (size_t)s.B * s.Tq * s.Hq * 3 * w.n_split;
@@ -217,7 +225,9 @@ struct Plan {
 
 Plan make_plan(const Shape& s, bool select_inside, size_t ws_bytes, const WsLayout& wl) {
     Plan p{NSA_PATH_ROWWISE, 1};
-    if (nsa::attn_tc_supported(s)) {
+    if (use_decode(s) && ws_bytes >= wl.total) {
+        p = {NSA_PATH_DECODE, 2};
+    } else if (nsa::attn_tc_supported(s)) {
         if (use_block_major(s) && ws_bytes >= wl.total) p = {NSA_PATH_BLOCK_MAJOR, 7};
         else if (wl.n_split > 1 && ws_bytes >= wl.total) p = {NSA_PATH_SPLIT_K, 2};
         else p = {NSA_PATH_QUERY_MAJOR, 1};
@@ -363,6 +373,15 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, o_sel, 1,
                                                nullptr, nullptr, ob, cs));
     }
+    if (plan.path == NSA_PATH_DECODE) {
+        float* dec_o = reinterpret_cast<float*>(ws + wl.dec_o);
+        float* dec_lse = reinterpret_cast<float*>(ws + wl.dec_lse);
+        g_timing.mark("attn_dec", cs);
+        st = cuda_status(nsa::launch_attn_dec(s, qb, kb, vb, kcb, vcb, sel_idx, dec_o, dec_lse, cs));
+        if (st != NSA_OK) return st;
+        g_timing.mark("dec_merge", cs);
+        return cuda_status(nsa::launch_dec_merge(s, dec_o, dec_lse, gates, ob, cs));
+    }
     if (plan.path == NSA_PATH_SPLIT_K) {
         float* split_o = reinterpret_cast<float*>(ws + wl.split_o);
         float* split_lse = reinterpret_cast<float*>(ws + wl.split_lse);
@@ -422,8 +441,9 @@ nsa_status nsa_get_device_status(int32_t* status) {
     if (!status) return NSA_ERR_INVALID_ARG;
     const int v1 = nsa::read_and_clear_tc_status();
     const int v2 = nsa::read_and_clear_bm_status();
-    if (v1 < 0 || v2 < 0) return NSA_ERR_CUDA;
-    *status = v1 ? v1 : v2;
+    const int v3 = nsa::read_and_clear_dec_status();
+    if (v1 < 0 || v2 < 0 || v3 < 0) return NSA_ERR_CUDA;
+    *status = v1 ? v1 : (v2 ? v2 : v3);
     return NSA_OK;
 }
 

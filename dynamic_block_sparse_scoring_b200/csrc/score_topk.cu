@@ -29,7 +29,7 @@ constexpr int ST_RPW = ST_RT / 8;   // rows per warp
 enum { MODE_SELECT = 0, MODE_SCORES = 1, MODE_SELECT_FROM_SCORES = 2 };
 
 template <int MODE>
-__global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
                                                            const float* __restrict__ kbar,
                                                            const float* __restrict__ scores_in,
                                                            float* __restrict__ scores_out,
@@ -61,17 +61,44 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
             float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             if (r < nrows) {
                 const __nv_bfloat16* src = q + (((size_t)b * s.Tq + i0 + r) * s.Hq + h0) * d + vec * 8;
-                for (int hh = 0; hh < nh; ++hh) {
-                    float f[8];
-                    unpack8(*reinterpret_cast<const uint4*>(src + (size_t)hh * d), f);
+                // the unit's heads in groups of 8, every load of a group issued before
+                // any is summed (the rows are far apart: one HBM round trip per group)
+                for (int h8 = 0; h8 < nh; h8 += 8) {
+                    uint4 raw[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+                    for (int hh = 0; hh < 8; ++hh)
+                        if (h8 + hh < nh) raw[hh] = *reinterpret_cast<const uint4*>(src + (size_t)(h8 + hh) * d);
+#pragma unroll
+                    for (int hh = 0; hh < 8; ++hh) {
+                        if (h8 + hh >= nh) break;
+                        float f[8];
+                        unpack8(raw[hh], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+                    }
                 }
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) qs[r * ld + vec * 8 + e] = acc[e];
         }
     }
+
+    // pooled-key chunks go through registers: the loads of chunk j + 1 are issued
+    // before chunk j is scored, so their latency overlaps the FFMA and top-k work
+    constexpr int KREG = ST_KC * 192 / 4 / ST_NT;    // float4 per thread; d = 256 loads the rest late
+    float4 kreg[KREG];
+    const float* kb_base = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * d;
+    auto load_chunk = [&](int c0) {
+        const int nk = min(ST_KC, cmax - c0);
+        const int nf4 = d / 4;
+#pragma unroll
+        for (int e = 0; e < KREG; ++e) {
+            const int p = tid + e * ST_NT;
+            if (p < nk * nf4)
+                kreg[e] = *reinterpret_cast<const float4*>(kb_base + (size_t)(c0 + p / nf4) * d + (p % nf4) * 4);
+        }
+    };
+    if (MODE != MODE_SELECT_FROM_SCORES && cmax > 0) load_chunk(0);
 
     const int K1 = s.topk - 1;               // past blocks kept per row
     unsigned long long key[ST_RPW];      // lane's slot of rows ST_RPW*warp + j
@@ -81,14 +108,17 @@ __global__ void __launch_bounds__(ST_NT) score_topk_kernel(Shape s, const __nv_b
     for (int b0 = 0; b0 < cmax; b0 += ST_KC) {
         const int nk = min(ST_KC, cmax - b0);
         if (MODE != MODE_SELECT_FROM_SCORES) {
-            const float* src = kbar + ((size_t)(b * s.Hkv + kvh) * s.nb_full + b0) * d;
             const int nf4 = d / 4;
-            for (int p = tid; p < nk * nf4; p += ST_NT) {
-                const int r = p / nf4, c4 = p % nf4;
-                *reinterpret_cast<float4*>(ks + r * ld + c4 * 4) =
-                    *reinterpret_cast<const float4*>(src + (size_t)r * d + c4 * 4);
+#pragma unroll
+            for (int e = 0; e < KREG; ++e) {
+                const int p = tid + e * ST_NT;
+                if (p < nk * nf4) *reinterpret_cast<float4*>(ks + (p / nf4) * ld + (p % nf4) * 4) = kreg[e];
             }
+            for (int p = KREG * ST_NT + tid; p < nk * nf4; p += ST_NT)
+                *reinterpret_cast<float4*>(ks + (p / nf4) * ld + (p % nf4) * 4) =
+                    *reinterpret_cast<const float4*>(kb_base + (size_t)(b0 + p / nf4) * d + (p % nf4) * 4);
             __syncthreads();
+            if (b0 + ST_KC < cmax) load_chunk(b0 + ST_KC);
             // register tile: thread -> rows 4*rg .. 4*rg+3, blocks bg, bg+16, bg+32, bg+48
             const int rg = tid >> 4, bg = tid & 15;
             float acc[4][4];

@@ -200,7 +200,9 @@ nsa_status nsa_get_device_status(int32_t* status);
 #define NSA_PATH_ROWWISE 0       /* shapes outside the tensor-core kernels' limits */
 #define NSA_PATH_QUERY_MAJOR 1   /* tensor cores; selected branch over each tile's block union */
 #define NSA_PATH_BLOCK_MAJOR 2   /* + selected branch block-major (long prefills, full workspace) */
-#define NSA_PATH_SPLIT_K 3       /* + each tile's keys split over several CTAs (few tiles, e.g. decode) */
+#define NSA_PATH_SPLIT_K 3       /* + each tile's keys split over several CTAs (few tiles) */
+#define NSA_PATH_DECODE 4        /* tensor cores with the keys as the MMA M dimension: <= 4 query
+                                    rows per sequence, 8 or 16 heads per group, d_v 128, full workspace */
 
 /*
  * The organisation nsa_sparse_attn_fwd picks for `cfg` with a workspace of
@@ -227,8 +229,9 @@ nsa_status nsa_attn_plan(const nsa_config* cfg, int select_inside, size_t ws_byt
  * no call was timed).  Stage names: "select" (score + top-k when idx is
  * NULL), "index" (block-major inverted index), "sel_bm" (block-major selected
  * branch), "sel_merge", "attn_tc" (tensor-core branches + gated merge),
- * "split_merge", "rowwise".  Each stage's time runs from its first launch to
- * the next stage's first launch on the same stream.
+ * "split_merge", "attn_dec" (few-query kernel), "dec_merge", "rowwise".
+ * Each stage's time runs from its first launch to the next stage's first
+ * launch on the same stream.
  */
 #define NSA_TIMING_MAX_STAGES 8
 nsa_status nsa_timing_enable(int32_t on);

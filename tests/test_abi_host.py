@@ -64,11 +64,13 @@ def test_workspace_sizes(abi):
     wl = WORKLOADS["nsa64k"]
     n = abi.nsa_workspace_size(abi.config(wl))
     assert n >= wl.seqlen_q * wl.h_kv * wl.top_k * wl.group * wl.d_v * 2
-    # decode keeps the selected branch in the query-major kernel and splits each
-    # tile's keys over several CTAs (partials + merge)
+    # decode runs the few-query kernel (keys as the MMA M dimension, partials + merge)
     wl = WORKLOADS["decode64x64k"]
     cfg = abi.config(wl)
-    assert abi.nsa_attn_plan(cfg, True, abi.nsa_workspace_size(cfg))[0] == "split-k"
+    assert abi.nsa_attn_plan(cfg, True, abi.nsa_workspace_size(cfg)) == ("decode", 3)
+    # 4 heads per group: the query-major kernel with each tile's keys split over CTAs
+    cfg4 = abi.config(WORKLOADS["tiny"].with_(seqlen_q=1, seqlen_kv=900, q_pos0=899))
+    assert abi.nsa_attn_plan(cfg4, True, abi.nsa_workspace_size(cfg4))[0] == "split-k"
     assert abi.nsa_attn_plan(cfg, True, abi.nsa_workspace_size_min(cfg))[0] == "query-major"
     assert abi.nsa_attn_plan(abi.config(WORKLOADS["nsa64k"]), True,
                              abi.nsa_workspace_size(abi.config(WORKLOADS["nsa64k"])))[0] == "block-major"

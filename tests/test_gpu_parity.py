@@ -50,6 +50,22 @@ EDGE = {
     "few_queries": TINY.with_(name="few_queries", seqlen_q=5, seqlen_kv=900, q_pos0=895),
     "decode_small": WORKLOADS["decode64x64k"].with_(name="decode_small", batch=3, seqlen_kv=3000,
                                                      q_pos0=2999),
+    # few-query kernel (keys as the MMA M dimension): groups of 8 and 16 heads, up to 4 queries,
+    # caches shorter than the window / a compressed block, ragged blocks, 128-key blocks,
+    # selected-only ungated
+    "dec_g8_tq3": WORKLOADS["decode64x64k"].with_(name="dec_g8_tq3", batch=2, seqlen_q=3,
+                                                   seqlen_kv=2500, q_pos0=2497, h_q=16, h_kv=2,
+                                                   d_qk=128),
+    "dec_short": WORKLOADS["decode64x64k"].with_(name="dec_short", batch=2, seqlen_kv=100,
+                                                  q_pos0=99),
+    "dec_tiny_cache": WORKLOADS["decode64x64k"].with_(name="dec_tiny_cache", batch=2, seqlen_kv=20,
+                                                       q_pos0=19),
+    "dec_ragged": WORKLOADS["decode64x64k"].with_(name="dec_ragged", batch=2, seqlen_kv=1000,
+                                                   q_pos0=999, d_qk=64),
+    "dec_bs128": WORKLOADS["decode64x64k"].with_(name="dec_bs128", batch=2, seqlen_kv=3000,
+                                                  q_pos0=2999, sel_block=128, top_k=8),
+    "dec_sel_only": WORKLOADS["decode64x64k"].with_(name="dec_sel_only", batch=2, seqlen_kv=1500,
+                                                     q_pos0=1499, branches=BR_SEL, gated=False),
     # block-major selected branch (groups of 8 and 16 heads, sel_block 64, >= 256 queries)
     "bm_g8_ragged": WORKLOADS["nsa64k"].with_(name="bm_g8_ragged", seqlen_q=1000, seqlen_kv=1000,
                                               h_q=16, h_kv=2, d_qk=128, d_v=128),
