@@ -64,34 +64,40 @@ struct DecArgs {
     float scale_log2;
 };
 
+constexpr int NKS = 3;              // K stages (released when QK completes)
+constexpr int NVS = 2;              // V stages (released when PV completes)
+
 template <int DQK>
 struct DecSmem {
     static constexpr int QC = DQK / 64;
-    static constexpr int K_OFF = 0;                             // 2 stages x QC chunks
-    static constexpr int V_OFF = K_OFF + 2 * QC * CH;           // 2 stages x 2 chunks
-    static constexpr int Q_OFF = V_OFF + 2 * 2 * CH;            // 2 buffers x QC chunks
-    static constexpr int P_OFF = Q_OFF + 2 * QC * QCH;          // 2 buffers x 2 chunks
-    static constexpr int RED_OFF = P_OFF + 2 * 2 * PCH;         // [4 warps][NH] fp32
-    static constexpr int BAR_OFF = RED_OFF + 4 * NH * 4;
-    // q_full[2] q_empty[2] kv_full[2] kv_empty[2] s_full[2] s_free[2] p_full[2] pv_done[2]
-    // o_full o_free
-    static constexpr int NBAR = 18;
+    static constexpr int K_OFF = 0;                             // NKS stages x QC chunks
+    static constexpr int V_OFF = K_OFF + NKS * QC * CH;         // NVS stages x 2 chunks
+    static constexpr int Q_OFF = V_OFF + NVS * 2 * CH;          // 2 buffers x QC chunks
+    static constexpr int P_OFF = Q_OFF + 2 * QC * QCH;          // 1 buffer x 2 chunks
+    static constexpr int RED_OFF = P_OFF + 2 * PCH;             // [3][4 warps][NH] fp32
+    static constexpr int BAR_OFF = RED_OFF + 3 * 4 * NH * 4;
+    // q_full[2] q_empty[2] k_full[3] k_empty[3] v_full[2] v_empty[2] s_full[2] s_free[2]
+    // p_full pv_done o_full o_free
+    static constexpr int NBAR = 22;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int ALLOC = MISC_OFF + 64 + 1024;
+    static_assert(ALLOC <= 232448, "shared memory");
 };
 
 struct DecBars {
     uint64_t* b;
     __device__ __forceinline__ uint64_t* q_full(int i) const { return b + i; }
     __device__ __forceinline__ uint64_t* q_empty(int i) const { return b + 2 + i; }
-    __device__ __forceinline__ uint64_t* kv_full(int i) const { return b + 4 + i; }
-    __device__ __forceinline__ uint64_t* kv_empty(int i) const { return b + 6 + i; }
-    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 8 + i; }
-    __device__ __forceinline__ uint64_t* s_free(int i) const { return b + 10 + i; }
-    __device__ __forceinline__ uint64_t* p_full(int i) const { return b + 12 + i; }
-    __device__ __forceinline__ uint64_t* pv_done(int i) const { return b + 14 + i; }
-    __device__ __forceinline__ uint64_t* o_full() const { return b + 16; }
-    __device__ __forceinline__ uint64_t* o_free() const { return b + 17; }
+    __device__ __forceinline__ uint64_t* k_full(int i) const { return b + 4 + i; }
+    __device__ __forceinline__ uint64_t* k_empty(int i) const { return b + 7 + i; }
+    __device__ __forceinline__ uint64_t* v_full(int i) const { return b + 10 + i; }
+    __device__ __forceinline__ uint64_t* v_empty(int i) const { return b + 12 + i; }
+    __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 14 + i; }
+    __device__ __forceinline__ uint64_t* s_free(int i) const { return b + 16 + i; }
+    __device__ __forceinline__ uint64_t* p_full() const { return b + 18; }
+    __device__ __forceinline__ uint64_t* pv_done() const { return b + 19; }
+    __device__ __forceinline__ uint64_t* o_full() const { return b + 20; }
+    __device__ __forceinline__ uint64_t* o_free() const { return b + 21; }
 };
 
 // What one work item covers; every role derives it the same way.
@@ -188,13 +194,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bar.q_full(i), 1);
             tc::mbar_init(bar.q_empty(i), 1);
-            tc::mbar_init(bar.kv_full(i), 1);
-            tc::mbar_init(bar.kv_empty(i), 1);
+            tc::mbar_init(bar.v_full(i), 1);
+            tc::mbar_init(bar.v_empty(i), 1);
             tc::mbar_init(bar.s_full(i), 1);
             tc::mbar_init(bar.s_free(i), 4);
-            tc::mbar_init(bar.p_full(i), 4);
-            tc::mbar_init(bar.pv_done(i), 1);
         }
+        for (int i = 0; i < NKS; ++i) {
+            tc::mbar_init(bar.k_full(i), 1);
+            tc::mbar_init(bar.k_empty(i), 1);
+        }
+        tc::mbar_init(bar.p_full(), 4);
+        tc::mbar_init(bar.pv_done(), 1);
         tc::mbar_init(bar.o_full(), 1);
         tc::mbar_init(bar.o_free(), 4);
         *abort_flag = 0;
@@ -213,13 +223,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // K of tile n is loaded as soon as QK(n - NKS) has completed; V of tile n
+        // is issued after K of tile n + 1, so the value loads never hold back
+        // the key loads that the MMA needs first.
         bool ok = true;
-        uint32_t tcount = 0, qcount = 0;
+        uint32_t kcount = 0, vcount = 0, qcount = 0;
+        struct VJob {
+            int cmp, sel, row0, row1, plane;
+        } pend{0, 0, 0, 0, -1};
+        auto issue_v = [&](const VJob& v) -> bool {
+            const int vs = vcount & 1;
+            if (!dec_warp_wait(bar.v_empty(vs), ((vcount >> 1) & 1) ^ 1, abort_flag)) return false;
+            uint8_t* vst = sm + L::V_OFF + vs * 2 * CH;
+            if (v.sel) {
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar.v_full(vs), 2 * CH);
+                __syncwarp();
+                if (lane < 4) {
+                    const int h = lane >> 1, c = lane & 1;
+                    tc::tma_load_3d(vst + c * CH + h * (CH / 2), &map_v64, bar.v_full(vs), 64 * c,
+                                    h ? v.row1 : v.row0, v.plane);
+                }
+            } else {
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar.v_full(vs), 2 * CH);
+                __syncwarp();
+                if (lane < 2)
+                    tc::tma_load_3d(vst + lane * CH, v.cmp ? &map_vc : &map_v128, bar.v_full(vs), 64 * lane,
+                                    v.row0, v.plane);
+            }
+            ++vcount;
+            return true;
+        };
         for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
             const Item it = item_info(a, item);
             if (it.t0 >= it.t1) continue;
-            const int kvh = it.u;                    // group-shared selection: unit = KV head
-            const int plane = it.b * s.Hkv + kvh;
+            const int plane = it.b * s.Hkv + it.u;   // group-shared selection: unit = KV head
             const int qb = qcount & 1;
             if (!dec_warp_wait(bar.q_empty(qb), ((qcount >> 1) & 1) ^ 1, abort_flag)) {
                 ok = false;
@@ -231,52 +268,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::tma_load_4d(sm + L::Q_OFF + (qb * L::QC + lane) * QCH, &map_q, bar.q_full(qb),
                                 64 * lane, it.u * a.hpt, it.i, it.b);
             ++qcount;
-            for (int j = it.t0; j < it.t1; ++j, ++tcount) {
-                const int st = tcount & 1;
-                if (!dec_warp_wait(bar.kv_empty(st), ((tcount >> 1) & 1) ^ 1, abort_flag)) {
+            for (int j = it.t0; j < it.t1; ++j) {
+                VJob cur{it.br == B_CMP, it.br == B_SEL, 0, 0, plane};
+                if (it.br == B_SEL) {
+                    // an odd last segment is paired with itself (masked by the softmax),
+                    // so that a stage never holds stale or uninitialised rows
+                    const int e1 = 2 * j + 1;
+                    cur.row0 = seg_start(a, it, 2 * j);
+                    cur.row1 = e1 < it.nseg ? seg_start(a, it, e1) : cur.row0;
+                } else {
+                    cur.row0 = cur.cmp ? j * DT : it.win_lo + j * DT;
+                }
+                const int ks = kcount % NKS;
+                if (!dec_warp_wait(bar.k_empty(ks), ((kcount / NKS) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                uint8_t* kst = sm + L::K_OFF + st * L::QC * CH;
-                uint8_t* vst = sm + L::V_OFF + st * 2 * CH;
-                if (it.br == B_SEL) {
-                    // an odd last segment is paired with itself (masked by the softmax),
-                    // so that the stage never holds stale or uninitialised V rows
-                    const int e0 = 2 * j, e1 = 2 * j + 1;
-                    const int r0 = seg_start(a, it, e0);
-                    const int r1 = e1 < it.nseg ? seg_start(a, it, e1) : r0;
-                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.kv_full(st), 2 * (L::QC + 2) * (CH / 2));
-                    __syncwarp();
-                    // lanes [0, QC) K chunks, [QC, QC+2) V chunks; second segment on lanes +8
-                    const int h = lane >> 3, c = lane & 7;
-                    if (h < 2 && c < L::QC + 2) {
-                        const int row = h ? r1 : r0;
-                        if (c < L::QC)
-                            tc::tma_load_3d(kst + c * CH + h * (CH / 2), &map_k64, bar.kv_full(st), 64 * c, row, plane);
-                        else
-                            tc::tma_load_3d(vst + (c - L::QC) * CH + h * (CH / 2), &map_v64, bar.kv_full(st),
-                                            64 * (c - L::QC), row, plane);
+                uint8_t* kst = sm + L::K_OFF + ks * L::QC * CH;
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar.k_full(ks), L::QC * CH);
+                __syncwarp();
+                if (cur.sel) {
+                    if (lane < 2 * L::QC) {
+                        const int h = lane / L::QC, c = lane % L::QC;
+                        tc::tma_load_3d(kst + c * CH + h * (CH / 2), &map_k64, bar.k_full(ks), 64 * c,
+                                        h ? cur.row1 : cur.row0, plane);
                     }
-                } else {
-                    const bool cmp = it.br == B_CMP;
-                    const int row = cmp ? j * DT : it.win_lo + j * DT;
-                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.kv_full(st), (L::QC + 2) * CH);
-                    __syncwarp();
-                    if (lane < L::QC)
-                        tc::tma_load_3d(kst + lane * CH, cmp ? &map_kc : &map_k128, bar.kv_full(st), 64 * lane, row, plane);
-                    else if (lane < L::QC + 2)
-                        tc::tma_load_3d(vst + (lane - L::QC) * CH, cmp ? &map_vc : &map_v128, bar.kv_full(st),
-                                        64 * (lane - L::QC), row, plane);
+                } else if (lane < L::QC) {
+                    tc::tma_load_3d(kst + lane * CH, cur.cmp ? &map_kc : &map_k128, bar.k_full(ks), 64 * lane,
+                                    cur.row0, plane);
                 }
+                ++kcount;
+                if (pend.plane >= 0 && !issue_v(pend)) {
+                    ok = false;
+                    break;
+                }
+                pend = cur;
             }
         }
+        if (ok && pend.plane >= 0 && !issue_v(pend)) ok = false;
         if (!ok) dec_abort(abort_flag);
         // wait for every copy still in flight before the CTA may exit
         volatile int never = 0;
+        for (uint32_t st = 0; st < NKS; ++st)
+            if (kcount > st) {
+                const uint32_t last = st + ((kcount - 1 - st) / NKS) * NKS;
+                tc::mbar_wait(bar.k_full(st), (last / NKS) & 1, &never, WAIT_NS);
+            }
         for (uint32_t st = 0; st < 2; ++st) {
-            if (tcount > st) {
-                const uint32_t last = st + ((tcount - 1 - st) / 2) * 2;
-                tc::mbar_wait(bar.kv_full(st), (last >> 1) & 1, &never, WAIT_NS);
+            if (vcount > st) {
+                const uint32_t last = st + ((vcount - 1 - st) / 2) * 2;
+                tc::mbar_wait(bar.v_full(st), (last >> 1) & 1, &never, WAIT_NS);
             }
             if (qcount > st) {
                 const uint32_t last = st + ((qcount - 1 - st) / 2) * 2;
@@ -294,22 +335,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t p_base = tc::smem_u32(sm + L::P_OFF);
             bool ok = true;
             uint32_t tcount = 0, qcount = 0, ocount = 0;
+            // O^T += V^T P^T for tile n (V stage n & 1, the single P buffer)
             auto issue_pv = [&](uint32_t n, bool first) -> bool {
-                const int pb = n & 1;
-                if (!tc::mbar_wait(bar.p_full(pb), (n >> 1) & 1, abort_flag, WAIT_NS)) return false;
+                const int vs = n & 1;
+                if (!tc::mbar_wait(bar.p_full(), n & 1, abort_flag, WAIT_NS) ||
+                    !tc::mbar_wait(bar.v_full(vs), (n >> 1) & 1, abort_flag, WAIT_NS))
+                    return false;
                 // the first PV of an item overwrites O: the previous item's epilogue must have read it
                 if (first && ocount > 0 && !tc::mbar_wait(bar.o_free(), (ocount - 1) & 1, abort_flag, WAIT_NS))
                     return false;
                 tc::fence_after_sync();
-                const uint32_t vst = v_base + pb * 2 * CH;
-                const uint32_t pst = p_base + pb * 2 * PCH;
+                const uint32_t vst = v_base + vs * 2 * CH;
 #pragma unroll
                 for (int kk = 0; kk < DT / 16; ++kk)
                     tc::mma_ss(tO, tc::sdesc_sw128(vst + kk * 2048, CH, 1024),
-                               tc::sdesc_sw128(pst + (kk >> 2) * PCH + (kk & 3) * 32, 16, 1024), idesc_pv,
+                               tc::sdesc_sw128(p_base + (kk >> 2) * PCH + (kk & 3) * 32, 16, 1024), idesc_pv,
                                (first && kk == 0) ? 0u : 1u);
-                tc::mma_commit(bar.kv_empty(pb));
-                tc::mma_commit(bar.pv_done(pb));
+                tc::mma_commit(bar.v_empty(vs));
+                tc::mma_commit(bar.pv_done());
                 return true;
             };
             for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
@@ -322,20 +365,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 const uint32_t qst = q_base + qb * L::QC * QCH;
                 for (int j = it.t0; j < it.t1; ++j, ++tcount) {
-                    const int st = tcount & 1;
-                    if (!tc::mbar_wait(bar.kv_full(st), (tcount >> 1) & 1, abort_flag, WAIT_NS) ||
-                        (tcount >= 2 && !tc::mbar_wait(bar.s_free(st), ((tcount >> 1) & 1) ^ 1, abort_flag, WAIT_NS))) {
+                    const int ks = tcount % NKS, sb = tcount & 1;
+                    if (!tc::mbar_wait(bar.k_full(ks), (tcount / NKS) & 1, abort_flag, WAIT_NS) ||
+                        (tcount >= 2 && !tc::mbar_wait(bar.s_free(sb), ((tcount >> 1) & 1) ^ 1, abort_flag, WAIT_NS))) {
                         ok = false;
                         break;
                     }
                     tc::fence_after_sync();
-                    const uint32_t kst = k_base + st * L::QC * CH;
+                    const uint32_t kst = k_base + ks * L::QC * CH;
 #pragma unroll
                     for (int kk = 0; kk < DQK / 16; ++kk)
-                        tc::mma_ss(tS(st), tc::sdesc_sw128(kst + (kk >> 2) * CH + (kk & 3) * 32, 16, 1024),
+                        tc::mma_ss(tS(sb), tc::sdesc_sw128(kst + (kk >> 2) * CH + (kk & 3) * 32, 16, 1024),
                                    tc::sdesc_sw128(qst + (kk >> 2) * QCH + (kk & 3) * 32, 16, 1024), idesc_qk,
                                    kk > 0 ? 1u : 0u);
-                    tc::mma_commit(bar.s_full(st));
+                    tc::mma_commit(bar.s_full(sb));
+                    tc::mma_commit(bar.k_empty(ks));
                     if (j == it.t1 - 1) tc::mma_commit(bar.q_empty(qb));
                     if (j > it.t0 && !issue_pv(tcount - 1, j - 1 == it.t0)) {
                         ok = false;
@@ -353,19 +397,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) dec_abort(abort_flag);
             volatile int never = 0;
-            // the last commit arrives once everything issued before it completed
+            // the last epilogue has read O (and every MMA before its commit completed)
             if (ocount > 0) tc::mbar_wait(bar.o_free(), (ocount - 1) & 1, &never, WAIT_NS);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
+        // One vote barrier per tile: it publishes the warps' per-head maxima
+        // (red[tile & 1]) and makes every wait's outcome uniform, so that all
+        // four warps leave together if one of them timed out.
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;            // key of the tile; d_v lane of O^T
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        float* red = reinterpret_cast<float*>(sm + L::RED_OFF);     // [4][NH]
+        float* red = reinterpret_cast<float*>(sm + L::RED_OFF);     // [3][4][NH]
         uint8_t* pbuf = sm + L::P_OFF;
         const int wq = warp - 2;                      // 0..3, slot in red
-        bool ok = true;
+        bool ok = true, ok_prev = true;
         uint32_t tcount = 0, ocount = 0;
         for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
             const Item it = item_info(a, item);
@@ -384,6 +431,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             for (int j = it.t0; j < it.t1; ++j, ++tcount) {
                 const int sb = tcount & 1;
+                float* rt = red + sb * 4 * NH;
                 // key of this thread and whether the query sees it
                 bool valid;
                 if (it.br == B_CMP) {
@@ -408,10 +456,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int h = 0; h < NH; ++h) {
                         x[h] = (valid && h < a.hpt) ? __uint_as_float(sv[h]) * a.scale_log2 : -INFINITY;
                         const int m = warp_max_i(f2ord(x[h]));
-                        if (lane == h) red[wq * NH + h] = ord2f(m);
+                        if (lane == h) rt[wq * NH + h] = ord2f(m);
                     }
                 }
-                if (!tc::named_bar_and(1, 128, okw)) {
+                if (!tc::named_bar_and(1, 128, okw && ok_prev)) {
                     ok = false;
                     break;
                 }
@@ -420,7 +468,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float alpha[NH];
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
-                    const float tm = fmaxf(fmaxf(red[h], red[NH + h]), fmaxf(red[2 * NH + h], red[3 * NH + h]));
+                    const float tm = fmaxf(fmaxf(rt[h], rt[NH + h]), fmaxf(rt[2 * NH + h], rt[3 * NH + h]));
                     alpha[h] = 1.f;
                     if (tm > mrun[h] + 8.f) {
                         alpha[h] = tc::ex2(mrun[h] - tm);      // 0 when mrun = -inf
@@ -429,11 +477,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         rescale = true;
                     }
                 }
-                bool ok2 = true;
-                if (rescale && j > it.t0) {
-                    // O^T holds tiles < j: wait for PV(j - 1), then scale its head columns
-                    ok2 = dec_warp_wait(bar.pv_done((tcount - 1) & 1), ((tcount - 1) >> 1) & 1, abort_flag);
-                    if (ok2) {
+                // the P buffer (and O, for a rescale) is free once PV of the previous tile completed
+                ok_prev = tcount == 0 || dec_warp_wait(bar.pv_done(), (tcount - 1) & 1, abort_flag);
+                if (ok_prev) {
+                    if (rescale && j > it.t0) {
                         tc::fence_after_sync();
                         uint32_t ov[NH];
                         tc::tmem_ld16(tO + lane_off, ov);
@@ -443,12 +490,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tc::tmem_st16(tO + lane_off, ov);
                         tc::tmem_wait_st();
                     }
-                }
-                // P^T buffer sb was last read by PV(tcount - 2)
-                if (ok2 && tcount >= 2)
-                    ok2 = dec_warp_wait(bar.pv_done(sb), ((tcount >> 1) & 1) ^ 1, abort_flag);
-                if (ok2) {
-                    uint8_t* pb = pbuf + sb * 2 * PCH + (r >> 6) * PCH;
+                    uint8_t* pb = pbuf + (r >> 6) * PCH;
                     const int unit16 = (r & 63) >> 3;
 #pragma unroll
                     for (int h = 0; h < NH; ++h) {
@@ -460,16 +502,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tc::fence_before_sync();
                     tc::fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
-                }
-                if (!tc::named_bar_and(1, 128, ok2)) {
-                    ok = false;
-                    break;
+                    if (lane == 0) tc::mbar_arrive(bar.p_full());
                 }
             }
             if (!ok) break;
             // epilogue: o = O^T / l per head, lse = m + log2 l
             bool okw = dec_warp_wait(bar.o_full(), ocount & 1, abort_flag);
+            float* rs = red + 2 * 4 * NH;
             uint32_t ov[NH];
             if (okw) {
                 tc::fence_after_sync();
@@ -481,22 +520,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
                     const float v = warp_sum(lsum[h]);
-                    if (lane == h) red[wq * NH + h] = v;
+                    if (lane == h) rs[wq * NH + h] = v;
                 }
             }
-            if (!tc::named_bar_and(1, 128, okw)) {
+            if (!tc::named_bar_and(1, 128, okw && ok_prev)) {
                 ok = false;
                 break;
             }
             ++ocount;
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
-                const float l = (red[h] + red[NH + h]) + (red[2 * NH + h] + red[3 * NH + h]);
+                const float l = (rs[h] + rs[NH + h]) + (rs[2 * NH + h] + rs[3 * NH + h]);
                 if (h < a.hpt) po[h * DV + r] = l > 0.f ? __uint_as_float(ov[h]) / l : 0.f;
                 if (r == h) pl[h] = l > 0.f ? mrun[h] + __log2f(l) : -INFINITY;
             }
-            // red is rewritten by the next tile only after everyone has read it
-            tc::named_bar_sync(1, 128);
         }
         if (!ok) dec_abort(abort_flag);
     }
