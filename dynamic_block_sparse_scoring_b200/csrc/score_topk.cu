@@ -17,7 +17,11 @@
 // and then by lower block id.
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace nsa {
 
@@ -27,6 +31,51 @@ constexpr int ST_NT = 256;  // threads per CTA (8 warps x 8 rows of top-k state)
 constexpr int ST_RPW = ST_RT / 8;   // rows per warp
 
 enum { MODE_SELECT = 0, MODE_SCORES = 1, MODE_SELECT_FROM_SCORES = 2 };
+
+// Merges the 32 candidate keys of a warp (one per lane, 0 = none) into the
+// warp's running list: the K1 largest keys so far, descending, one per lane
+// (lanes >= K1 hold 0); `thr` is the list's smallest key (lane K1 - 1).
+// A few survivors of the threshold are inserted one at a time; four or more
+// are bitonic-sorted across the lanes and bitonic-merged with the list.
+__device__ __forceinline__ void warp_list_merge(unsigned long long& key, unsigned long long& thr,
+                                                unsigned long long ck, int K1, int lane) {
+    unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
+    if (__popc(mask) >= 4) {
+        unsigned long long v = ck > thr ? ck : 0ull;
+#pragma unroll
+        for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+                const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+                v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+            }
+        // v descending; the larger of key[l] and v[31 - l] is the top 32 of both, bitonic
+        const unsigned long long vr = __shfl_sync(0xffffffffu, v, 31 - lane);
+        unsigned long long w = key > vr ? key : vr;
+#pragma unroll
+        for (int j = 16; j > 0; j >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, w, j);
+            w = (lane & j) == 0 ? (w > o ? w : o) : (w < o ? w : o);
+        }
+        key = lane < K1 ? w : 0ull;
+        thr = __shfl_sync(0xffffffffu, key, K1 - 1);
+        return;
+    }
+    while (mask) {
+        const int src = __ffs(mask) - 1;
+        const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
+        const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && key > x));
+        const unsigned long long up = __shfl_up_sync(0xffffffffu, key, 1);
+        if (lane < K1) {
+            if (lane == p) key = x;
+            else if (lane > p) key = up;
+        }
+        thr = __shfl_sync(0xffffffffu, key, K1 - 1);
+        mask &= ~(1u << src);
+        mask &= __ballot_sync(0xffffffffu, ck > thr);
+    }
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
@@ -189,21 +238,7 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
                     const int jj = lane + 32 * half;
                     const float sv = ss[r * (ST_KC + 1) + jj];
                     const unsigned long long ck = (sv != -INFINITY) ? score_key(sv, b0 + jj) : 0ull;
-                    unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
-                    while (mask) {
-                        const int src = __ffs(mask) - 1;
-                        const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
-                        const unsigned long long mine = key[j];
-                        const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && mine > x));
-                        const unsigned long long up = __shfl_up_sync(0xffffffffu, mine, 1);
-                        if (lane < K1) {
-                            if (lane == p) key[j] = x;
-                            else if (lane > p) key[j] = up;
-                        }
-                        thr = __shfl_sync(0xffffffffu, key[j], K1 - 1);
-                        mask &= ~(1u << src);
-                        mask &= __ballot_sync(0xffffffffu, ck > thr);
-                    }
+                    warp_list_merge(key[j], thr, ck, K1, lane);
                 }
             }
         }
@@ -242,19 +277,31 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
     }
 }
 
-// Few query rows (decode): one CTA per (query, unit, sequence).  Each of its
-// 32 warps scores a contiguous range of past blocks (the lanes split the d_qk
-// dot product, so a pooled key row is one coalesced read) and keeps its own
-// running top-(k-1); the warp lists are then merged by warp 0.
-constexpr int SR_NT = 1024;             // 32 warps: more pooled rows in flight per CTA
+// Few query rows (decode): a cluster of SR_CL CTAs per (query, unit,
+// sequence).  Each CTA scores an equal share of the past blocks into its
+// shared memory: its warps take 16 pooled rows at a time with every load
+// issued before any is used (the lanes split the d_qk dot product, so a
+// pooled row is one coalesced read), which keeps the memory round trips per
+// CTA to one or two.  CTA 0 then reads the cluster's scores through
+// distributed shared memory, warp w taking CTA w's share into a running
+// top-(k-1), and the eight warp lists are merged as a tree.
+constexpr int SR_CL = 8;                // CTAs per query row (cluster size)
+constexpr int SR_NT = 256;
 constexpr int SR_NW = SR_NT / 32;
+constexpr int SR_QLD = 256;             // row stride of the per-head query staging
+constexpr int SR_MAXC = 512;            // scores per CTA: up to SR_CL * 512 past blocks
+constexpr int SR_RB = 16;               // pooled rows per load round of a warp
 
-__global__ void __launch_bounds__(SR_NT, 1) select_rows_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
-                                                            const float* __restrict__ kbar,
-                                                            int32_t* __restrict__ idx) {
+__global__ void __cluster_dims__(SR_CL, 1, 1) __launch_bounds__(SR_NT, 2)
+    select_rows_kernel(Shape s, const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
+                       int32_t* __restrict__ idx) {
     __shared__ float qs[256];
+    __shared__ float qh[16 * SR_QLD];                 // per-head query rows (<= 16 heads)
+    __shared__ float sc[SR_MAXC];                     // this CTA's scores
     __shared__ unsigned long long lists[SR_NW][32];
-    const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    const int i = blockIdx.x / SR_CL, u = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int d = s.dqk;
     const int kvh = s.per_head ? u / s.G : u;
@@ -263,90 +310,103 @@ __global__ void __launch_bounds__(SR_NT, 1) select_rows_kernel(Shape s, const __
     const int cr = t / s.bs;
     const int ncand = min(cr, s.nb_full);
     const int K1 = s.topk - 1;
-    for (int c = tid; c < d; c += SR_NT) {
-        float acc = 0.f;
-        const __nv_bfloat16* src = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d + c;
-        for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += bf2f(src[(size_t)hh * d]);
-        qs[c] = acc;
+    // summed query: 16-byte loads of (head, 8 columns), all issued before any is
+    // used (one memory round trip), staged per head and summed in head order
+    {
+        const int nvec = d / 8, np = s.heads_per_unit * nvec;
+        const uint4* src = reinterpret_cast<const uint4*>(q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d);
+        for (int p0 = 0; p0 < np; p0 += 4 * SR_NT) {
+            uint4 raw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (p0 + tid + e * SR_NT < np) raw[e] = src[p0 + tid + e * SR_NT];   // head h at h * nvec
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int p = p0 + tid + e * SR_NT;
+                if (p < np) unpack8(raw[e], qh + (p / nvec) * SR_QLD + (p % nvec) * 8);
+            }
+        }
+        __syncthreads();
+        for (int c = tid; c < d; c += SR_NT) {
+            float acc = 0.f;
+            for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += qh[hh * SR_QLD + c];
+            qs[c] = acc;
+        }
     }
     __syncthreads();
-    unsigned long long key = 0ull;               // this lane's slot of the warp's list
-    unsigned long long thr = 0ull;
-    const int per = (ncand + SR_NW - 1) / SR_NW;
-    const int j0 = warp * per, j1 = min(ncand, j0 + per);
-    const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * d;
-    for (int jb = j0; jb < j1; jb += 32) {
-        // 32 blocks per round: every lane ends up holding the score of block jb + lane
-        float mine = -INFINITY;
-        for (int jj = 0; jj < 32 && jb + jj < j1; jj += 8) {
-            // eight pooled rows in flight at once
-            float part[8];
+    // this CTA's share of the past blocks, scored into sc[]
+    const int per_cta = (ncand + SR_CL - 1) / SR_CL;
+    const int c0 = crank * per_cta, n_cta = max(0, min(ncand, c0 + per_cta) - c0);
+    const float* kb = kbar + ((size_t)(b * s.Hkv + kvh) * s.nb_full + c0) * d;
+    const int ncc = (d + 31) / 32;                    // 2..8 columns per lane
+    for (int r0 = warp * SR_RB; r0 < n_cta; r0 += SR_NW * SR_RB) {
+        // every load of the round first, then the dot products
+        float v[SR_RB][6];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                part[e] = 0.f;
-                if (jb + jj + e < j1) {
-                    const float* row = kb + (size_t)(jb + jj + e) * d;
+        for (int e = 0; e < SR_RB; ++e) {
+            const float* row = kb + (size_t)min(r0 + e, n_cta - 1) * d;
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {      // d <= 256: all loads issued together
-                        const int c = lane + 32 * cc;
-                        if (c < d) part[e] = fmaf(qs[c], row[c], part[e]);
-                    }
-                }
-            }
+            for (int cc = 0; cc < 6; ++cc) v[e][cc] = cc < ncc ? __ldg(row + lane + 32 * cc) : 0.f;
+        }
+        float part[SR_RB];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float tot = warp_sum(part[e]);
-                if (lane == jj + e) mine = s.scale * tot;
+        for (int e = 0; e < SR_RB; ++e) {
+            part[e] = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 6; ++cc)
+                if (cc < ncc) part[e] = fmaf(qs[lane + 32 * cc], v[e][cc], part[e]);
+        }
+        // d = 256: the last two columns of each lane
+        if (ncc > 6) {
+#pragma unroll
+            for (int e = 0; e < SR_RB; ++e) {
+                const float* row = kb + (size_t)min(r0 + e, n_cta - 1) * d;
+                part[e] = fmaf(qs[lane + 192], __ldg(row + lane + 192), part[e]);
+                part[e] = fmaf(qs[lane + 224], __ldg(row + lane + 224), part[e]);
             }
         }
-        if (K1 > 0) {
-            const unsigned long long ck = (jb + lane < j1) ? score_key(mine, jb + lane) : 0ull;
-            unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
-            while (mask) {
-                const int src = __ffs(mask) - 1;
-                const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
-                const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && key > x));
-                const unsigned long long up = __shfl_up_sync(0xffffffffu, key, 1);
-                if (lane < K1) {
-                    if (lane == p) key = x;
-                    else if (lane > p) key = up;
-                }
-                thr = __shfl_sync(0xffffffffu, key, K1 - 1);
-                mask &= ~(1u << src);
-                mask &= __ballot_sync(0xffffffffu, ck > thr);
-            }
+#pragma unroll
+        for (int e = 0; e < SR_RB; ++e) {
+            const float tot = warp_sum(part[e]);
+            if (lane == 0 && r0 + e < n_cta) sc[r0 + e] = s.scale * tot;
         }
     }
-    lists[warp][lane] = key;
-    __syncthreads();
-    if (warp != 0) return;
-    // merge the other warps' lists into warp 0's
-    for (int w = 1; w < SR_NW && K1 > 0; ++w) {
-        const unsigned long long ck = lists[w][lane];
-        unsigned mask = __ballot_sync(0xffffffffu, ck > thr);
-        while (mask) {
-            const int src = __ffs(mask) - 1;
-            const unsigned long long x = __shfl_sync(0xffffffffu, ck, src);
-            const int p = __popc(__ballot_sync(0xffffffffu, lane < K1 && key > x));
-            const unsigned long long up = __shfl_up_sync(0xffffffffu, key, 1);
-            if (lane < K1) {
-                if (lane == p) key = x;
-                else if (lane > p) key = up;
+    cluster.sync();
+    if (crank == 0) {
+        // warp w: top-(k-1) of CTA w's scores
+        unsigned long long key = 0ull, thr = 0ull;
+        const int w0 = warp * per_cta, nw = max(0, min(ncand, w0 + per_cta) - w0);
+        const float* rsc = cluster.map_shared_rank(sc, warp);
+        if (K1 > 0)
+            for (int e0 = 0; e0 < nw; e0 += 32) {
+                const int e = e0 + lane;
+                const unsigned long long ck = e < nw ? score_key(rsc[e], w0 + e) : 0ull;
+                warp_list_merge(key, thr, ck, K1, lane);
             }
-            thr = __shfl_sync(0xffffffffu, key, K1 - 1);
-            mask &= ~(1u << src);
-            mask &= __ballot_sync(0xffffffffu, ck > thr);
+        lists[warp][lane] = key;
+        __syncthreads();
+        // tree merge of the warp lists: 8 -> 4 -> 2 -> 1
+        for (int step = 1; step < SR_NW; step <<= 1) {
+            if ((warp & (2 * step - 1)) == 0 && K1 > 0) {
+                warp_list_merge(key, thr, lists[warp + step][lane], K1, lane);
+                lists[warp][lane] = key;
+            }
+            __syncthreads();
+        }
+        if (warp == 0) {
+            const bool have = lane < K1 && key != 0ull;
+            const int blk = have ? key_block(key) : 0x7fffffff;
+            const int npast = __popc(__ballot_sync(0xffffffffu, have));
+            int rank = 0;
+            for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, blk, o) < blk) ? 1 : 0;
+            int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
+            if (have) dst[rank] = blk;
+            if (lane == 0) dst[npast] = cr;
+            if (lane > npast && lane < s.topk) dst[lane] = -1;
         }
     }
-    const bool have = lane < K1 && key != 0ull;
-    const int blk = have ? key_block(key) : 0x7fffffff;
-    const int npast = __popc(__ballot_sync(0xffffffffu, have));
-    int rank = 0;
-    for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, blk, o) < blk) ? 1 : 0;
-    int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
-    if (have) dst[rank] = blk;
-    if (lane == 0) dst[npast] = cr;
-    if (lane > npast && lane < s.topk) dst[lane] = -1;
+    // every CTA's scores stay in place until CTA 0 has read them
+    cluster.sync();
 }
 
 cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
@@ -367,9 +427,9 @@ cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const floa
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         score_topk_kernel<MODE_SELECT_FROM_SCORES><<<grid, ST_NT, smem, st>>>(
             s, nullptr, nullptr, scores_in, nullptr, idx);
-    } else if (s.Tq <= 16) {
+    } else if (s.Tq <= 16 && s.heads_per_unit <= 16 && s.nb_full <= SR_CL * SR_MAXC) {
         // few query rows: a 64-row score tile would be mostly empty
-        select_rows_kernel<<<dim3(s.Tq, s.Hsel, s.B), SR_NT, 0, st>>>(s, q, kbar, idx);
+        select_rows_kernel<<<dim3(s.Tq * SR_CL, s.Hsel, s.B), SR_NT, 0, st>>>(s, q, kbar, idx);
     } else {
         cudaFuncSetAttribute(score_topk_kernel<MODE_SELECT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
