@@ -113,4 +113,5 @@ cudaError_t launch_attn_dec(const Shape& s, const __nv_bfloat16* q, const __nv_b
 cudaError_t launch_dec_merge(const Shape& s, const float* part_o, const float* part_lse,
                              const float* gates, __nv_bfloat16* out, cudaStream_t st);
 int read_and_clear_dec_status();
+int read_and_clear_select_status();
 }  // namespace nsa

@@ -442,8 +442,9 @@ nsa_status nsa_get_device_status(int32_t* status) {
     const int v1 = nsa::read_and_clear_tc_status();
     const int v2 = nsa::read_and_clear_bm_status();
     const int v3 = nsa::read_and_clear_dec_status();
-    if (v1 < 0 || v2 < 0 || v3 < 0) return NSA_ERR_CUDA;
-    *status = v1 ? v1 : (v2 ? v2 : v3);
+    const int v4 = nsa::read_and_clear_select_status();
+    if (v1 < 0 || v2 < 0 || v3 < 0 || v4 < 0) return NSA_ERR_CUDA;
+    *status = v1 ? v1 : (v2 ? v2 : (v3 ? v3 : v4));
     return NSA_OK;
 }
 

@@ -17,13 +17,13 @@
 // and then by lower block id.
 #include <math.h>
 
-#include <cooperative_groups.h>
-
 #include "common.cuh"
+#include "tc.cuh"
 
-namespace cg = cooperative_groups;
 
 namespace nsa {
+
+__device__ int g_select_status = 0;
 
 constexpr int ST_RT = 64;   // query rows per CTA
 constexpr int ST_KC = 64;   // pooled keys per chunk
@@ -277,31 +277,32 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
     }
 }
 
-// Few query rows (decode): a cluster of SR_CL CTAs per (query, unit,
-// sequence).  Each CTA scores an equal share of the past blocks into its
-// shared memory: its warps take 16 pooled rows at a time with every load
-// issued before any is used (the lanes split the d_qk dot product, so a
-// pooled row is one coalesced read), which keeps the memory round trips per
-// CTA to one or two.  CTA 0 then reads the cluster's scores through
-// distributed shared memory, warp w taking CTA w's share into a running
-// top-(k-1), and the eight warp lists are merged as a tree.
-constexpr int SR_CL = 8;                // CTAs per query row (cluster size)
-constexpr int SR_NT = 256;
+// Few query rows (decode): one 1024-thread CTA per (query, unit, sequence),
+// two per SM.  The row's pooled keys are contiguous in memory; they stream
+// through two shared-memory buffers in bulk copies (TMA engine), the next
+// round in flight while the warps score the current one (the lanes split the
+// d_qk dot product of a pooled row).  The scores collect in shared memory;
+// then every warp takes a share into a running top-(k-1) and the 32 warp lists
+// are merged as a tree.
+constexpr int SR_NT = 1024;
 constexpr int SR_NW = SR_NT / 32;
-constexpr int SR_QLD = 256;             // row stride of the per-head query staging
-constexpr int SR_MAXC = 512;            // scores per CTA: up to SR_CL * 512 past blocks
-constexpr int SR_RB = 16;               // pooled rows per load round of a warp
+constexpr int SR_MAXC = 2048;           // past blocks per row held in shared memory
+constexpr int SR_KBYTES = 40 * 1024;    // one pooled-key buffer (two of them)
+constexpr int SR_QBYTES = 16 * 256 * 2; // the unit's query rows (<= 16 heads, d <= 256)
+constexpr int SR_SMEM = 2 * SR_KBYTES + SR_QBYTES + 256 * 4 + SR_MAXC * 4 + 64;
 
-__global__ void __cluster_dims__(SR_CL, 1, 1) __launch_bounds__(SR_NT, 2)
+__global__ void __launch_bounds__(SR_NT, 2)
     select_rows_kernel(Shape s, const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
                        int32_t* __restrict__ idx) {
-    __shared__ float qs[256];
-    __shared__ float qh[16 * SR_QLD];                 // per-head query rows (<= 16 heads)
-    __shared__ float sc[SR_MAXC];                     // this CTA's scores
-    __shared__ unsigned long long lists[SR_NW][32];
-    cg::cluster_group cluster = cg::this_cluster();
-    const int crank = (int)cluster.block_rank();
-    const int i = blockIdx.x / SR_CL, u = blockIdx.y, b = blockIdx.z;
+    extern __shared__ __align__(128) uint8_t sr_smem[];
+    float* kbuf = reinterpret_cast<float*>(sr_smem);                                  // 2 x [rows][d]
+    __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(sr_smem + 2 * SR_KBYTES);  // [heads][d]
+    float* qs = reinterpret_cast<float*>(sr_smem + 2 * SR_KBYTES + SR_QBYTES);       // [d]
+    float* sc = qs + 256;                                                             // [SR_MAXC]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sc + SR_MAXC);                        // [2]
+    // the warp lists reuse the key buffers once every round is scored
+    unsigned long long* lists = reinterpret_cast<unsigned long long*>(sr_smem);
+    const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int d = s.dqk;
     const int kvh = s.per_head ? u / s.G : u;
@@ -310,103 +311,87 @@ __global__ void __cluster_dims__(SR_CL, 1, 1) __launch_bounds__(SR_NT, 2)
     const int cr = t / s.bs;
     const int ncand = min(cr, s.nb_full);
     const int K1 = s.topk - 1;
-    // summed query: 16-byte loads of (head, 8 columns), all issued before any is
-    // used (one memory round trip), staged per head and summed in head order
-    {
-        const int nvec = d / 8, np = s.heads_per_unit * nvec;
-        const uint4* src = reinterpret_cast<const uint4*>(q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d);
-        for (int p0 = 0; p0 < np; p0 += 4 * SR_NT) {
-            uint4 raw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                if (p0 + tid + e * SR_NT < np) raw[e] = src[p0 + tid + e * SR_NT];   // head h at h * nvec
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int p = p0 + tid + e * SR_NT;
-                if (p < np) unpack8(raw[e], qh + (p / nvec) * SR_QLD + (p % nvec) * 8);
-            }
-        }
-        __syncthreads();
-        for (int c = tid; c < d; c += SR_NT) {
-            float acc = 0.f;
-            for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += qh[hh * SR_QLD + c];
-            qs[c] = acc;
-        }
+    const int rows_round = SR_KBYTES / (d * 4);
+    const int nrounds = max(1, (ncand + rows_round - 1) / rows_round);
+    const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * d;
+    const __nv_bfloat16* qrow = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d;
+    const uint32_t qbytes = (uint32_t)s.heads_per_unit * d * 2;
+    auto issue = [&](int r) {                // thread 0: round r into buffer r & 1
+        const int nr = max(0, min(rows_round, ncand - r * rows_round));
+        const uint32_t kbytes = (uint32_t)nr * d * 4;
+        tc::mbar_arrive_expect_tx(bar + (r & 1), kbytes + (r == 0 ? qbytes : 0u));
+        if (r == 0) tc::bulk_load(qraw, qrow, qbytes, bar);
+        if (nr > 0)
+            tc::bulk_load(kbuf + (size_t)(r & 1) * (SR_KBYTES / 4), kb + (size_t)r * rows_round * d, kbytes,
+                          bar + (r & 1));
+    };
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(bar + 1, 1);
+        tc::fence_mbar_init();
+        issue(0);
+        if (nrounds > 1) issue(1);
     }
     __syncthreads();
-    // this CTA's share of the past blocks, scored into sc[]
-    const int per_cta = (ncand + SR_CL - 1) / SR_CL;
-    const int c0 = crank * per_cta, n_cta = max(0, min(ncand, c0 + per_cta) - c0);
-    const float* kb = kbar + ((size_t)(b * s.Hkv + kvh) * s.nb_full + c0) * d;
-    const int ncc = (d + 31) / 32;                    // 2..8 columns per lane
-    for (int r0 = warp * SR_RB; r0 < n_cta; r0 += SR_NW * SR_RB) {
-        // every load of the round first, then the dot products
-        float v[SR_RB][6];
-#pragma unroll
-        for (int e = 0; e < SR_RB; ++e) {
-            const float* row = kb + (size_t)min(r0 + e, n_cta - 1) * d;
-#pragma unroll
-            for (int cc = 0; cc < 6; ++cc) v[e][cc] = cc < ncc ? __ldg(row + lane + 32 * cc) : 0.f;
-        }
-        float part[SR_RB];
-#pragma unroll
-        for (int e = 0; e < SR_RB; ++e) {
-            part[e] = 0.f;
-#pragma unroll
-            for (int cc = 0; cc < 6; ++cc)
-                if (cc < ncc) part[e] = fmaf(qs[lane + 32 * cc], v[e][cc], part[e]);
-        }
-        // d = 256: the last two columns of each lane
-        if (ncc > 6) {
-#pragma unroll
-            for (int e = 0; e < SR_RB; ++e) {
-                const float* row = kb + (size_t)min(r0 + e, n_cta - 1) * d;
-                part[e] = fmaf(qs[lane + 192], __ldg(row + lane + 192), part[e]);
-                part[e] = fmaf(qs[lane + 224], __ldg(row + lane + 224), part[e]);
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < SR_RB; ++e) {
-            const float tot = warp_sum(part[e]);
-            if (lane == 0 && r0 + e < n_cta) sc[r0 + e] = s.scale * tot;
-        }
-    }
-    cluster.sync();
-    if (crank == 0) {
-        // warp w: top-(k-1) of CTA w's scores
-        unsigned long long key = 0ull, thr = 0ull;
-        const int w0 = warp * per_cta, nw = max(0, min(ncand, w0 + per_cta) - w0);
-        const float* rsc = cluster.map_shared_rank(sc, warp);
-        if (K1 > 0)
-            for (int e0 = 0; e0 < nw; e0 += 32) {
-                const int e = e0 + lane;
-                const unsigned long long ck = e < nw ? score_key(rsc[e], w0 + e) : 0ull;
-                warp_list_merge(key, thr, ck, K1, lane);
-            }
-        lists[warp][lane] = key;
-        __syncthreads();
-        // tree merge of the warp lists: 8 -> 4 -> 2 -> 1
-        for (int step = 1; step < SR_NW; step <<= 1) {
-            if ((warp & (2 * step - 1)) == 0 && K1 > 0) {
-                warp_list_merge(key, thr, lists[warp + step][lane], K1, lane);
-                lists[warp][lane] = key;
+    bool ok = true;
+    volatile int no_abort = 0;
+    for (int r = 0; r < nrounds; ++r) {
+        ok = tc::mbar_wait(bar + (r & 1), (r >> 1) & 1, &no_abort, 1000000000ull) && ok;
+        if (r == 0) {
+            // summed query, heads added in order
+            for (int c = tid; c < d; c += SR_NT) {
+                float acc = 0.f;
+                for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += bf2f(qraw[hh * d + c]);
+                qs[c] = acc;
             }
             __syncthreads();
         }
-        if (warp == 0) {
-            const bool have = lane < K1 && key != 0ull;
-            const int blk = have ? key_block(key) : 0x7fffffff;
-            const int npast = __popc(__ballot_sync(0xffffffffu, have));
-            int rank = 0;
-            for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, blk, o) < blk) ? 1 : 0;
-            int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
-            if (have) dst[rank] = blk;
-            if (lane == 0) dst[npast] = cr;
-            if (lane > npast && lane < s.topk) dst[lane] = -1;
+        const float* buf = kbuf + (size_t)(r & 1) * (SR_KBYTES / 4);
+        const int nr = max(0, min(rows_round, ncand - r * rows_round));
+        for (int rr = warp; rr < nr; rr += SR_NW) {
+            const float* row = buf + (size_t)rr * d;
+            float part = 0.f;
+            for (int c = lane; c < d; c += 32) part = fmaf(qs[c], row[c], part);
+            part = warp_sum(part);
+            if (lane == 0) sc[r * rows_round + rr] = s.scale * part;
+        }
+        __syncthreads();                      // buffer r & 1 consumed
+        if (tid == 0 && r + 2 < nrounds) issue(r + 2);
+    }
+    // a copy that never landed only records an error (the row's ids are then invalid)
+    if (!ok) atomicExch(&g_select_status, (int)NSA_ERR_TIMEOUT);
+    // every warp: top-(k-1) of its share of the scores
+    unsigned long long key = 0ull, thr = 0ull;
+    if (K1 > 0) {
+        const int per = (ncand + SR_NW - 1) / SR_NW;
+        const int w0 = warp * per, nw = max(0, min(ncand, w0 + per) - w0);
+        for (int e0 = 0; e0 < nw; e0 += 32) {
+            const int e = e0 + lane;
+            const unsigned long long ck = e < nw ? score_key(sc[w0 + e], w0 + e) : 0ull;
+            warp_list_merge(key, thr, ck, K1, lane);
         }
     }
-    // every CTA's scores stay in place until CTA 0 has read them
-    cluster.sync();
+    lists[warp * 32 + lane] = key;
+    __syncthreads();
+    // tree merge of the warp lists: 32 -> 16 -> ... -> 1
+    for (int step = 1; step < SR_NW; step <<= 1) {
+        if ((warp & (2 * step - 1)) == 0 && K1 > 0) {
+            warp_list_merge(key, thr, lists[(warp + step) * 32 + lane], K1, lane);
+            lists[warp * 32 + lane] = key;
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+        const bool have = lane < K1 && key != 0ull;
+        const int blk = have ? key_block(key) : 0x7fffffff;
+        const int npast = __popc(__ballot_sync(0xffffffffu, have));
+        int rank = 0;
+        for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, blk, o) < blk) ? 1 : 0;
+        int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
+        if (have) dst[rank] = blk;
+        if (lane == 0) dst[npast] = cr;
+        if (lane > npast && lane < s.topk) dst[lane] = -1;
+    }
 }
 
 cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
@@ -427,9 +412,10 @@ cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const floa
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         score_topk_kernel<MODE_SELECT_FROM_SCORES><<<grid, ST_NT, smem, st>>>(
             s, nullptr, nullptr, scores_in, nullptr, idx);
-    } else if (s.Tq <= 16 && s.heads_per_unit <= 16 && s.nb_full <= SR_CL * SR_MAXC) {
+    } else if (s.Tq <= 16 && s.heads_per_unit <= 16 && s.nb_full <= SR_MAXC && s.dqk <= 256) {
         // few query rows: a 64-row score tile would be mostly empty
-        select_rows_kernel<<<dim3(s.Tq * SR_CL, s.Hsel, s.B), SR_NT, 0, st>>>(s, q, kbar, idx);
+        cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SR_SMEM);
+        select_rows_kernel<<<dim3(s.Tq, s.Hsel, s.B), SR_NT, SR_SMEM, st>>>(s, q, kbar, idx);
     } else {
         cudaFuncSetAttribute(score_topk_kernel<MODE_SELECT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -437,6 +423,13 @@ cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const floa
                                                                   idx);
     }
     return cudaGetLastError();
+}
+
+int read_and_clear_select_status() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_select_status, sizeof(int)) != cudaSuccess) return -1;
+    cudaMemcpyToSymbol(g_select_status, &zero, sizeof(int));
+    return v;
 }
 
 }  // namespace nsa
