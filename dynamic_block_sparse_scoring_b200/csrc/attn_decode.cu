@@ -109,9 +109,12 @@ struct Item {
     int win_lo;         // window: first key
     int nseg;           // selected: 64-key segments of the kept blocks
     const int32_t* irow;
+    int blk_lane;       // warp form: lane e holds kept block e (selected items)
 };
 
-__device__ __forceinline__ Item item_info(const DecArgs& a, int item) {
+// `warp_form`: called by a whole warp, which reads the query's kept blocks
+// once (one coalesced load, lane e = block e) instead of one load per use.
+__device__ __forceinline__ Item item_info(const DecArgs& a, int item, bool warp_form = false) {
     const Shape& s = a.s;
     Item it;
     const int unit = item / a.ni_all;
@@ -127,6 +130,7 @@ __device__ __forceinline__ Item item_info(const DecArgs& a, int item) {
     it.win_lo = 0;
     it.nseg = 0;
     it.irow = nullptr;
+    it.blk_lane = -1;
     int ntiles = 0;
     if (it.br == B_CMP) {
         it.n_vis = it.t >= s.lc - 1 ? min((it.t - s.lc + 1) / s.sc + 1, s.n_cmp) : 0;
@@ -134,7 +138,13 @@ __device__ __forceinline__ Item item_info(const DecArgs& a, int item) {
     } else if (it.br == B_SEL) {
         it.irow = a.idx + (((size_t)it.b * s.Hsel + it.u) * s.Tq + it.i) * s.topk;
         int nv = 0;
-        for (int e = 0; e < s.topk; ++e) nv += it.irow[e] >= 0 ? 1 : 0;
+        if (warp_form) {
+            const int lane = threadIdx.x & 31;
+            it.blk_lane = lane < s.topk ? it.irow[lane] : -1;
+            nv = __popc(__ballot_sync(0xffffffffu, it.blk_lane >= 0));
+        } else {
+            for (int e = 0; e < s.topk; ++e) nv += it.irow[e] >= 0 ? 1 : 0;
+        }
         it.nseg = nv * a.spb;
         ntiles = (it.nseg + 1) / 2;
     } else {
@@ -146,9 +156,10 @@ __device__ __forceinline__ Item item_info(const DecArgs& a, int item) {
     return it;
 }
 
-// First key of 64-key segment e of a selected item (kept blocks ascending, -1 padded last).
+// First key of 64-key segment e of a selected item (kept blocks ascending, -1
+// padded last), from the warp-form block list; every lane of the warp calls it.
 __device__ __forceinline__ int seg_start(const DecArgs& a, const Item& it, int e) {
-    const int blk = it.irow[e / a.spb];
+    const int blk = __shfl_sync(0xffffffffu, it.blk_lane, (e / a.spb) & 31);
     return blk * a.s.bs + (e % a.spb) * 64;
 }
 
@@ -254,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             return true;
         };
         for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
-            const Item it = item_info(a, item);
+            const Item it = item_info(a, item, true);
             if (it.t0 >= it.t1) continue;
             const int plane = it.b * s.Hkv + it.u;   // group-shared selection: unit = KV head
             const int qb = qcount & 1;
@@ -275,7 +286,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // so that a stage never holds stale or uninitialised rows
                     const int e1 = 2 * j + 1;
                     cur.row0 = seg_start(a, it, 2 * j);
-                    cur.row1 = e1 < it.nseg ? seg_start(a, it, e1) : cur.row0;
+                    const int s1 = seg_start(a, it, e1);
+                    cur.row1 = e1 < it.nseg ? s1 : cur.row0;
                 } else {
                     cur.row0 = cur.cmp ? j * DT : it.win_lo + j * DT;
                 }
@@ -415,7 +427,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool ok = true, ok_prev = true;
         uint32_t tcount = 0, ocount = 0;
         for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
-            const Item it = item_info(a, item);
+            const Item it = item_info(a, item, true);
             float* po = a.part_o + (size_t)item * NH * DV;
             float* pl = a.part_lse + (size_t)item * NH;
             if (it.t0 >= it.t1) {
@@ -438,7 +450,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     valid = j * DT + r < it.n_vis;
                 } else if (it.br == B_SEL) {
                     const int e = 2 * j + (r >> 6);
-                    valid = e < it.nseg && seg_start(a, it, e) + (r & 63) <= it.t;
+                    const int st0 = seg_start(a, it, e);
+                    valid = e < it.nseg && st0 + (r & 63) <= it.t;
                 } else {
                     valid = it.win_lo + j * DT + r <= it.t;
                 }

@@ -287,19 +287,20 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
 constexpr int SR_NT = 1024;
 constexpr int SR_NW = SR_NT / 32;
 constexpr int SR_MAXC = 2048;           // past blocks per row held in shared memory
-constexpr int SR_KBYTES = 40 * 1024;    // one pooled-key buffer (two of them)
+constexpr int SR_NBUF = 2;              // pooled-key buffers (rounds in flight)
+constexpr int SR_KBYTES = 80 * 1024 / SR_NBUF;   // one pooled-key buffer
 constexpr int SR_QBYTES = 16 * 256 * 2; // the unit's query rows (<= 16 heads, d <= 256)
-constexpr int SR_SMEM = 2 * SR_KBYTES + SR_QBYTES + 256 * 4 + SR_MAXC * 4 + 64;
+constexpr int SR_SMEM = SR_NBUF * SR_KBYTES + SR_QBYTES + 256 * 4 + SR_MAXC * 4 + 8 * SR_NBUF;
 
 __global__ void __launch_bounds__(SR_NT, 2)
     select_rows_kernel(Shape s, const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
                        int32_t* __restrict__ idx) {
     extern __shared__ __align__(128) uint8_t sr_smem[];
-    float* kbuf = reinterpret_cast<float*>(sr_smem);                                  // 2 x [rows][d]
-    __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(sr_smem + 2 * SR_KBYTES);  // [heads][d]
-    float* qs = reinterpret_cast<float*>(sr_smem + 2 * SR_KBYTES + SR_QBYTES);       // [d]
+    float* kbuf = reinterpret_cast<float*>(sr_smem);                                  // NBUF x [rows][d]
+    __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(sr_smem + SR_NBUF * SR_KBYTES);  // [heads][d]
+    float* qs = reinterpret_cast<float*>(sr_smem + SR_NBUF * SR_KBYTES + SR_QBYTES);       // [d]
     float* sc = qs + 256;                                                             // [SR_MAXC]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sc + SR_MAXC);                        // [2]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sc + SR_MAXC);                        // [NBUF]
     // the warp lists reuse the key buffers once every round is scored
     unsigned long long* lists = reinterpret_cast<unsigned long long*>(sr_smem);
     const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
@@ -316,27 +317,25 @@ __global__ void __launch_bounds__(SR_NT, 2)
     const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * d;
     const __nv_bfloat16* qrow = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d;
     const uint32_t qbytes = (uint32_t)s.heads_per_unit * d * 2;
-    auto issue = [&](int r) {                // thread 0: round r into buffer r & 1
+    auto issue = [&](int r) {                // thread 0: round r into buffer r % NBUF
         const int nr = max(0, min(rows_round, ncand - r * rows_round));
         const uint32_t kbytes = (uint32_t)nr * d * 4;
-        tc::mbar_arrive_expect_tx(bar + (r & 1), kbytes + (r == 0 ? qbytes : 0u));
+        const int bi = r % SR_NBUF;
+        tc::mbar_arrive_expect_tx(bar + bi, kbytes + (r == 0 ? qbytes : 0u));
         if (r == 0) tc::bulk_load(qraw, qrow, qbytes, bar);
         if (nr > 0)
-            tc::bulk_load(kbuf + (size_t)(r & 1) * (SR_KBYTES / 4), kb + (size_t)r * rows_round * d, kbytes,
-                          bar + (r & 1));
+            tc::bulk_load(kbuf + (size_t)bi * (SR_KBYTES / 4), kb + (size_t)r * rows_round * d, kbytes, bar + bi);
     };
     if (tid == 0) {
-        tc::mbar_init(bar, 1);
-        tc::mbar_init(bar + 1, 1);
+        for (int k = 0; k < SR_NBUF; ++k) tc::mbar_init(bar + k, 1);
         tc::fence_mbar_init();
-        issue(0);
-        if (nrounds > 1) issue(1);
+        for (int k = 0; k < SR_NBUF && k < nrounds; ++k) issue(k);
     }
     __syncthreads();
     bool ok = true;
     volatile int no_abort = 0;
     for (int r = 0; r < nrounds; ++r) {
-        ok = tc::mbar_wait(bar + (r & 1), (r >> 1) & 1, &no_abort, 1000000000ull) && ok;
+        ok = tc::mbar_wait(bar + r % SR_NBUF, (r / SR_NBUF) & 1, &no_abort, 1000000000ull) && ok;
         if (r == 0) {
             // summed query, heads added in order
             for (int c = tid; c < d; c += SR_NT) {
@@ -346,7 +345,7 @@ __global__ void __launch_bounds__(SR_NT, 2)
             }
             __syncthreads();
         }
-        const float* buf = kbuf + (size_t)(r & 1) * (SR_KBYTES / 4);
+        const float* buf = kbuf + (size_t)(r % SR_NBUF) * (SR_KBYTES / 4);
         const int nr = max(0, min(rows_round, ncand - r * rows_round));
         for (int rr = warp; rr < nr; rr += SR_NW) {
             const float* row = buf + (size_t)rr * d;
@@ -355,8 +354,8 @@ __global__ void __launch_bounds__(SR_NT, 2)
             part = warp_sum(part);
             if (lane == 0) sc[r * rows_round + rr] = s.scale * part;
         }
-        __syncthreads();                      // buffer r & 1 consumed
-        if (tid == 0 && r + 2 < nrounds) issue(r + 2);
+        __syncthreads();                      // buffer r % NBUF consumed
+        if (tid == 0 && r + SR_NBUF < nrounds) issue(r + SR_NBUF);
     }
     // a copy that never landed only records an error (the row's ids are then invalid)
     if (!ok) atomicExch(&g_select_status, (int)NSA_ERR_TIMEOUT);
