@@ -66,6 +66,10 @@ EDGE = {
                                                   q_pos0=2999, sel_block=128, top_k=8),
     "dec_sel_only": WORKLOADS["decode64x64k"].with_(name="dec_sel_only", batch=2, seqlen_kv=1500,
                                                      q_pos0=1499, branches=BR_SEL, gated=False),
+    # more work items per (sequence, group) than the in-kernel merge stages: separate merge
+    "dec_long_cache": WORKLOADS["decode64x64k"].with_(name="dec_long_cache", batch=1,
+                                                       seqlen_kv=110000, q_pos0=109999, h_q=32,
+                                                       h_kv=2),
     # block-major selected branch (groups of 8 and 16 heads, sel_block 64, >= 256 queries)
     "bm_g8_ragged": WORKLOADS["nsa64k"].with_(name="bm_g8_ragged", seqlen_q=1000, seqlen_kv=1000,
                                               h_q=16, h_kv=2, d_qk=128, d_v=128),
