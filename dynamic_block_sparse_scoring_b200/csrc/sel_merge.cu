@@ -17,43 +17,45 @@ namespace {
 
 constexpr int MG_MAXK = 16;   // slots per query handled here (the block-major path needs top_k <= 16)
 
-__global__ void __launch_bounds__(256) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
+__global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
                                                         const __nv_bfloat16* __restrict__ part_o,
                                                         const float* __restrict__ part_lse,
                                                         __nv_bfloat16* __restrict__ o_sel) {
+    // one CTA per query: the query's slot count and its (slot, head) log-sum-exps
+    // are staged once in shared memory (one coalesced read), so that every thread
+    // issues only its 16-byte partial loads
+    __shared__ float lse_s[MG_MAXK * 16];
+    __shared__ int nvalid_s;
     const int hpt = s.heads_per_unit, c8n = s.dv / 8;
-    const int per_tok = hpt * c8n;
-    const int tok_per_cta = blockDim.x / per_tok;
-    const int tl = threadIdx.x / per_tok, rem = threadIdx.x % per_tok;
-    const int h = rem / c8n, c8 = rem % c8n;
-    const int qi = blockIdx.x * tok_per_cta + tl;
-    const int u = blockIdx.y, b = blockIdx.z;
-    if (tl >= tok_per_cta || qi >= s.Tq) return;
+    const int qi = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
+    const int h = threadIdx.x / c8n, c8 = threadIdx.x % c8n;
     const size_t prow0 = ((size_t)(b * s.Hsel + u) * s.Tq + qi) * s.topk;
-    // the kept blocks fill the first slots (ascending, -1 padded)
-    const int32_t* irow = idx + prow0;
-    int nvalid = 0;
-#pragma unroll
-    for (int sl = 0; sl < MG_MAXK; ++sl) nvalid += (sl < s.topk && irow[sl] >= 0) ? 1 : 0;
-    float lse[MG_MAXK];
+    if (threadIdx.x < 32) {
+        // the kept blocks fill the first slots (ascending, -1 padded)
+        const int blk = threadIdx.x < s.topk ? idx[prow0 + threadIdx.x] : -1;
+        const int nv = __popc(__ballot_sync(0xffffffffu, blk >= 0));
+        if (threadIdx.x == 0) nvalid_s = nv;
+    }
+    for (int e = threadIdx.x; e < s.topk * hpt; e += blockDim.x)
+        lse_s[e] = __ldcs(part_lse + prow0 * hpt + e);
+    __syncthreads();
+    if (h >= hpt) return;
+    const int nvalid = nvalid_s;
     uint4 raw[MG_MAXK];
+#pragma unroll
+    for (int sl = 0; sl < MG_MAXK; ++sl)              // every load of the row issued at once
+        if (sl < nvalid)
+            raw[sl] = __ldcs(reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8));
     float m = -INFINITY;
 #pragma unroll
-    for (int sl = 0; sl < MG_MAXK; ++sl) {             // every load of the row issued at once
-        lse[sl] = -INFINITY;
-        if (sl < nvalid) {
-            lse[sl] = __ldcs(part_lse + (prow0 + sl) * hpt + h);
-            raw[sl] = __ldcs(reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8));
-        }
-    }
-#pragma unroll
-    for (int sl = 0; sl < MG_MAXK; ++sl) m = fmaxf(m, lse[sl]);
+    for (int sl = 0; sl < MG_MAXK; ++sl)
+        if (sl < nvalid) m = fmaxf(m, lse_s[sl * hpt + h]);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     float wsum = 0.f;
 #pragma unroll
     for (int sl = 0; sl < MG_MAXK; ++sl) {
         if (sl >= nvalid) break;
-        const float w = exp2f(lse[sl] - m);
+        const float w = exp2f(lse_s[sl * hpt + h] - m);
         wsum += w;
         float f[8];
         unpack8(raw[sl], f);
@@ -72,10 +74,10 @@ __global__ void __launch_bounds__(256) sel_merge_kernel(Shape s, const int32_t* 
 
 cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
                              const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st) {
-    const int per_tok = s.heads_per_unit * (s.dv / 8);
-    const int tok_per_cta = per_tok >= 256 ? 1 : 256 / per_tok;
-    dim3 grid((s.Tq + tok_per_cta - 1) / tok_per_cta, s.Hsel, s.B);
-    sel_merge_kernel<<<grid, tok_per_cta * per_tok, 0, st>>>(s, idx, part_o, part_lse, o_sel);
+    // one CTA per query row: heads x 16-byte columns threads (<= 16 x 16)
+    const int threads = ((s.heads_per_unit * (s.dv / 8) + 31) / 32) * 32;
+    dim3 grid(s.Tq, s.Hsel, s.B);
+    sel_merge_kernel<<<grid, std::max(threads, 32), 0, st>>>(s, idx, part_o, part_lse, o_sel);
     return cudaGetLastError();
 }
 
