@@ -52,6 +52,7 @@ STAGE_KERNELS = {
     "rowwise": ("attn_rowwise_kernel", os.path.join(CSRC, "attn_rowwise.cu")),
     "attn_dec": ("dec_kernel", os.path.join(CSRC, "attn_decode.cu")),
     "dec_merge": ("dec_merge_kernel", os.path.join(CSRC, "attn_decode.cu")),
+    "select": ("score_tc_kernel", os.path.join(CSRC, "score_tc.cu")),
 }
 
 
@@ -213,10 +214,10 @@ class Prefill:
         self.launches_per_step = 0
 
     def attn_launches(self) -> int:
-        """Kernels nsa_sparse_attn_fwd launches with an external idx (the library reports
-        its own plan: block-major adds the index build, its attention kernel and the
-        partial merge; split-K adds the split merge)."""
-        self.path, n = self.abi.nsa_attn_plan(self.cfg, False, self.ws_bytes)
+        """Kernels nsa_sparse_attn_fwd launches with the selection inside (the library
+        reports its own plan: the selection, block-major adds the index build, its
+        attention kernel and the partial merge; split-K and decode add a merge)."""
+        self.path, n = self.abi.nsa_attn_plan(self.cfg, bool(self.wl.branches & 2), self.ws_bytes)
         return n
 
     def step(self, ev=None, pool=True):
@@ -230,18 +231,20 @@ class Prefill:
                 int(self.wl.branches & 1 > 0)
         if ev:
             ev[1].record()
-        if self.wl.branches & 2:
-            a.nsa_topk_select(self.cfg, x["q"], p["kbar"], None, self.idx)
-            n += 1
-        if ev:
             ev[2].record()
+        # selection inside the call (idx NULL): it leaves the selected ids at the start
+        # of the workspace, read back into self.idx after the timed steps
         a.nsa_sparse_attn_fwd(self.cfg, x["q"], x["k"], x["v"], p["kbar"], p["kcmp"], p["vcmp"],
-                              x["gates"], self.idx if self.wl.branches & 2 else None, self.out,
-                              self.ws, self.ws_bytes)
+                              x["gates"], None, self.out, self.ws, self.ws_bytes)
         n += self.attn_launches()
         if ev:
             ev[3].record()
         self.launches_per_step = n
+
+    def selected_ids(self):
+        if self.wl.branches & 2:
+            self.idx.copy_(self.ws[:4 * self.idx.numel()].view(torch.int32).view(self.idx.shape))
+        return self.idx
 
 
 def barrier(world):
@@ -299,6 +302,22 @@ def stage_rooflines(wl: Workload, path: str, stage_ms: dict, idx: torch.Tensor, 
     out = {}
     for name, ms in stage_ms.items():
         if ms <= 0:
+            continue
+        if name == "select":
+            if wl.seqlen_q > 16:         # tensor cores, tf32 (3 products per pair; 1 counted)
+                work = fl["score"] * B
+                peak = pk["bf16_tflops"] * 1.1 / 2.25
+                ach = work / (ms / 1e3) / 1e12
+                out[name] = {"ms": ms, "bound": "tensor", "unit": "TFLOP/s", "work": work,
+                             "achieved": ach, "peak": peak, "frac": ach / peak,
+                             "peak_note": "tf32 = measured bf16 x 1.1/2.25 (nominal ratio)"}
+            else:                        # few rows: streams the pooled keys
+                t = np.arange(wl.seqlen_q) + wl.q_pos0
+                cand = np.minimum(t // wl.sel_block, wl.seqlen_kv // wl.sel_block)
+                work = float(cand.sum()) * wl.d_qk * 4 * B * wl.h_sel / max(1, wl.h_sel // wl.h_kv)
+                ach = work / (ms / 1e3) / 1e9
+                out[name] = {"ms": ms, "bound": "hbm", "unit": "GB/s", "work": work,
+                             "achieved": ach, "peak": pk["hbm_gbs"], "frac": ach / pk["hbm_gbs"]}
             continue
         if name in ("attn_tc", "sel_bm", "rowwise"):
             if name == "sel_bm":
@@ -450,7 +469,7 @@ def run_decode(world: int, steps: int, warmup: int):
     path = pf.path
     ms_stream = float(per[:, 1:].sum(axis=1).mean())
     ms = max_over_ranks(graph_steps(pf, steps, warmup, world), world)
-    nbytes = decode_bytes(wl, pf.idx)
+    nbytes = decode_bytes(wl, pf.selected_ids())
     pk, _ = peaks()
     gbs = nbytes / (ms / 1e3) / 1e9 * world
     del pf
@@ -459,7 +478,7 @@ def run_decode(world: int, steps: int, warmup: int):
             "bytes_per_step": nbytes, "frac": gbs / world / pk["hbm_gbs"],
             "peak_gbs": pk["hbm_gbs"], "path": path, "timing": "CUDA graph replay",
             "ms_per_step_stream": ms_stream,
-            "stage_ms": {"select": float(per[:, 1].mean()), **dec_stages}}
+            "stage_ms": dec_stages}
 
 
 def run_ours(args):
@@ -487,7 +506,7 @@ def run_ours(args):
     tokens = wl.seqlen_q * wl.batch * world / (ms / 1e3)
     pk, src = peaks()
     pf.attn_launches()
-    stages = stage_rooflines(wl, pf.path, stage_ms, pf.idx, pk)
+    stages = stage_rooflines(wl, pf.path, stage_ms, pf.selected_ids(), pk)
     stage_ms_all = {k: max_over_ranks(v["ms"], world) for k, v in stages.items()}
     dom = max(stages, key=lambda k: stages[k]["ms"])
     d = dict(stages[dom])
@@ -534,8 +553,8 @@ def run_ours(args):
                            "parallelism": f"independent sequences x{world}",
                            "l2": "256 MB flush before every step; inputs > L2"},
                 "tokens_per_s": tokens, "algorithmic_flops_per_step": fl_all,
-                "stage_ms": {"pool": float(per[:, 0].mean()), "select": float(per[:, 1].mean()),
-                             "attn": float(per[:, 2].mean())},
+                "stage_ms": {"pool": float(per[:, 0].mean()), "select": stage_ms.get("select", 0.0),
+                             "attn": float(per[:, 2].mean()) - stage_ms.get("select", 0.0)},
                 "roofline": roof, "peaks": src, "cpu_baseline": cpu, "e2e": e2e,
                 "decode": decode, "gpu_launches": launches, "clocks": clk,
                 "wall_s_timed_region": wall}

@@ -114,4 +114,11 @@ cudaError_t launch_dec_merge(const Shape& s, const float* part_o, const float* p
                              const float* gates, __nv_bfloat16* out, cudaStream_t st);
 int read_and_clear_dec_status();
 int read_and_clear_select_status();
+// selection on the tensor cores, 3xTF32 (score_tc.cu)
+bool score_tc_supported(const Shape& s);
+size_t score_tc_q_floats(const Shape& s);   // each of qh, ql
+size_t score_tc_k_floats(const Shape& s);   // each of kh, kl
+cudaError_t launch_score_tc(const Shape& s, const __nv_bfloat16* q, const float* kbar, float* qh, float* ql,
+                            float* kh, float* kl, int32_t* idx, cudaStream_t st);
+int read_and_clear_sctc_status();
 }  // namespace nsa

@@ -88,14 +88,19 @@ bool use_block_major(const Shape& s) {
            s.Tq >= 256;
 }
 
+// Selection inside nsa_sparse_attn_fwd on the tensor cores: prefill-sized
+// problems (the few-row kernel serves <= 16 rows).
+bool use_score_tc(const Shape& s) { return nsa::score_tc_supported(s) && s.Tq > 16; }
+
 // Few query rows per sequence (decode): keys as the MMA M dimension.
 bool use_decode(const Shape& s) { return nsa::attn_dec_supported(s); }
 
 // Workspace regions, each 256-byte aligned, in this order.
 struct WsLayout {
     size_t idx = 0, cnt = 0, off = 0, item_off = 0, cursor = 0, list = 0, items = 0, part_o = 0,
-           part_lse = 0, o_sel = 0, split_o = 0, split_lse = 0, dec_o = 0, dec_lse = 0, total = 0,
-           minimal = 0;
+           part_lse = 0, o_sel = 0, split_o = 0, split_lse = 0, dec_o = 0, dec_lse = 0, sc_qh = 0,
+           sc_ql = 0, sc_kh = 0, sc_kl = 0, total = 0, minimal = 0;
+    bool sc = false;    // the selection inside the call runs on the tensor cores
     int n_split = 1;
 };
 
@@ -109,6 +114,14 @@ WsLayout ws_layout(const Shape& s) {
     };
     if (s.flags & NSA_BR_SEL) w.idx = take(idx_bytes(s));
     w.minimal = at;
+    // split operands of the tensor-core selection (prefill)
+    if (use_score_tc(s)) {
+        w.sc = true;
+        w.sc_qh = take(nsa::score_tc_q_floats(s) * 4);
+        w.sc_ql = take(nsa::score_tc_q_floats(s) * 4);
+        w.sc_kh = take(nsa::score_tc_k_floats(s) * 4);
+        w.sc_kl = take(nsa::score_tc_k_floats(s) * 4);
+    }
     // split-K partials for problems with few work tiles (decode)
     if (use_decode(s)) {
         const size_t items = nsa::attn_dec_items(s);
@@ -232,7 +245,8 @@ Plan make_plan(const Shape& s, bool select_inside, size_t ws_bytes, const WsLayo
         else if (wl.n_split > 1 && ws_bytes >= wl.total) p = {NSA_PATH_SPLIT_K, 2};
         else p = {NSA_PATH_QUERY_MAJOR, 1};
     }
-    if (select_inside) p.kernels += 1;
+    // selection inside the call: the tensor-core selection (split + split + score) or one kernel
+    if (select_inside) p.kernels += (wl.sc && ws_bytes >= wl.total) ? 3 : 1;
     return p;
 }
 
@@ -339,7 +353,13 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
     TimingScope timing(cs);
     if (sel && !idx) {
         g_timing.mark("select", cs);
-        st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
+        if (wl.sc && ws_bytes >= wl.total)
+            st = cuda_status(nsa::launch_score_tc(s, qb, kbar, reinterpret_cast<float*>(ws + wl.sc_qh),
+                                                  reinterpret_cast<float*>(ws + wl.sc_ql),
+                                                  reinterpret_cast<float*>(ws + wl.sc_kh),
+                                                  reinterpret_cast<float*>(ws + wl.sc_kl), sel_idx, cs));
+        else
+            st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
         if (st != NSA_OK) return st;
     }
     const Plan plan = make_plan(s, false, ws ? ws_bytes : 0, wl);
@@ -443,8 +463,9 @@ nsa_status nsa_get_device_status(int32_t* status) {
     const int v2 = nsa::read_and_clear_bm_status();
     const int v3 = nsa::read_and_clear_dec_status();
     const int v4 = nsa::read_and_clear_select_status();
-    if (v1 < 0 || v2 < 0 || v3 < 0 || v4 < 0) return NSA_ERR_CUDA;
-    *status = v1 ? v1 : (v2 ? v2 : (v3 ? v3 : v4));
+    const int v5 = nsa::read_and_clear_sctc_status();
+    if (v1 < 0 || v2 < 0 || v3 < 0 || v4 < 0 || v5 < 0) return NSA_ERR_CUDA;
+    *status = v1 ? v1 : (v2 ? v2 : (v3 ? v3 : (v4 ? v4 : v5)));
     return NSA_OK;
 }
 

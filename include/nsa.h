@@ -154,7 +154,10 @@ nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kb
  * fp32; out is rounded to bf16 once.
  * idx may be NULL, in which case the blocks are selected as nsa_topk_select
  * does (needs q, kbar and at least nsa_workspace_size_min() bytes of
- * workspace); otherwise kbar may be NULL.  A workspace of
+ * workspace; with nsa_workspace_size() bytes and more than 16 query rows the
+ * scores run on the tensor cores, three tf32 products per pair), and the
+ * selected ids are left in the first B*Hsel*Tq*top_k int32 of the workspace,
+ * laid out like idx; otherwise kbar may be NULL.  A workspace of
  * nsa_workspace_size() bytes enables the block-major selected branch (each
  * selected KV block attended once for all the queries that kept it); a
  * smaller one (or NULL with an external idx) computes the same result with

@@ -52,8 +52,15 @@ class GpuRun:
             self.idx = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, wl.top_k, dtype=torch.int32,
                                    device="cuda")
             abi.nsa_topk_select(self.cfg, self.x["q"], self.pooled["kbar"], None, self.idx)
+        # the forward with the selection inside the call; it leaves its selected ids at
+        # the start of the workspace
+        ws = torch.empty(max(abi.nsa_workspace_size(self.cfg), 1), dtype=torch.uint8, device="cuda")
         self.out, _ = abi.forward(self.cfg, self.x["q"], self.x["k"], self.x["v"],
-                                  self.x["gates"], pooled=self.pooled)
+                                  self.x["gates"], pooled=self.pooled, workspace=ws)
+        self.idx_fwd = None
+        if self.idx is not None:
+            n = self.idx.numel()
+            self.idx_fwd = ws[:4 * n].view(torch.int32).view(self.idx.shape).clone()
         torch.cuda.synchronize()
         assert abi.nsa_get_device_status() == 0, "a kernel's bounded wait timed out"
 

@@ -96,9 +96,12 @@ def compare_run(run: GpuRun, rows_per_seq, seqs=None):
             s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
                                wl.per_head_select, nb_all)
             ora_idx, gap = O.select_blocks(s, pos, wl.sel_block, wl.top_k)
+            # the stand-alone selection and the one inside the forward call
             gpu_idx = run.idx[b].index_select(1, rows_t).cpu().numpy()
             check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
-            idx_for_out = gpu_idx
+            fwd_idx = run.idx_fwd[b].index_select(1, rows_t).cpu().numpy()
+            check_idx(fwd_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
+            idx_for_out = fwd_idx
         else:
             idx_for_out = None
         # outputs, with the oracle attending over the blocks the GPU kept
@@ -193,18 +196,18 @@ def test_full_size_prefill_sampled_rows(name):
     extra += [r for r in (8190, 8191, 8192, 8193) if r < T]
     rows = row_sample(T, stride=max(1, T // 384), head=128, extra=extra)
     compare_run(run, rows)
-    # every row of the selection: structural invariants
-    idx = run.idx[0]
-    t = torch.arange(T, device="cuda") + wl.q_pos0
-    c = (t // wl.sel_block).view(1, T, 1)
-    valid = idx >= 0
-    n = valid.sum(-1)
-    assert torch.equal(n, torch.clamp(c.view(1, T) + 1, max=wl.top_k).expand_as(n))
-    assert bool(((idx == c) & valid).any(-1).all())                   # current block kept
-    assert bool((idx < c + 1).all())                                   # causal blocks only
-    srt = torch.where(valid, idx, torch.full_like(idx, 1 << 30))
-    ascending = (srt[..., 1:] > srt[..., :-1]) | ~valid[..., 1:]
-    assert bool(ascending.all())                                       # ascending, no repeats
+    # every row of both selections: structural invariants
+    for idx in (run.idx[0], run.idx_fwd[0]):
+        t = torch.arange(T, device="cuda") + wl.q_pos0
+        c = (t // wl.sel_block).view(1, T, 1)
+        valid = idx >= 0
+        n = valid.sum(-1)
+        assert torch.equal(n, torch.clamp(c.view(1, T) + 1, max=wl.top_k).expand_as(n))
+        assert bool(((idx == c) & valid).any(-1).all())               # current block kept
+        assert bool((idx < c + 1).all())                               # causal blocks only
+        srt = torch.where(valid, idx, torch.full_like(idx, 1 << 30))
+        ascending = (srt[..., 1:] > srt[..., :-1]) | ~valid[..., 1:]
+        assert bool(ascending.all())                                   # ascending, no repeats
 
 
 def test_decode_sampled_sequences():
@@ -233,6 +236,9 @@ def test_minimal_workspace_path_matches_oracle(name):
     check_out(f64(out[0]), ora, f"{name} minimal workspace")
     # the two selected-branch organisations agree with each other as well; each is
     # within the output tolerance of the oracle, so they are within twice it of
-    # each other (a bf16 output of magnitude 2-4 can round one ulp = 0.0156 apart)
-    err = np.abs(f64(out[0]) - f64(run.out[0]))
+    # each other (a bf16 output of magnitude 2-4 can round one ulp = 0.0156 apart).
+    # Rows whose two selections differ (a near-tie resolved differently by the
+    # stand-alone and the in-call selection) are compared with the oracle only.
+    same = (run.idx[0] == run.idx_fwd[0]).all(dim=0).all(dim=-1).cpu().numpy()
+    err = np.abs(f64(out[0]) - f64(run.out[0]))[same]
     assert err.max() <= 2 * OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS
