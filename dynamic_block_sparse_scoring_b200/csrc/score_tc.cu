@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(SNT, 1)
             lb[i] = 0;
         }
         float thr = -INFINITY;
+        float* cand = reinterpret_cast<float*>(sm + 2 * STAGE + 1024);   // [SQ][33]
         bool ok = true;
         for (int nt = 0; nt < n_nt; ++nt) {
             const int sb = nt & 1;
@@ -279,25 +280,35 @@ __global__ void __launch_bounds__(SNT, 1)
                 tc::tmem_ld32(tmem + sb * SN + lane_off + cc * 32, v);
                 tc::tmem_wait_ld();
                 const int blk0 = nt * SN + cc * 32;
+                // candidates above the threshold go to this thread's shared-memory slots
+                // and a bit mask; the list update then runs once per such candidate
+                // (one copy of the insertion code keeps the loop small)
+                uint32_t pass = 0;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float sc = s.scale * __uint_as_float(v[j]);
                     if (blk0 + j < ncand && sc > thr) {
-                        // insert (sc, block) into the descending list
-                        float xs = sc;
-                        int xb = blk0 + j;
-#pragma unroll
-                        for (int i = K1 - 1; i > 0; --i) {
-                            const bool gp = xs > ls[i - 1], gc = xs > ls[i];
-                            ls[i] = gp ? ls[i - 1] : (gc ? xs : ls[i]);
-                            lb[i] = gp ? lb[i - 1] : (gc ? xb : lb[i]);
-                        }
-                        if (xs > ls[0]) {
-                            ls[0] = xs;
-                            lb[0] = xb;
-                        }
-                        thr = ls[K1 - 1];
+                        pass |= 1u << j;
+                        cand[r * 33 + j] = sc;
                     }
+                }
+                while (pass) {
+                    const int j = __ffs(pass) - 1;
+                    pass &= pass - 1;
+                    const float xs = cand[r * 33 + j];
+                    if (!(xs > thr)) continue;
+                    const int xb = blk0 + j;
+#pragma unroll
+                    for (int i = K1 - 1; i > 0; --i) {
+                        const bool gp = xs > ls[i - 1], gc = xs > ls[i];
+                        ls[i] = gp ? ls[i - 1] : (gc ? xs : ls[i]);
+                        lb[i] = gp ? lb[i - 1] : (gc ? xb : lb[i]);
+                    }
+                    if (xs > ls[0]) {
+                        ls[0] = xs;
+                        lb[0] = xb;
+                    }
+                    thr = ls[K1 - 1];
                 }
             }
             tc::fence_before_sync();
@@ -373,7 +384,7 @@ cudaError_t launch_sc_impl(const Shape& s, const float* qh, const float* ql, con
     a.s = s;
     a.idx = idx;
     a.n_tt = (s.Tq + SQ - 1) / SQ;
-    const int smem = 2 * STAGE + 128 + 1024;
+    const int smem = 2 * STAGE + 1024 + SQ * 33 * 4 + 1024;
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D, K1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     score_tc_kernel<D, K1><<<dim3(a.n_tt, s.Hsel, s.B), SNT, smem, st>>>(mqh, mql, mkh, mkl, a);
