@@ -557,6 +557,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 1) tc::tmem_dealloc(tmem, 64);
 }
 
+constexpr int MG_BATCH = 8;         // items of a branch whose loads the merge issues together
+
 // out[b, i, h] = sum over branches of gate * (log-sum-exp merge of the branch's items)
 __global__ void __launch_bounds__(256) dec_merge_kernel(Shape s, DecArgs a, const float* __restrict__ gates,
                                                         __nv_bfloat16* __restrict__ out) {
@@ -578,20 +580,44 @@ __global__ void __launch_bounds__(256) dec_merge_kernel(Shape s, DecArgs a, cons
             if (n == 0) continue;
             const size_t it0 = unit * a.ni_all + k0;
             k0 += n;
-            float m = -INFINITY;
-            for (int k = 0; k < n; ++k) m = fmaxf(m, a.part_lse[(it0 + k) * NH + hl]);
-            if (m == -INFINITY) continue;                // empty branch: o = 0
-            float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f;
-            for (int k = 0; k < n; ++k) {
-                const float w = exp2f(a.part_lse[(it0 + k) * NH + hl] - m);
-                wsum += w;
-                const float4* src = reinterpret_cast<const float4*>(a.part_o + ((it0 + k) * NH + hl) * DV + c8 * 8);
-                const float4 x0 = src[0], x1 = src[1];
-                o[0] = fmaf(w, x0.x, o[0]); o[1] = fmaf(w, x0.y, o[1]);
-                o[2] = fmaf(w, x0.z, o[2]); o[3] = fmaf(w, x0.w, o[3]);
-                o[4] = fmaf(w, x1.x, o[4]); o[5] = fmaf(w, x1.y, o[5]);
-                o[6] = fmaf(w, x1.z, o[6]); o[7] = fmaf(w, x1.w, o[7]);
+            float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f, m = -INFINITY;
+            // up to MG_BATCH items of the branch: every load issued before any is used
+            for (int kb = 0; kb < n; kb += MG_BATCH) {
+                float lse[MG_BATCH];
+                float4 x0[MG_BATCH], x1[MG_BATCH];
+#pragma unroll
+                for (int k = 0; k < MG_BATCH; ++k) {
+                    lse[k] = -INFINITY;
+                    if (kb + k < n) {
+                        lse[k] = a.part_lse[(it0 + kb + k) * NH + hl];
+                        const float4* src =
+                            reinterpret_cast<const float4*>(a.part_o + ((it0 + kb + k) * NH + hl) * DV + c8 * 8);
+                        x0[k] = src[0];
+                        x1[k] = src[1];
+                    }
+                }
+                float mb = m;
+#pragma unroll
+                for (int k = 0; k < MG_BATCH; ++k) mb = fmaxf(mb, lse[k]);
+                if (mb == -INFINITY) continue;          // nothing visible so far
+                // rescale what earlier batches accumulated to the new maximum
+                const float sc = m == -INFINITY ? 0.f : exp2f(m - mb);
+                wsum *= sc;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) o[q] *= sc;
+                m = mb;
+#pragma unroll
+                for (int k = 0; k < MG_BATCH; ++k) {
+                    if (kb + k >= n) break;
+                    const float w = exp2f(lse[k] - m);    // 0 for an empty item (lse = -inf)
+                    wsum += w;
+                    o[0] = fmaf(w, x0[k].x, o[0]); o[1] = fmaf(w, x0[k].y, o[1]);
+                    o[2] = fmaf(w, x0[k].z, o[2]); o[3] = fmaf(w, x0[k].w, o[3]);
+                    o[4] = fmaf(w, x1[k].x, o[4]); o[5] = fmaf(w, x1[k].y, o[5]);
+                    o[6] = fmaf(w, x1[k].z, o[6]); o[7] = fmaf(w, x1[k].w, o[7]);
+                }
             }
+            if (m == -INFINITY) continue;                // empty branch: o = 0
             const float g = gates ? gates[row * 3 + br] : 1.f;
             const float f = g / wsum;
 #pragma unroll
