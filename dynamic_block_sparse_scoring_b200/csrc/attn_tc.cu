@@ -25,10 +25,11 @@
 // gate * O / l into an fp32 accumulator row in TMEM; the row is rounded to
 // bf16 once at the end.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer (one
-// lane) and TMEM owner, warps 2-9 softmax/epilogue (two warpgroups, each
-// thread half a row).  Persistent CTAs, one per
-// SM.  Every wait is bounded; a timeout raises a CTA-wide abort, records
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one
+// lane) and TMEM owner, warps 2-3 idle, warps 4-11 softmax/epilogue (two
+// warpgroups, each thread half a row).  Warpgroup 0 hands registers to the
+// softmax warpgroups (setmaxnreg), whose code would otherwise spill under the
+// per-thread limit of a 384-thread CTA.  Persistent CTAs, one per SM.  Every wait is bounded; a timeout raises a CTA-wide abort, records
 // NSA_ERR_TIMEOUT in g_tc_status, drains in-flight copies and MMAs, frees
 // TMEM and returns.
 #include <cudaTypedefs.h>
@@ -55,7 +56,7 @@ constexpr int CHUNK = 16384;     // one 128-row x 64-column bf16 operand chunk
 constexpr int HALF = 8192;       // one 64-row segment of a chunk
 constexpr uint64_t WAIT_NS = 1000000000ull;   // 1 s per wait
 constexpr int MAX_UNION = 1024;  // (tokens per tile) x top_k entries of the selected branch
-constexpr int NTHREADS = 320;    // producer warp, MMA warp, two softmax warpgroups
+constexpr int NTHREADS = 384;    // warpgroup 0: producer warp, MMA warp (+2 idle); two softmax warpgroups
 
 enum { BR_CMP = 0, BR_SEL = 1, BR_WIN = 2, BR_END = 3 };
 
@@ -473,6 +474,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS0 = tmem, tO = tmem + 256, tAcc = tmem + 384;
 
+    if (warp < 4) {
+        // warpgroup 0 gives registers to the softmax warpgroups: 4 x 32 x 56 + 8 x 32 x 216
+        // = 62464 of the 384 x 168 = 64512 the block was launched with
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         Producer<DQK, DV> p{a, sm, bar, abort_flag, &map_q, &map_k, &map_v, &map_kc, &map_vc};
@@ -559,14 +564,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
         }
         __syncwarp();
+    }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
         // ---------------------------------------------------------- softmax / epilogue
         // Two warpgroups; thread (half, r) owns row r and key columns
         // [64*half, 64*half + 64) of every S tile (= segment `half`), and
         // columns [half*DV/2, (half+1)*DV/2) of O and Acc.  The two halves of a
         // row exchange their partial max (every tile) and partial sum (at
         // branch ends) through shared memory.
-        const int half = (warp - 2) >> 2;
+        const int half = (warp - 4) >> 2;
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
         const int r = quarter * 32 + lane;          // tile row of this thread
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
