@@ -161,9 +161,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile
     return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, abort_flag, WAIT_NS));
 }
 
-// Barrier among the 256 softmax threads only (named barrier 1).
+// Barrier between the two softmax warps that hold the two halves of the same
+// rows (warps w and w + 4 of the softmax warpgroups): named barrier 2 + w % 4.
 __device__ __forceinline__ void named_sync_softmax() {
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync %0, 64;" ::"r"(2 + (int)((threadIdx.x >> 5) & 3)) : "memory");
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
@@ -746,14 +747,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::tmem_st32(tS0 + sb * 128 + lane_off + half * 32, sv);
                 tc::tmem_wait_st();
 
-                // O may be touched only after the previous P V has landed
+                // O may be touched only after the previous P V has landed; the wait is
+                // skipped when this tile neither rescales O nor closes a branch (P V of
+                // tile k is the k-th completion of pv_done, so the parity stays known)
                 if (have_prev) {
-                    if (!warp_wait(bar.pv_done(), npv & 1, abort_flag)) {
-                        ok = false;
-                        break;
+                    const bool touch_o = (new_branch && cur_br >= 0) || __any_sync(0xffffffffu, rescale);
+                    if (touch_o) {
+                        if (!warp_wait(bar.pv_done(), npv & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
                     }
                     ++npv;
-                    tc::fence_after_sync();
                 }
                 if (new_branch && cur_br >= 0) correction(cur_br);
                 if (new_branch) l = 0.f;
