@@ -277,102 +277,124 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
     }
 }
 
-// Few query rows (decode): one 1024-thread CTA per (query, unit, sequence),
-// two per SM.  The row's pooled keys are contiguous in memory; they stream
-// through two shared-memory buffers in bulk copies (TMA engine), the next
-// round in flight while the warps score the current one (the lanes split the
-// d_qk dot product of a pooled row).  The scores collect in shared memory;
-// then every warp takes a share into a running top-(k-1) and the 32 warp lists
-// are merged as a tree.
-constexpr int SR_NT = 1024;
+// Few query rows (decode): one 256-thread CTA per (query, unit, sequence),
+// two per SM.  The row's pooled keys are contiguous in memory.  Every warp
+// streams its own contiguous share of them through a private ring of
+// shared-memory slots with bulk copies (TMA engine) on its own mbarriers, so
+// no warp waits for another while keys arrive; the lanes split the d_qk dot
+// product of a pooled row.  The scores collect in shared memory, every warp
+// folds its share into a running top-(k-1), and the warp lists are merged as
+// a tree.
+// Eight warps with four 3 KB slots each measured faster at decode (64 x 65536
+// tokens, d_qk 192) than 16 warps x 2 slots, 4 warps x 8 slots or 4 warps x
+// 4 slots of 6 KB, all with the same 96 KB ring (53.5 us against 57-60 us).
+constexpr int SR_NT = 256;
 constexpr int SR_NW = SR_NT / 32;
 constexpr int SR_MAXC = 2048;           // past blocks per row held in shared memory
-constexpr int SR_NBUF = 2;              // pooled-key buffers (rounds in flight)
-constexpr int SR_KBYTES = 80 * 1024 / SR_NBUF;   // one pooled-key buffer
-constexpr int SR_QBYTES = 16 * 256 * 2; // the unit's query rows (<= 16 heads, d <= 256)
-constexpr int SR_SMEM = SR_NBUF * SR_KBYTES + SR_QBYTES + 256 * 4 + SR_MAXC * 4 + 8 * SR_NBUF;
+constexpr int SR_NSLOT = 4;             // slots per warp (copies in flight)
+constexpr int SR_SLOT = 3072;           // bytes per slot (4 pooled rows at d_qk = 192)
+constexpr int SR_RING = SR_NW * SR_NSLOT * SR_SLOT;
+constexpr int SR_SMEM = SR_RING + SR_MAXC * 4 + 256 * 4 + SR_NW * SR_NSLOT * 8;
+static_assert(SR_NW * 32 * 8 <= SR_RING, "the warp lists reuse the ring");
+static_assert(SR_SLOT % 1024 == 0, "a slot holds at least one pooled row at every d_qk");
 
+template <int D>
 __global__ void __launch_bounds__(SR_NT, 2)
     select_rows_kernel(Shape s, const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
                        int32_t* __restrict__ idx) {
+    constexpr int RPS = SR_SLOT / (D * 4);       // pooled rows per slot
+    constexpr int NSEG = D / 64;                 // float2 columns per lane
     extern __shared__ __align__(128) uint8_t sr_smem[];
-    float* kbuf = reinterpret_cast<float*>(sr_smem);                                  // NBUF x [rows][d]
-    __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(sr_smem + SR_NBUF * SR_KBYTES);  // [heads][d]
-    float* qs = reinterpret_cast<float*>(sr_smem + SR_NBUF * SR_KBYTES + SR_QBYTES);       // [d]
-    float* sc = qs + 256;                                                             // [SR_MAXC]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sc + SR_MAXC);                        // [NBUF]
-    // the warp lists reuse the key buffers once every round is scored
+    float* sc = reinterpret_cast<float*>(sr_smem + SR_RING);                 // [SR_MAXC]
+    float* qs = sc + SR_MAXC;                                                  // [D]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(qs + 256);                   // [NW][NSLOT]
+    // the warp lists reuse the ring once every warp has scored its share
     unsigned long long* lists = reinterpret_cast<unsigned long long*>(sr_smem);
     const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int d = s.dqk;
     const int kvh = s.per_head ? u / s.G : u;
     const int h0 = s.per_head ? u : u * s.G;
     const int t = s.q0 + i;
     const int cr = t / s.bs;
     const int ncand = min(cr, s.nb_full);
     const int K1 = s.topk - 1;
-    const int rows_round = SR_KBYTES / (d * 4);
-    const int nrounds = max(1, (ncand + rows_round - 1) / rows_round);
-    const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * d;
-    const __nv_bfloat16* qrow = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * d;
-    const uint32_t qbytes = (uint32_t)s.heads_per_unit * d * 2;
-    auto issue = [&](int r) {                // thread 0: round r into buffer r % NBUF
-        const int nr = max(0, min(rows_round, ncand - r * rows_round));
-        const uint32_t kbytes = (uint32_t)nr * d * 4;
-        const int bi = r % SR_NBUF;
-        tc::mbar_arrive_expect_tx(bar + bi, kbytes + (r == 0 ? qbytes : 0u));
-        if (r == 0) tc::bulk_load(qraw, qrow, qbytes, bar);
-        if (nr > 0)
-            tc::bulk_load(kbuf + (size_t)bi * (SR_KBYTES / 4), kb + (size_t)r * rows_round * d, kbytes, bar + bi);
+    const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * D;
+    // this warp's contiguous share of the candidates
+    const int per = (ncand + SR_NW - 1) / SR_NW;
+    const int w0 = min(ncand, warp * per), nw = min(ncand, w0 + per) - w0;
+    const int nchunk = (nw + RPS - 1) / RPS;
+    uint8_t* ring = sr_smem + (size_t)warp * SR_NSLOT * SR_SLOT;
+    uint64_t* wb = bars + warp * SR_NSLOT;
+    auto issue = [&](int c) {               // lane 0: chunk c into slot c % NSLOT
+        const int nr = min(RPS, nw - c * RPS);
+        const uint32_t bytes = (uint32_t)nr * D * 4;
+        uint64_t* bar = wb + c % SR_NSLOT;
+        tc::mbar_arrive_expect_tx(bar, bytes);
+        tc::bulk_load(ring + (c % SR_NSLOT) * SR_SLOT, kb + (size_t)(w0 + c * RPS) * D, bytes, bar);
     };
-    if (tid == 0) {
-        for (int k = 0; k < SR_NBUF; ++k) tc::mbar_init(bar + k, 1);
+    if (lane == 0) {
+        for (int k = 0; k < SR_NSLOT; ++k) tc::mbar_init(wb + k, 1);
         tc::fence_mbar_init();
-        for (int k = 0; k < SR_NBUF && k < nrounds; ++k) issue(k);
+        for (int c = 0; c < SR_NSLOT && c < nchunk; ++c) issue(c);
+    }
+    // summed query, heads added in order (while the first copies are in flight)
+    const __nv_bfloat16* qrow = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * D;
+    for (int c = tid; c < D; c += SR_NT) {
+        float acc = 0.f;
+        for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += bf2f(qrow[hh * D + c]);
+        qs[c] = acc;
     }
     __syncthreads();
+    float2 qv[NSEG];
+#pragma unroll
+    for (int j = 0; j < NSEG; ++j) qv[j] = *reinterpret_cast<const float2*>(qs + 64 * j + 2 * lane);
     bool ok = true;
     volatile int no_abort = 0;
-    for (int r = 0; r < nrounds; ++r) {
-        ok = tc::mbar_wait(bar + r % SR_NBUF, (r / SR_NBUF) & 1, &no_abort, 1000000000ull) && ok;
-        if (r == 0) {
-            // summed query, heads added in order
-            for (int c = tid; c < d; c += SR_NT) {
-                float acc = 0.f;
-                for (int hh = 0; hh < s.heads_per_unit; ++hh) acc += bf2f(qraw[hh * d + c]);
-                qs[c] = acc;
+    for (int c = 0; c < nchunk; ++c) {
+        ok = tc::mbar_wait(wb + c % SR_NSLOT, (c / SR_NSLOT) & 1, &no_abort, 1000000000ull) && ok;
+        const float* buf = reinterpret_cast<const float*>(ring + (c % SR_NSLOT) * SR_SLOT);
+        const int nr = min(RPS, nw - c * RPS);
+        float part[RPS];
+#pragma unroll
+        for (int rr = 0; rr < RPS; ++rr) {
+            part[rr] = 0.f;
+            if (rr < nr) {
+#pragma unroll
+                for (int j = 0; j < NSEG; ++j) {
+                    const float2 kv = *reinterpret_cast<const float2*>(buf + rr * D + 64 * j + 2 * lane);
+                    part[rr] = fmaf(qv[j].x, kv.x, part[rr]);
+                    part[rr] = fmaf(qv[j].y, kv.y, part[rr]);
+                }
             }
-            __syncthreads();
         }
-        const float* buf = kbuf + (size_t)(r % SR_NBUF) * (SR_KBYTES / 4);
-        const int nr = max(0, min(rows_round, ncand - r * rows_round));
-        for (int rr = warp; rr < nr; rr += SR_NW) {
-            const float* row = buf + (size_t)rr * d;
-            float part = 0.f;
-            for (int c = lane; c < d; c += 32) part = fmaf(qs[c], row[c], part);
-            part = warp_sum(part);
-            if (lane == 0) sc[r * rows_round + rr] = s.scale * part;
-        }
-        __syncthreads();                      // buffer r % NBUF consumed
-        if (tid == 0 && r + SR_NBUF < nrounds) issue(r + SR_NBUF);
+        __syncwarp();                        // every lane has read the slot
+        if (lane == 0 && c + SR_NSLOT < nchunk) issue(c + SR_NSLOT);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int rr = 0; rr < RPS; ++rr) part[rr] += __shfl_xor_sync(0xffffffffu, part[rr], off);
+        float mine = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < RPS; ++rr)
+            if (lane == rr) mine = part[rr];
+        if (lane < nr) sc[w0 + c * RPS + lane] = s.scale * mine;
     }
     // a copy that never landed only records an error (the row's ids are then invalid)
     if (!ok) atomicExch(&g_select_status, (int)NSA_ERR_TIMEOUT);
-    // every warp: top-(k-1) of its share of the scores
+    __syncwarp();
+    // the warp's top-(k-1) of its own share
     unsigned long long key = 0ull, thr = 0ull;
     if (K1 > 0) {
-        const int per = (ncand + SR_NW - 1) / SR_NW;
-        const int w0 = warp * per, nw = max(0, min(ncand, w0 + per) - w0);
         for (int e0 = 0; e0 < nw; e0 += 32) {
             const int e = e0 + lane;
             const unsigned long long ck = e < nw ? score_key(sc[w0 + e], w0 + e) : 0ull;
             warp_list_merge(key, thr, ck, K1, lane);
         }
     }
+    __syncthreads();                          // every warp is done with its ring
     lists[warp * 32 + lane] = key;
     __syncthreads();
-    // tree merge of the warp lists: 32 -> 16 -> ... -> 1
+    // tree merge of the warp lists
     for (int step = 1; step < SR_NW; step <<= 1) {
         if ((warp & (2 * step - 1)) == 0 && K1 > 0) {
             warp_list_merge(key, thr, lists[(warp + step) * 32 + lane], K1, lane);
@@ -391,6 +413,13 @@ __global__ void __launch_bounds__(SR_NT, 2)
         if (lane == 0) dst[npast] = cr;
         if (lane > npast && lane < s.topk) dst[lane] = -1;
     }
+}
+
+template <int D>
+void launch_select_rows(const Shape& s, const __nv_bfloat16* q, const float* kbar, int32_t* idx,
+                        cudaStream_t st) {
+    cudaFuncSetAttribute(select_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SR_SMEM);
+    select_rows_kernel<D><<<dim3(s.Tq, s.Hsel, s.B), SR_NT, SR_SMEM, st>>>(s, q, kbar, idx);
 }
 
 cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
@@ -413,8 +442,10 @@ cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const floa
             s, nullptr, nullptr, scores_in, nullptr, idx);
     } else if (s.Tq <= 16 && s.heads_per_unit <= 16 && s.nb_full <= SR_MAXC && s.dqk <= 256) {
         // few query rows: a 64-row score tile would be mostly empty
-        cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SR_SMEM);
-        select_rows_kernel<<<dim3(s.Tq, s.Hsel, s.B), SR_NT, SR_SMEM, st>>>(s, q, kbar, idx);
+        if (s.dqk == 64) launch_select_rows<64>(s, q, kbar, idx, st);
+        else if (s.dqk == 128) launch_select_rows<128>(s, q, kbar, idx, st);
+        else if (s.dqk == 192) launch_select_rows<192>(s, q, kbar, idx, st);
+        else launch_select_rows<256>(s, q, kbar, idx, st);
     } else {
         cudaFuncSetAttribute(score_topk_kernel<MODE_SELECT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
