@@ -156,6 +156,28 @@ __device__ __forceinline__ Item item_info(const DecArgs& a, int item, bool warp_
     return it;
 }
 
+// Item id of this CTA's k-th work item, or -1 past the last.  The items are
+// taken branch by branch (every compressed item, then the selected, then the
+// window ones, each in unit order) and dealt to the CTAs back and forth
+// (0 .. G-1, G-1 .. 0, ...), so that every CTA gets a near-equal number of
+// tiles: the compressed and selected items are the long ones.  The id itself
+// stays unit-major (unit * ni_all + branch offset + sub-range), which is how
+// the partials are laid out for the merge.
+__device__ __forceinline__ int item_at(const DecArgs& a, int k) {
+    const int G = gridDim.x, c = blockIdx.x;
+    const int p = (k >> 1) * 2 * G + ((k & 1) ? 2 * G - 1 - c : c);
+    if (p >= a.n_items) return -1;
+    const int units = a.n_items / a.ni_all;
+    int q = p, off = 0;
+    for (int br = 0; br < 3; ++br) {
+        const int nb = units * a.ni[br];
+        if (q < nb) return (q / a.ni[br]) * a.ni_all + off + q % a.ni[br];
+        q -= nb;
+        off += a.ni[br];
+    }
+    return -1;
+}
+
 // First key of 64-key segment e of a selected item (kept blocks ascending, -1
 // padded last), from the warp-form block list; every lane of the warp calls it.
 __device__ __forceinline__ int seg_start(const DecArgs& a, const Item& it, int e) {
@@ -264,7 +286,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             ++vcount;
             return true;
         };
-        for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+        for (int k = 0, item; ok && (item = item_at(a, k)) >= 0; ++k) {
             const Item it = item_info(a, item, true);
             if (it.t0 >= it.t1) continue;
             const int plane = it.b * s.Hkv + it.u;   // group-shared selection: unit = KV head
@@ -367,7 +389,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::mma_commit(bar.pv_done());
                 return true;
             };
-            for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+            for (int k = 0, item; ok && (item = item_at(a, k)) >= 0; ++k) {
                 const Item it = item_info(a, item);
                 if (it.t0 >= it.t1) continue;
                 const int qb = qcount & 1;
@@ -426,7 +448,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int wq = warp - 2;                      // 0..3, slot in red
         bool ok = true, ok_prev = true;
         uint32_t tcount = 0, ocount = 0;
-        for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+        for (int k = 0, item; ok && (item = item_at(a, k)) >= 0; ++k) {
             const Item it = item_info(a, item, true);
             float* po = a.part_o + (size_t)item * NH * DV;
             float* pl = a.part_lse + (size_t)item * NH;
