@@ -48,6 +48,8 @@ EDGE = {
                                cmp_stride=1),
     # a few queries at the end of a cache (the few-row selection kernel; split-K)
     "few_queries": TINY.with_(name="few_queries", seqlen_q=5, seqlen_kv=900, q_pos0=895),
+    "few_d256": TINY.with_(name="few_d256", seqlen_q=4, seqlen_kv=2000, q_pos0=1996, h_q=4, h_kv=2,
+                           d_qk=256, d_v=256),
     "decode_small": WORKLOADS["decode64x64k"].with_(name="decode_small", batch=3, seqlen_kv=3000,
                                                      q_pos0=2999),
     # few-query kernel (keys as the MMA M dimension): groups of 8 and 16 heads, up to 4 queries,
