@@ -252,12 +252,25 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The largest of every rank's `v` (the slowest rank's time).  Every rank must
+    call it the same number of times in the same order."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput (units per second): every rank processes the same
+    number of units (weak scaling), and the job takes as long as its slowest rank."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
+def rank_seed(rank: int, decode: bool = False) -> int:
+    """Each rank draws its own independent problem."""
+    return (1000 if decode else 0) + rank
 
 
 def timed_steps(pf: Prefill, steps: int, warmup: int, world: int, pool=True):
@@ -484,7 +497,7 @@ def graph_steps(pf: Prefill, steps: int, warmup: int, world: int) -> float:
 
 def run_decode(world: int, steps: int, warmup: int):
     wl = WORKLOADS["decode64x64k"]
-    pf = Prefill(wl, seed=1000 + (torch.distributed.get_rank() if world > 1 else 0))
+    pf = Prefill(wl, seed=rank_seed(torch.distributed.get_rank() if world > 1 else 0, decode=True))
     pf.step()                        # pooled cache built once (cache maintenance, not timed)
     torch.cuda.synchronize()
     per, _, dec_stages = timed_steps(pf, steps, warmup, world, pool=False)
@@ -494,7 +507,7 @@ def run_decode(world: int, steps: int, warmup: int):
     ms = max_over_ranks(graph_steps(pf, steps, warmup, world), world)
     nbytes = decode_bytes(wl, pf.selected_ids())
     pk, _ = peaks()
-    gbs = nbytes / (ms / 1e3) / 1e9 * world
+    gbs = job_rate(nbytes, world, ms) / 1e9
     del pf
     torch.cuda.empty_cache()
     return {"workload": wl.name, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
@@ -515,7 +528,7 @@ def run_ours(args):
         wl = wl.with_(seqlen_q=args.seqlen, seqlen_kv=args.seqlen)
     if args.batch:
         wl = wl.with_(batch=args.batch)
-    pf = Prefill(wl, seed=rank)
+    pf = Prefill(wl, seed=rank_seed(rank))
     clocks = ClockSampler(torch.cuda.current_device())
     # warm-up and timed region (clocks sampled during it)
     clocks.start()
@@ -525,8 +538,8 @@ def run_ours(args):
     ms = max_over_ranks(float(step_ms.mean()), world)
     fl = algorithmic_flops(wl)
     fl_all = fl["total"] * wl.batch * world
-    value = fl_all / (ms / 1e3) / 1e12
-    tokens = wl.seqlen_q * wl.batch * world / (ms / 1e3)
+    value = job_rate(fl["total"] * wl.batch, world, ms) / 1e12
+    tokens = job_rate(wl.seqlen_q * wl.batch, world, ms)
     pk, src = peaks()
     pf.attn_launches()
     stages = stage_rooflines(wl, pf.path, stage_ms, pf.selected_ids(), pk)
@@ -551,7 +564,8 @@ def run_ours(args):
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_steps(pf, max(4, args.steps), 2, world)
         e2e_ms = max_over_ranks(e2e_ms, world)
-        e2e = {"value": fl_all / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": job_rate(fl["total"] * wl.batch, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     x_cpu = None
     if rank == 0 and not args.no_cpu_baseline:
