@@ -48,6 +48,7 @@ STAGE_KERNELS = {
     "sel_bm": ("sel_bm_kernel", os.path.join(CSRC, "attn_sel_bm.cu")),
     "sel_merge": ("sel_merge_kernel", os.path.join(CSRC, "sel_merge.cu")),
     "index": ("sel_index", os.path.join(CSRC, "sel_index.cu")),
+    "expand": ("expand_kernel", os.path.join(CSRC, "sel_index.cu")),
     "split_merge": ("split_merge_kernel", os.path.join(CSRC, "attn_tc.cu")),
     "rowwise": ("attn_rowwise_kernel", os.path.join(CSRC, "attn_rowwise.cu")),
     "attn_dec": ("dec_kernel", os.path.join(CSRC, "attn_decode.cu")),
@@ -312,6 +313,15 @@ def stage_rooflines(wl: Workload, path: str, stage_ms: dict, idx: torch.Tensor, 
     B = wl.batch
     idx_bytes = idx.numel() * 4
     n_valid = int((idx >= 0).sum().item()) if wl.branches & 2 else 0
+    hpt = wl.h_q // wl.h_sel
+    # the selected branch alone with one head per unit runs over 64-key sub-blocks: a kept
+    # block is one partial per sub-block that starts at or before the query
+    spb = wl.sel_block // 64 if (wl.branches == 2 and hpt == 1 and wl.sel_block % 64 == 0) else 1
+    n_parts = n_valid
+    if spb > 1 and n_valid:
+        ic = idx.cpu().numpy()
+        t = (np.arange(wl.seqlen_q) + wl.q_pos0)[None, None, :, None]
+        n_parts = int(np.where(ic >= 0, np.clip((t - ic * wl.sel_block) // 64 + 1, 0, spb), 0).sum())
     out = {}
     for name, ms in stage_ms.items():
         if ms <= 0:
@@ -343,11 +353,12 @@ def stage_rooflines(wl: Workload, path: str, stage_ms: dict, idx: torch.Tensor, 
             out[name] = {"ms": ms, "bound": "tensor", "unit": "TFLOP/s", "work": work,
                          "achieved": ach, "peak": pk["bf16_tflops"], "frac": ach / pk["bf16_tflops"]}
         else:
-            hpt = wl.h_q // wl.h_sel
             if name == "sel_merge":      # read every valid partial (o bf16 + lse), write o_sel
-                work = n_valid * hpt * (2 * wl.d_v + 4) + B * wl.seqlen_q * wl.h_q * wl.d_v * 2 + idx_bytes
+                work = n_parts * hpt * (2 * wl.d_v + 4) + B * wl.seqlen_q * wl.h_q * wl.d_v * 2 + idx_bytes * spb
             elif name == "index":        # read idx twice, write the pair lists
-                work = 2 * idx_bytes + n_valid * 4
+                work = 2 * idx_bytes * spb + n_parts * 4
+            elif name == "expand":       # read the kept blocks, write their sub-blocks
+                work = idx_bytes * (1 + spb)
             else:                        # split merge: fp32 (o, l, m) per split, branch and row
                 work = 0.0
             ach = work / (ms / 1e3) / 1e9

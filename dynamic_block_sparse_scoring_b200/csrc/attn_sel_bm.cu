@@ -49,9 +49,11 @@ constexpr int NM = 8;               // item descriptors in flight
 constexpr int CHUNK_Q = 16384;      // 128 rows x 64 columns bf16
 constexpr int CHUNK_KV = 8192;      // 64 rows x 64 columns bf16
 constexpr uint64_t WAIT_NS = 1000000000ull;
-constexpr int MAX_TOK = 16;
 constexpr int NQ = 2;               // query-gather stages
 
+// MT = most queries in one item: 16 when a unit stacks 8 or 16 heads under each
+// query, 128 when a unit is one head (per-head selection).
+template <int MT>
 struct ItemMeta {
     int valid;          // 0 = end of the stream
     int lidx;           // list id = (chunk * B * Hsel + b * Hsel + u) * nb_all + j
@@ -60,7 +62,7 @@ struct ItemMeta {
     int new_block;      // first item on this K/V stage load
     int last_of_block;  // last item using this K/V stage load
     int pad[2];
-    int tok[MAX_TOK];   // query * 32 + slot
+    int tok[MT];        // query * 32 + slot
 };
 
 struct BmArgs {
@@ -76,7 +78,7 @@ struct BmArgs {
     float scale_log2;
 };
 
-template <int DQK, int DV>
+template <int DQK, int DV, int MT>
 struct BmSmem {
     static constexpr int QC = DQK / 64, VC = DV / 64;
     static constexpr int Q_OFF = 0;                                  // NQ stages
@@ -84,7 +86,7 @@ struct BmSmem {
     static constexpr int V_OFF = K_OFF + 2 * QC * CHUNK_KV;           // 2 stages
     static constexpr int STG_OFF = V_OFF + 2 * VC * CHUNK_KV;        // 2 x [BM rows x 128 B]
     static constexpr int META_OFF = STG_OFF + 2 * BM * 128;
-    static constexpr int ROW_OFF = META_OFF + NM * (int)sizeof(ItemMeta);   // row m, l [2][2][BM]
+    static constexpr int ROW_OFF = META_OFF + NM * (int)sizeof(ItemMeta<MT>);   // row m, l [2][2][BM]
     static constexpr int BAR_OFF = ROW_OFF + 4 * BM * 4;
     // q_full[NQ] q_empty[NQ] kv_full[2] kv_empty[2] meta_full[NM] meta_empty[NM]
     // s_full[2] p_full[2] o_full[2] o_free[2] drain
@@ -118,12 +120,14 @@ __device__ __forceinline__ void bm_abort(volatile int* abort_flag) {
     atomicExch(&g_bm_status, (int)NSA_ERR_TIMEOUT);
 }
 
-template <int DQK, int DV>
+template <int DQK, int DV, int MT>
 __global__ void __launch_bounds__(NTHREADS, 1)
     sel_bm_kernel(const __grid_constant__ CUtensorMap map_qg, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v,
                   const __grid_constant__ CUtensorMap map_po, const BmArgs a) {
-    using L = BmSmem<DQK, DV>;
+    using L = BmSmem<DQK, DV, MT>;
+    using ItemMeta = nsa::ItemMeta<MT>;
+    constexpr int NG = (MT + 31) / 32;      // lane groups covering an item's queries
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -217,6 +221,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         while (ok && ends < 2) {
             while (i >= i_end && chunk + 1 < a.n_chunks) chunk_range(++chunk, i, i_end);
             ItemMeta m;
+            bool meta_ready = false;     // this item's metadata slot already waited for
             m.valid = i < i_end;
             m.lidx = m.n = m.kvs = m.new_block = m.last_of_block = 0;
             if (m.valid) {
@@ -255,22 +260,53 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     prev_lidx = it.x;
                 }
                 m.kvs = kvs;
-                const int tokv = list_at(it.y, m.n);
-                for (int tt = 0; tt < MAX_TOK; ++tt) m.tok[tt] = __shfl_sync(0xffffffffu, tokv, tt);
-                const int qs = li % NQ;
-                if (!bm_warp_wait(bar.q_empty(qs), ((li / NQ) & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
-                __syncwarp();
-                // one TMA per (query, 64-column chunk), spread over the lanes; the
-                // query rows are reused by the chunk's other blocks, so keep them in L2
-                for (int e = lane; e < m.n * L::QC; e += 32) {
-                    const int tt = e / L::QC, c = e % L::QC;
-                    tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
-                                         &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b,
-                                         q_policy);
+                if constexpr (MT <= 32) {
+                    const int tokv = list_at(it.y, m.n);
+                    for (int tt = 0; tt < MT; ++tt) m.tok[tt] = __shfl_sync(0xffffffffu, tokv, tt);
+                    const int qs = li % NQ;
+                    if (!bm_warp_wait(bar.q_empty(qs), ((li / NQ) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
+                    __syncwarp();
+                    // one TMA per (query, 64-column chunk), spread over the lanes; the
+                    // query rows are reused by the chunk's other blocks, so keep them in L2
+                    for (int e = lane; e < m.n * L::QC; e += 32) {
+                        const int tt = e / L::QC, c = e % L::QC;
+                        tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
+                                             &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b,
+                                             q_policy);
+                    }
+                } else {
+                    // more queries than lanes: they go straight into the item's
+                    // metadata slot, which the Q loads then read back
+                    const int slot = li % NM;
+                    if (!bm_warp_wait(bar.meta_empty(slot), ((li / NM) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    meta_ready = true;
+                    for (int g = 0; g < NG; ++g) {
+                        const int n_g = min(32, m.n - 32 * g);
+                        if (n_g <= 0) break;
+                        const int tokv = list_at(it.y + 32 * g, n_g);
+                        if (lane < n_g) metas[slot].tok[32 * g + lane] = tokv;
+                    }
+                    __syncwarp();
+                    const int qs = li % NQ;
+                    if (!bm_warp_wait(bar.q_empty(qs), ((li / NQ) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
+                    __syncwarp();
+                    for (int e = lane; e < m.n * L::QC; e += 32) {
+                        const int tt = e / L::QC, c = e % L::QC;
+                        tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
+                                             &map_qg, bar.q_full(qs), 64 * c, h0, metas[slot].tok[tt] >> 5, b,
+                                             q_policy);
+                    }
                 }
                 ++q_loads;
                 ++i;
@@ -278,12 +314,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ++ends;    // two end markers: each softmax warpgroup sees one
             }
             const int slot = li % NM;
-            if (!bm_warp_wait(bar.meta_empty(slot), ((li / NM) & 1) ^ 1, abort_flag)) {
+            if (!meta_ready && !bm_warp_wait(bar.meta_empty(slot), ((li / NM) & 1) ^ 1, abort_flag)) {
                 ok = false;
                 break;
             }
             if (lane == 0) {
-                metas[slot] = m;
+                if constexpr (MT <= 32) {
+                    metas[slot] = m;
+                } else {
+                    ItemMeta& d = metas[slot];
+                    d.valid = m.valid;
+                    d.lidx = m.lidx;
+                    d.n = m.n;
+                    d.kvs = m.kvs;
+                    d.new_block = m.new_block;
+                    d.last_of_block = m.last_of_block;
+                }
                 tc::mbar_arrive(bar.meta_full(slot));
             }
             ++li;
@@ -400,7 +446,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             const ItemMeta& mref = metas[slot];
             const int valid = mref.valid, lidx = mref.lidx, n = mref.n;
-            const int tokr = tt < MAX_TOK ? mref.tok[tt] : 0;
+            const int tokr = tt < MT ? mref.tok[tt] : 0;
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
             if (!valid) break;
@@ -499,14 +545,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int li = 0;; ++li) {
             const int slot = li % NM;
             bool okw = bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag);
-            int valid = 0, lidx = 0, n = 0, tokr = 0, tok_lane = 0;
+            int valid = 0, lidx = 0, n = 0, tokr = 0;
+            int tok_lane[NG];             // the queries whose stores this lane issues
+#pragma unroll
+            for (int g = 0; g < NG; ++g) tok_lane[g] = 0;
             if (okw) {
                 const ItemMeta& mref = metas[slot];
                 valid = mref.valid;
                 lidx = mref.lidx;
                 n = mref.n;
-                tokr = tt < MAX_TOK ? mref.tok[tt] : 0;
-                tok_lane = lane < MAX_TOK ? mref.tok[lane] : 0;
+                tokr = tt < MT ? mref.tok[tt] : 0;
+#pragma unroll
+                for (int g = 0; g < NG; ++g) tok_lane[g] = 32 * g + lane < MT ? mref.tok[32 * g + lane] : 0;
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
             }
@@ -529,8 +579,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int bu = (lidx / nb_all) % bhsel;
             const float m = row_m[sb * BM + r], l = row_l[sb * BM + r];
             const size_t prow = (((size_t)bu * a.s.Tq + (tokr >> 5)) * a.s.topk + (tokr & 31)) * a.hpt + hl;
-            // first partial row of the query this lane stores (issuer warp)
-            const int prow_q = (int)((((size_t)bu * a.s.Tq + (tok_lane >> 5)) * a.s.topk + (tok_lane & 31)) * a.hpt);
+            // first partial row of each query this lane stores (issuer warp)
+            int prow_q[NG];
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+                prow_q[g] = (int)((((size_t)bu * a.s.Tq + (tok_lane[g] >> 5)) * a.s.topk + (tok_lane[g] & 31)) * a.hpt);
 #pragma unroll 1
             for (int c = 0; c < DV; c += 64, ++halves) {
                 uint32_t o[64];
@@ -560,10 +613,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::fence_proxy_async_smem();
                 tc::named_bar_sync(1, 128);
                 if (issuer) {
-                    if (lane < n)
-                        tc::tma_store_2d_hint(&map_po,
-                                              sm + L::STG_OFF + (halves & 1) * (BM * 128) + lane * a.hpt * 128,
-                                              c, prow_q, st_policy);
+#pragma unroll
+                    for (int g = 0; g < NG; ++g)
+                        if (32 * g + lane < n)
+                            tc::tma_store_2d_hint(&map_po,
+                                                  sm + L::STG_OFF + (halves & 1) * (BM * 128) +
+                                                      (32 * g + lane) * a.hpt * 128,
+                                                  c, prow_q[g], st_policy);
                     tc::bulk_commit();
                 }
             }
@@ -602,7 +658,7 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DQK, int DV>
+template <int DQK, int DV, int MT>
 cudaError_t launch_bm_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const SelIndex& x, __nv_bfloat16* part_o,
                            float* part_lse, cudaStream_t st) {
@@ -639,11 +695,12 @@ cudaError_t launch_bm_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bf
     int dev = 0, nsm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    const int smem = BmSmem<DQK, DV>::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(sel_bm_kernel<DQK, DV>,
+    const int smem = BmSmem<DQK, DV, MT>::ALLOC;
+    static_assert(BmSmem<DQK, DV, MT>::ALLOC <= 232448, "shared memory");
+    cudaError_t e = cudaFuncSetAttribute(sel_bm_kernel<DQK, DV, MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    sel_bm_kernel<DQK, DV><<<nsm, NTHREADS, smem, st>>>(mq, mk, mv, mpo, a);
+    sel_bm_kernel<DQK, DV, MT><<<nsm, NTHREADS, smem, st>>>(mq, mk, mv, mpo, a);
     return cudaGetLastError();
 }
 
@@ -655,15 +712,19 @@ bool sel_bm_supported(const Shape& s) {
     if (s.dv != 64 && s.dv != 128) return false;
     if (s.bs != BLK) return false;
     const int hpt = s.heads_per_unit;
+    // a slot is 5 bits of a list entry; the merge of groups takes up to 16 slots
+    const bool shape_ok = ((hpt == 8 || hpt == 16) && s.topk <= 16) || (hpt == 1 && s.topk <= 32);
     // partial rows are addressed by 32-bit TMA coordinates
-    return (hpt == 8 || hpt == 16) && s.topk <= 16 && sel_partial_rows(s) < (size_t(1) << 31);
+    return shape_ok && sel_partial_rows(s) < (size_t(1) << 31);
 }
 
 cudaError_t launch_sel_bm(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                           const __nv_bfloat16* v, const SelIndex& x, __nv_bfloat16* part_o,
                           float* part_lse, cudaStream_t st) {
-#define NSA_BM_CASE(A, B) \
-    if (s.dqk == A && s.dv == B) return launch_bm_impl<A, B>(s, q, k, v, x, part_o, part_lse, st);
+#define NSA_BM_CASE(A, B)                                                              \
+    if (s.dqk == A && s.dv == B)                                                       \
+        return s.heads_per_unit == 1 ? launch_bm_impl<A, B, 128>(s, q, k, v, x, part_o, part_lse, st) \
+                                     : launch_bm_impl<A, B, 16>(s, q, k, v, x, part_o, part_lse, st);
     NSA_BM_CASE(64, 64)
     NSA_BM_CASE(128, 128)
     NSA_BM_CASE(192, 128)

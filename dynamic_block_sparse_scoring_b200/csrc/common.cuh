@@ -96,6 +96,13 @@ cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o
 int read_and_clear_tc_status();
 cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
                              const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st);
+// selected branch alone, one head per unit: out = g_sel * (merge of the row's
+// sub-block partials), written directly (sel_merge.cu); s is the sub-block shape
+cudaError_t launch_sel_merge_out(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
+                                 const float* part_lse, const float* gates, __nv_bfloat16* out,
+                                 cudaStream_t st);
+// kept blocks -> the 64-key sub-blocks at or before the query (sel_index.cu)
+cudaError_t launch_sel_expand(const Shape& s, const int32_t* idx, int32_t* idx_sub, cudaStream_t st);
 // block-major selected branch (attn_sel_bm.cu)
 struct SelIndex;
 bool sel_bm_supported(const Shape& s);

@@ -88,6 +88,27 @@ bool use_block_major(const Shape& s) {
            s.Tq >= 256;
 }
 
+// The selected branch alone with one head per unit (MoBA's per-head
+// selection, blocks of any multiple of 64 keys): every kept block is cut into
+// its 64-key sub-blocks and the block-major kernel runs over those, the merge
+// writing out directly.  This is the problem restated with 64-key blocks and
+// top_k * (sel_block / 64) slots.
+Shape sub_block_shape(const Shape& s) {
+    Shape t = s;
+    t.topk = s.topk * (s.bs / 64);
+    t.bs = 64;
+    t.nb_full = s.Tk / 64;
+    t.nb_all = (s.Tk + 63) / 64;
+    return t;
+}
+
+bool use_sub_block_major(const Shape& s) {
+    if (!(s.flags & NSA_BR_SEL) || (s.flags & (NSA_BR_CMP | NSA_BR_WIN))) return false;
+    if (s.heads_per_unit != 1 || s.bs % 64 != 0 || s.Tq < 256) return false;
+    if (s.topk * (s.bs / 64) > 32) return false;
+    return nsa::sel_bm_supported(sub_block_shape(s));
+}
+
 // Selection inside nsa_sparse_attn_fwd on the tensor cores: prefill-sized
 // problems (the few-row kernel serves <= 16 rows).
 bool use_score_tc(const Shape& s) { return nsa::score_tc_supported(s) && s.Tq > 16; }
@@ -97,10 +118,11 @@ bool use_decode(const Shape& s) { return nsa::attn_dec_supported(s); }
 
 // Workspace regions, each 256-byte aligned, in this order.
 struct WsLayout {
-    size_t idx = 0, cnt = 0, off = 0, item_off = 0, cursor = 0, list = 0, items = 0, part_o = 0,
+    size_t idx = 0, idx_sub = 0, cnt = 0, off = 0, item_off = 0, cursor = 0, list = 0, items = 0, part_o = 0,
            part_lse = 0, o_sel = 0, split_o = 0, split_lse = 0, dec_o = 0, dec_lse = 0, sc_qh = 0,
            sc_ql = 0, sc_kh = 0, sc_kl = 0, total = 0, minimal = 0;
     bool sc = false;    // the selection inside the call runs on the tensor cores
+    bool sub = false;   // block-major over 64-key sub-blocks (selected branch alone)
     int n_split = 1;
 };
 
@@ -147,6 +169,20 @@ WsLayout ws_layout(const Shape& s) {
         w.part_o = take(nsa::sel_pairs_max(s) * s.heads_per_unit * s.dv * 2);
         w.part_lse = take(nsa::sel_pairs_max(s) * s.heads_per_unit * 4);
         w.o_sel = take((size_t)s.B * s.Tq * s.Hq * s.dv * 2);
+    } else if (use_sub_block_major(s)) {
+        const Shape t = sub_block_shape(s);
+        const size_t L = nsa::sel_lists(t);
+        const int tok = 128;                  // one head per unit: 128 queries per item
+        w.sub = true;
+        w.idx_sub = take(idx_bytes(t));
+        w.cnt = take(L * 4);
+        w.off = take((L + 1) * 4);
+        w.item_off = take((L + 1) * 4);
+        w.cursor = take(L * 4);
+        w.list = take(nsa::sel_list_alloc(t) * 4);
+        w.items = take(nsa::sel_items_max(t, tok) * sizeof(int4));
+        w.part_o = take(nsa::sel_pairs_max(t) * t.dv * 2);
+        w.part_lse = take(nsa::sel_pairs_max(t) * 4);
     }
     w.total = at;
     return w;
@@ -240,6 +276,8 @@ Plan make_plan(const Shape& s, bool select_inside, size_t ws_bytes, const WsLayo
     Plan p{NSA_PATH_ROWWISE, 1};
     if (use_decode(s) && ws_bytes >= wl.total) {
         p = {NSA_PATH_DECODE, 2};
+    } else if (use_sub_block_major(s) && ws_bytes >= wl.total) {
+        p = {NSA_PATH_BLOCK_MAJOR, 7};    // expand, index (4), block-major, merge into out
     } else if (nsa::attn_tc_supported(s)) {
         if (use_block_major(s) && ws_bytes >= wl.total) p = {NSA_PATH_BLOCK_MAJOR, 7};
         else if (wl.n_split > 1 && ws_bytes >= wl.total) p = {NSA_PATH_SPLIT_K, 2};
@@ -368,6 +406,30 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
         return cuda_status(nsa::launch_attn(s, qb, kb, vb, kcb, vcb, gates, sel_idx, ob, cs));
     }
     // block-major selected branch when the workspace holds its index and partials
+    if (plan.path == NSA_PATH_BLOCK_MAJOR && wl.sub) {
+        const Shape t = sub_block_shape(s);
+        int32_t* idx_sub = reinterpret_cast<int32_t*>(ws + wl.idx_sub);
+        nsa::SelIndex x;
+        x.cnt = reinterpret_cast<int32_t*>(ws + wl.cnt);
+        x.off = reinterpret_cast<int32_t*>(ws + wl.off);
+        x.item_off = reinterpret_cast<int32_t*>(ws + wl.item_off);
+        x.cursor = reinterpret_cast<int32_t*>(ws + wl.cursor);
+        x.list = reinterpret_cast<int32_t*>(ws + wl.list);
+        x.items = reinterpret_cast<int4*>(ws + wl.items);
+        __nv_bfloat16* part_o = reinterpret_cast<__nv_bfloat16*>(ws + wl.part_o);
+        float* part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
+        g_timing.mark("expand", cs);
+        st = cuda_status(nsa::launch_sel_expand(s, sel_idx, idx_sub, cs));
+        if (st != NSA_OK) return st;
+        g_timing.mark("index", cs);
+        st = cuda_status(nsa::launch_sel_index(t, idx_sub, x, 128, cs));
+        if (st != NSA_OK) return st;
+        g_timing.mark("sel_bm", cs);
+        st = cuda_status(nsa::launch_sel_bm(t, qb, kb, vb, x, part_o, part_lse, cs));
+        if (st != NSA_OK) return st;
+        g_timing.mark("sel_merge", cs);
+        return cuda_status(nsa::launch_sel_merge_out(t, idx_sub, part_o, part_lse, gates, ob, cs));
+    }
     if (plan.path == NSA_PATH_BLOCK_MAJOR) {
         nsa::SelIndex x;
         x.cnt = reinterpret_cast<int32_t*>(ws + wl.cnt);

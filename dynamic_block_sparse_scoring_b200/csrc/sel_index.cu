@@ -127,7 +127,39 @@ __global__ void make_items_kernel(const int32_t* __restrict__ off,
     }
 }
 
+// One head per unit with blocks longer than 64 keys: a kept block becomes its
+// 64-key sub-blocks, so that the block-major kernel (64 keys per item) serves
+// it unchanged.  The selected branch is one softmax over every key of the kept
+// blocks up to the query, and the sub-blocks starting after the query hold
+// none of those keys, so they are dropped.  Row r of idx_sub lists the
+// sub-blocks of row r's kept blocks in order (ascending), -1 padded to
+// top_k * (sel_block / 64) entries.
+__global__ void expand_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ idx_sub, size_t rows,
+                              int Tq, int q0, int topk, int bs, int spb) {
+    for (size_t r = (size_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows;
+         r += (size_t)gridDim.x * blockDim.x) {
+        const int t = q0 + (int)(r % Tq);
+        const int32_t* src = idx + r * topk;
+        int32_t* dst = idx_sub + r * (size_t)topk * spb;
+        int n = 0;
+        for (int e = 0; e < topk; ++e) {
+            const int blk = src[e];
+            if (blk < 0 || blk > t / bs) continue;      // only causal blocks are attended
+            for (int sb = 0; sb < spb && blk * bs + sb * 64 <= t; ++sb) dst[n++] = blk * spb + sb;
+        }
+        for (; n < topk * spb; ++n) dst[n] = -1;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_sel_expand(const Shape& s, const int32_t* idx, int32_t* idx_sub, cudaStream_t st) {
+    const size_t rows = (size_t)s.B * s.Hsel * s.Tq;
+    if (rows == 0) return cudaSuccess;
+    const int grid = (int)std::min<size_t>((rows + 255) / 256, 148 * 16);
+    expand_kernel<<<grid, 256, 0, st>>>(idx, idx_sub, rows, s.Tq, s.q0, s.topk, s.bs, s.bs / 64);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_sel_index(const Shape& s, const int32_t* idx, const SelIndex& x, int tok,
                              cudaStream_t st) {

@@ -70,7 +70,85 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_
         pack8(acc);
 }
 
+// Selected branch alone with one head per unit (MoBA's per-head selection;
+// Zhang Xiaojun #94 transcript (bidclub.ai), §7: every head keeps its own
+// blocks and the output is that branch alone).  A kept block reaches here as
+// its 64-key sub-blocks, each one slot with its own partial; the merge is the
+// same normaliser-weighted sum, taken in batches of MO_BATCH slots whose loads
+// are issued together (running maximum rescaled between batches), and the
+// result is written to out with the branch's gate.  One thread per 8 output
+// columns of a (query, head).
+constexpr int MO_BATCH = 8;
+
+__global__ void __launch_bounds__(256) sel_merge_out_kernel(Shape s, const int32_t* __restrict__ idx,
+                                                            const __nv_bfloat16* __restrict__ part_o,
+                                                            const float* __restrict__ part_lse,
+                                                            const float* __restrict__ gates,
+                                                            __nv_bfloat16* __restrict__ out) {
+    const int c8n = s.dv / 8;
+    const size_t total = (size_t)s.B * s.Tq * s.Hq * c8n;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int c8 = (int)(e % c8n);
+        const size_t row = e / c8n;                     // (b, query, head) of out
+        const int hq = (int)(row % s.Hq);
+        const int qi = (int)((row / s.Hq) % s.Tq);
+        const int b = (int)(row / ((size_t)s.Hq * s.Tq));
+        const size_t prow0 = ((size_t)(b * s.Hsel + hq) * s.Tq + qi) * s.topk;   // unit = head
+        // the kept sub-blocks fill the first slots (-1 padded)
+        int nvalid = 0;
+        while (nvalid < s.topk && idx[prow0 + nvalid] >= 0) ++nvalid;
+        float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f, m = -INFINITY;
+        for (int kb = 0; kb < nvalid; kb += MO_BATCH) {
+            float lse[MO_BATCH];
+            uint4 raw[MO_BATCH];
+#pragma unroll
+            for (int k = 0; k < MO_BATCH; ++k) {
+                lse[k] = -INFINITY;
+                if (kb + k < nvalid) {
+                    lse[k] = __ldcs(part_lse + prow0 + kb + k);
+                    raw[k] = __ldcs(reinterpret_cast<const uint4*>(part_o + (prow0 + kb + k) * s.dv + c8 * 8));
+                }
+            }
+            float mb = m;
+#pragma unroll
+            for (int k = 0; k < MO_BATCH; ++k) mb = fmaxf(mb, lse[k]);
+            if (mb == -INFINITY) continue;             // nothing visible so far
+            const float sc = m == -INFINITY ? 0.f : exp2f(m - mb);
+            wsum *= sc;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) o[q] *= sc;
+            m = mb;
+#pragma unroll
+            for (int k = 0; k < MO_BATCH; ++k) {
+                if (kb + k >= nvalid) break;
+                const float w = exp2f(lse[k] - m);
+                wsum += w;
+                float f[8];
+                unpack8(raw[k], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) o[q] = fmaf(w, f[q], o[q]);
+            }
+        }
+        const float g = gates ? gates[row * 3 + 1] : 1.f;
+        const float scale = wsum > 0.f ? g / wsum : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[q] *= scale;
+        *reinterpret_cast<uint4*>(out + row * s.dv + c8 * 8) = pack8(o);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_sel_merge_out(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
+                                 const float* part_lse, const float* gates, __nv_bfloat16* out,
+                                 cudaStream_t st) {
+    const size_t total = (size_t)s.B * s.Tq * s.Hq * (s.dv / 8);
+    if (total == 0) return cudaSuccess;
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
+    sel_merge_out_kernel<<<grid, 256, 0, st>>>(s, idx, part_o, part_lse, gates, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
                              const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st) {

@@ -75,6 +75,15 @@ def test_workspace_sizes(abi):
     assert abi.nsa_attn_plan(abi.config(WORKLOADS["nsa64k"]), True,
                              abi.nsa_workspace_size(abi.config(WORKLOADS["nsa64k"])))[0] == "block-major"
     assert abi.nsa_attn_plan(abi.config(WORKLOADS["moba32k"]), True, 0)[0] == "rowwise"
+    # MoBA (selected branch alone, one head per unit, 512-key blocks): block-major over
+    # 64-key sub-blocks; expand + 4 index kernels + block-major + merge, after the selection
+    moba = abi.config(WORKLOADS["moba32k"])
+    n = abi.nsa_workspace_size(moba)
+    wl = WORKLOADS["moba32k"]
+    slots = wl.top_k * (wl.sel_block // 64)
+    assert n >= wl.seqlen_q * wl.h_q * slots * wl.d_v * 2
+    assert abi.nsa_attn_plan(moba, True, n) == ("block-major", 8)
+    assert abi.nsa_attn_plan(moba, True, abi.nsa_workspace_size_min(moba))[0] == "rowwise"
 
 
 @pytest.mark.parametrize("bad,status", [

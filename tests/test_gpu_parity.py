@@ -72,6 +72,13 @@ EDGE = {
     "dec_long_cache": WORKLOADS["decode64x64k"].with_(name="dec_long_cache", batch=1,
                                                        seqlen_kv=110000, q_pos0=109999, h_q=32,
                                                        h_kv=2),
+    # selected branch alone with one head per unit: block-major over 64-key sub-blocks
+    # (128-key blocks under GQA with a ragged cache; 256-key blocks filling all 32 slots)
+    "sub_gqa_bs128": TINY.with_(name="sub_gqa_bs128", seqlen_q=700, seqlen_kv=1000, q_pos0=300,
+                                h_q=4, h_kv=2, d_qk=128, d_v=128, sel_block=128, top_k=4,
+                                branches=BR_SEL, per_head_select=True),
+    "sub_slots32": TINY.with_(name="sub_slots32", seqlen_q=300, seqlen_kv=2500, q_pos0=2200,
+                              h_q=2, h_kv=2, sel_block=256, top_k=8, branches=BR_SEL, gated=False),
     # block-major selected branch (groups of 8 and 16 heads, sel_block 64, >= 256 queries)
     "bm_g8_ragged": WORKLOADS["nsa64k"].with_(name="bm_g8_ragged", seqlen_q=1000, seqlen_kv=1000,
                                               h_q=16, h_kv=2, d_qk=128, d_v=128),

@@ -8,15 +8,17 @@ pytestmark = pytest.mark.gpu
 
 
 STAGES = {"rowwise": ["rowwise"], "query-major": ["attn_tc"], "split-k": ["attn_tc", "split_merge"],
-          "block-major": ["index", "sel_bm", "sel_merge", "attn_tc"]}
+          "block-major": ["index", "sel_bm", "sel_merge", "attn_tc"],
+          # the selected branch alone, one head per unit: 64-key sub-blocks, merged into out
+          "block-major-sub": ["expand", "index", "sel_bm", "sel_merge"]}
 
 
-@pytest.mark.parametrize("name,seqlen,want_path", [
-    ("tiny", None, "split-k"),
-    ("nsa64k", 1024, "block-major"),
-    ("moba32k", 1024, "rowwise"),
+@pytest.mark.parametrize("name,seqlen,want_path,stage_key", [
+    ("tiny", None, "split-k", "split-k"),
+    ("nsa64k", 1024, "block-major", "block-major"),
+    ("moba32k", 1024, "block-major", "block-major-sub"),
 ])
-def test_stage_timing_follows_the_plan(name, seqlen, want_path):
+def test_stage_timing_follows_the_plan(name, seqlen, want_path, stage_key):
     from dynamic_block_sparse_scoring_b200 import abi as a
     wl = WORKLOADS[name]
     if seqlen:
@@ -36,7 +38,7 @@ def test_stage_timing_follows_the_plan(name, seqlen, want_path):
     finally:
         a.nsa_timing_enable(False)
     assert path == want_path
-    assert [n for n, _ in stages] == ["select"] + STAGES[path], stages
+    assert [n for n, _ in stages] == ["select"] + STAGES[stage_key], stages
     assert all(ms > 0 for _, ms in stages)
     # after disabling, a call records nothing new; the last timed call stays readable
     a.nsa_sparse_attn_fwd(cfg, x["q"], x["k"], x["v"], pooled["kbar"], pooled["kcmp"],
