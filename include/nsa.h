@@ -95,7 +95,9 @@ typedef struct {
  * the selected block ids (when it selects them itself) plus, for long
  * prefills on the tensor-core path, the per-block query lists and the
  * per-(query, slot) partial outputs of the block-major selected branch
- * (about topk * heads * d_v * 2 bytes per query).  Writes 0 when no
+ * (about topk * heads * d_v * 2 bytes per query; with the selected branch
+ * alone and one head per selection unit, a slot per 64-key sub-block of a
+ * kept block, i.e. sel_block / 64 times as many).  Writes 0 when no
  * workspace is needed.  Pure host function.
  */
 nsa_status nsa_workspace_size(const nsa_config* cfg, size_t* bytes);
@@ -161,7 +163,12 @@ nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kb
  * nsa_workspace_size() bytes enables the block-major selected branch (each
  * selected KV block attended once for all the queries that kept it); a
  * smaller one (or NULL with an external idx) computes the same result with
- * the selected branch inside the query-major kernel.
+ * the selected branch inside the query-major kernel.  With the selected
+ * branch alone and one head per selection unit (MoBA's per-head selection,
+ * transcript #94 §7), at least 256 query rows, sel_block a multiple of 64
+ * and top_k * sel_block / 64 <= 32, the full workspace runs the block-major
+ * kernel over the 64-key sub-blocks of the kept blocks and writes out from
+ * their merge directly.
  * kcmp/vcmp are read only with NSA_BR_CMP.
  */
 nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void* k,
@@ -202,7 +209,9 @@ nsa_status nsa_get_device_status(int32_t* status);
 /* Organisations of nsa_sparse_attn_fwd (same results, different speed). */
 #define NSA_PATH_ROWWISE 0       /* shapes outside the tensor-core kernels' limits */
 #define NSA_PATH_QUERY_MAJOR 1   /* tensor cores; selected branch over each tile's block union */
-#define NSA_PATH_BLOCK_MAJOR 2   /* + selected branch block-major (long prefills, full workspace) */
+#define NSA_PATH_BLOCK_MAJOR 2   /* + selected branch block-major (long prefills, full workspace;
+                                    the selected branch alone with one head per unit: 64-key
+                                    sub-blocks, no query-major kernel) */
 #define NSA_PATH_SPLIT_K 3       /* + each tile's keys split over several CTAs (few tiles) */
 #define NSA_PATH_DECODE 4        /* tensor cores with the keys as the MMA M dimension: <= 4 query
                                     rows per sequence, 8 or 16 heads per group, d_v 128, full workspace */
@@ -230,7 +239,8 @@ nsa_status nsa_attn_plan(const nsa_config* cfg, int select_inside, size_t ws_byt
  * call and writes up to `max_stages` stage names (static strings) and
  * durations in milliseconds; *n_stages receives the number of stages (0 if
  * no call was timed).  Stage names: "select" (score + top-k when idx is
- * NULL), "index" (block-major inverted index), "sel_bm" (block-major selected
+ * NULL), "expand" (kept blocks to 64-key sub-blocks), "index" (block-major
+ * inverted index), "sel_bm" (block-major selected
  * branch), "sel_merge", "attn_tc" (tensor-core branches + gated merge),
  * "split_merge", "attn_dec" (few-query kernel), "dec_merge", "rowwise".
  * Each stage's time runs from its first launch to the next stage's first
