@@ -299,13 +299,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         ok = false;
                         break;
                     }
-                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
+                    // one head per query (hpt == 1): the query rows are gathered four
+                    // at a time from q viewed as [B * Tq * Hq rows, DQK]; the last
+                    // group repeats its final row (rows >= n are never used)
+                    const int n4 = (m.n + 3) / 4;
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), n4 * 4 * L::QC * 128);
                     __syncwarp();
-                    for (int e = lane; e < m.n * L::QC; e += 32) {
-                        const int tt = e / L::QC, c = e % L::QC;
-                        tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
-                                             &map_qg, bar.q_full(qs), 64 * c, h0, metas[slot].tok[tt] >> 5, b,
-                                             q_policy);
+                    const int* toks = metas[slot].tok;
+                    const int qrow0 = (b * a.s.Tq) * a.s.Hq + h0;
+                    for (int e = lane; e < n4 * L::QC; e += 32) {
+                        const int g4 = e / L::QC, c = e % L::QC;
+                        int r[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            r[k] = qrow0 + (toks[min(4 * g4 + k, m.n - 1)] >> 5) * a.s.Hq;
+                        tc::tma_gather4_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + 4 * g4 * 128, &map_qg,
+                                             bar.q_full(qs), 64 * c, r[0], r[1], r[2], r[3], q_policy);
                     }
                 }
                 ++q_loads;
@@ -689,7 +698,12 @@ cudaError_t launch_bm_impl(const Shape& s, const __nv_bfloat16* q, const __nv_bf
     const cuuint64_t pd[2] = {(cuuint64_t)DV, (cuuint64_t)sel_partial_rows(s)};
     const cuuint64_t ps[1] = {(cuuint64_t)DV * 2};
     const cuuint32_t pb[2] = {64, (cuuint32_t)a.hpt};
-    if (!encode(&mq, q, 4, qd, qs, qb) || !encode(&mk, k, 3, kd, ks, kb) ||
+    // one head per query: q as [B * Tq * Hq rows, DQK], one-row boxes for the 4-row gathers
+    const cuuint64_t qd2[2] = {(cuuint64_t)DQK, (cuuint64_t)s.B * s.Tq * s.Hq};
+    const cuuint64_t qs2[1] = {(cuuint64_t)DQK * 2};
+    const cuuint32_t qb2[2] = {64, 1};
+    const bool q_ok = MT > 32 ? encode(&mq, q, 2, qd2, qs2, qb2) : encode(&mq, q, 4, qd, qs, qb);
+    if (!q_ok || !encode(&mk, k, 3, kd, ks, kb) ||
         !encode(&mv, v, 3, vd, vs, kb) || !encode(&mpo, part_o, 2, pd, ps, pb))
         return cudaErrorInvalidValue;
     int dev = 0, nsm = 148;
@@ -713,7 +727,9 @@ bool sel_bm_supported(const Shape& s) {
     if (s.bs != BLK) return false;
     const int hpt = s.heads_per_unit;
     // a slot is 5 bits of a list entry; the merge of groups takes up to 16 slots
-    const bool shape_ok = ((hpt == 8 || hpt == 16) && s.topk <= 16) || (hpt == 1 && s.topk <= 32);
+    // (one head per query: q rows are gathered by a 32-bit row index)
+    const bool shape_ok = ((hpt == 8 || hpt == 16) && s.topk <= 16) ||
+                          (hpt == 1 && s.topk <= 32 && (size_t)s.B * s.Tq * s.Hq < (size_t(1) << 31));
     // partial rows are addressed by 32-bit TMA coordinates
     return shape_ok && sel_partial_rows(s) < (size_t(1) << 31);
 }

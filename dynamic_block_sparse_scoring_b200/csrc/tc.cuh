@@ -112,6 +112,19 @@ __device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// Four rows of a 2-D tensor map, gathered by row index into consecutive
+// 128-byte rows of shared memory (box: 64 columns x 1 row).  c0 is the column
+// (innermost) coordinate, r0..r3 the rows.
+__device__ __forceinline__ void tma_gather4_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                                 int r0, int r1, int r2, int r3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+        "r"(r3), "l"(policy)
+        : "memory");
+}
+
 // L2 policy for lines written once and read back much later (evict_first).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
