@@ -564,8 +564,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 lidx = mref.lidx;
                 n = mref.n;
                 tokr = tt < MT ? mref.tok[tt] : 0;
+                // (one head per query: lane l stores rows 4l .. 4l + 3, one scatter of four)
 #pragma unroll
-                for (int g = 0; g < NG; ++g) tok_lane[g] = 32 * g + lane < MT ? mref.tok[32 * g + lane] : 0;
+                for (int g = 0; g < NG; ++g) {
+                    const int qi = MT > 32 ? 4 * lane + g : 32 * g + lane;
+                    tok_lane[g] = qi < MT ? mref.tok[qi] : 0;
+                }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
             }
@@ -622,13 +626,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::fence_proxy_async_smem();
                 tc::named_bar_sync(1, 128);
                 if (issuer) {
+                    uint8_t* stg = sm + L::STG_OFF + (halves & 1) * (BM * 128);
+                    if constexpr (MT > 32) {
+                        static_assert(NG == 4, "one scatter of four rows per lane");
+                        if (4 * lane + 3 < n) {
+                            tc::tma_scatter4(&map_po, stg + 4 * lane * 128, c, prow_q[0], prow_q[1], prow_q[2],
+                                             prow_q[3]);
+                        } else {
 #pragma unroll
-                    for (int g = 0; g < NG; ++g)
-                        if (32 * g + lane < n)
-                            tc::tma_store_2d_hint(&map_po,
-                                                  sm + L::STG_OFF + (halves & 1) * (BM * 128) +
-                                                      (32 * g + lane) * a.hpt * 128,
-                                                  c, prow_q[g], st_policy);
+                            for (int g = 0; g < NG; ++g)
+                                if (4 * lane + g < n)
+                                    tc::tma_store_2d_hint(&map_po, stg + (4 * lane + g) * 128, c, prow_q[g],
+                                                          st_policy);
+                        }
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < NG; ++g)
+                            if (32 * g + lane < n)
+                                tc::tma_store_2d_hint(&map_po, stg + (32 * g + lane) * a.hpt * 128, c, prow_q[g],
+                                                      st_policy);
+                    }
                     tc::bulk_commit();
                 }
             }

@@ -125,6 +125,17 @@ __device__ __forceinline__ void tma_gather4_hint(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// Four consecutive 128-byte rows of shared memory scattered to rows r0..r3 of
+// a 2-D tensor map (box: 64 columns x 1 row) at column c0; completes in the
+// thread's bulk group like the other TMA stores.
+__device__ __forceinline__ void tma_scatter4(const CUtensorMap* map, const void* src, int c0, int r0, int r1,
+                                             int r2, int r3) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile::scatter4.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
 // L2 policy for lines written once and read back much later (evict_first).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
