@@ -152,3 +152,25 @@ def test_timing_read_without_a_timed_call(abi):
     assert L.nsa_timing_read(0, None, None, None) == 1
     assert L.nsa_timing_enable(0) == 0
     assert abi.nsa_timing_read() == []
+
+
+def test_sub_block_path_conditions(abi):
+    """The per-head block-major path over 64-key sub-blocks takes the selected branch
+    alone, one head per unit, >= 256 query rows, sel_block a multiple of 64 and at most
+    32 sub-block slots per row; anything else keeps its previous organisation."""
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS, BR_SEL, BR_WIN
+    moba = WORKLOADS["moba32k"].with_(seqlen_q=1024, seqlen_kv=1024)
+
+    def plan(wl):
+        cfg = abi.config(wl)
+        return abi.nsa_attn_plan(cfg, True, abi.nsa_workspace_size(cfg))
+
+    assert plan(moba) == ("block-major", 8)
+    assert plan(moba.with_(sel_block=128, top_k=16))[0] == "block-major"   # 32 slots
+    assert plan(moba.with_(sel_block=128, top_k=17))[0] == "rowwise"       # 34 slots
+    assert plan(moba.with_(seqlen_q=255, q_pos0=769))[0] == "rowwise"      # few rows
+    assert plan(moba.with_(sel_block=96))[0] == "rowwise"                  # not a multiple of 64
+    assert plan(moba.with_(branches=BR_SEL | BR_WIN, window=128))[0] == "rowwise"
+    # the workspace holds one partial row per sub-block slot
+    small = abi.nsa_workspace_size(abi.config(moba.with_(sel_block=64, top_k=3)))
+    assert abi.nsa_workspace_size(abi.config(moba)) > 4 * small
