@@ -321,6 +321,28 @@ def test_selected_branch_matches_sdpa_with_block_mask():
         np.testing.assert_allclose(out[t], sdpa(q[t], K[0], V[0], cfg["scale"], m), atol=1e-12)
 
 
+def test_selected_branch_over_sub_blocks_is_the_same_softmax():
+    """The selected branch is one softmax over every key of the kept blocks up to the
+    query, so cutting each kept block into sub-blocks and keeping those that start at or
+    before the query changes neither the key set nor the output (the restatement the
+    per-head block-major path runs: 512-key blocks as 64-key sub-blocks; 32 as 8 here)."""
+    T, bs, sub = 200, 32, 8
+    spb = bs // sub
+    cfg = cfg_of(h_q=4, h_kv=2, sel_block=bs, top_k=3, branches=2, per_head_select=True)
+    q, K, V, _ = rand_problem(cfg, T, seed=21)
+    out, idx, _ = run(cfg, q, K, V, None)
+    n_units = idx.shape[0]
+    idx_sub = np.full((n_units, T, cfg["top_k"] * spb), -1, np.int64)
+    for u in range(n_units):
+        for t in range(T):
+            subs = [b * spb + k for b in idx[u, t] if b >= 0 for k in range(spb) if b * bs + k * sub <= t]
+            assert sorted(O.selected_keys(idx[u, t], t, bs)) == sorted(O.selected_keys(subs, t, sub))
+            idx_sub[u, t, :len(subs)] = subs
+    cfg_sub = dict(cfg, sel_block=sub, top_k=cfg["top_k"] * spb)
+    out_sub, _, _ = run(cfg_sub, q, K, V, None, idx=idx_sub)
+    np.testing.assert_allclose(out_sub, out, atol=1e-12)
+
+
 def test_top1_keeps_only_the_own_block():
     T = 48
     cfg = cfg_of(h_q=2, h_kv=1, sel_block=8, top_k=1, branches=2)
