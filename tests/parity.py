@@ -85,7 +85,8 @@ def check_idx(gpu_idx: np.ndarray, ora_idx: np.ndarray, gap: np.ndarray, scores:
     for u, r in zip(*np.nonzero(differ)):
         c = int(positions[r]) // sel_block
         got = [int(b) for b in gpu_idx[u, r] if b >= 0]
-        assert got == sorted(got) and c in got and len(got) == min(top_k, c + 1)
+        # strictly ascending (no repeated id), own block kept, right size
+        assert got == sorted(set(got)) and c in got and len(got) == min(top_k, c + 1)
         past = [b for b in got if b != c]
         dropped = [b for b in range(c) if b not in past]
         if past and dropped:

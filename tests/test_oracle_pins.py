@@ -149,6 +149,22 @@ def test_golden_figure2_selection():
     assert idx[0, 0].tolist() == gd["expected_blocks"]
 
 
+def test_golden_selection_gap():
+    """The near-tie measure: last kept minus first dropped past score, in fp32."""
+    gd = golden("selection_gap.json")
+    b_s = gd["sel_block"]
+    for row in gd["rows"]:
+        s = np.array(row["scores"], dtype=np.float64)
+        c = row["position"] // b_s
+        scores = np.full((1, 1, c + 1), -np.inf)
+        scores[0, 0, :len(s)] = s
+        idx, gap = O.select_blocks(scores, np.array([row["position"]]), b_s, row["top_k"])
+        got = [int(x) for x in idx[0, 0] if x >= 0]
+        assert got == row["expected_blocks"]
+        want = np.inf if row["expected_gap"] == "inf" else float(row["expected_gap"])
+        assert gap[0, 0] == want, (gap[0, 0], want)
+
+
 # ---------------------------------------------------------------------------
 # Top-k selection
 # ---------------------------------------------------------------------------
@@ -469,6 +485,25 @@ def _mut_select_higher_index_on_tie(scores, positions, sel_block, top_k):
     return idx, gap
 
 
+def _mut_gap_one_place_late(scores, positions, sel_block, top_k):
+    """Tie gap measured between the first and second dropped scores."""
+    U, R, nb = scores.shape
+    idx = np.full((U, R, top_k), -1, dtype=np.int32)
+    gap = np.full((U, R), np.inf)
+    for u in range(U):
+        for r in range(R):
+            c = int(positions[r]) // sel_block
+            n_cand = min(c, nb)
+            s = scores[u, r, :n_cand]
+            order = np.argsort(-s, kind="stable")
+            chosen = sorted([int(b) for b in order[:min(top_k - 1, n_cand)]] + [c])
+            idx[u, r, :len(chosen)] = chosen
+            if n_cand > top_k:
+                s32 = s.astype(np.float32).astype(np.float64)
+                gap[u, r] = s32[order[top_k - 1]] - s32[order[top_k]]
+    return idx, gap
+
+
 def _mut_scores_max_not_sum(q_rows, positions, Kbar, h_q, h_kv, sel_block, scale, per_head,
                             n_blocks):
     R = q_rows.shape[0]
@@ -496,11 +531,13 @@ MUTATIONS = {
     "compressed token visible at its first token": ("compressed_keys", _mut_compressed_early),
     "block mean drops a key": ("pool_block_keys", _mut_pool_drops_last),
     "tie goes to higher index": ("select_blocks", _mut_select_higher_index_on_tie),
+    "tie gap one place late": ("select_blocks", _mut_gap_one_place_late),
     "group max instead of sum": ("block_scores", _mut_scores_max_not_sum),
     "softmax normaliser clipped": ("softmax_attention", _mut_softmax_no_max),
 }
 
 PINS = [test_golden_uniform_query_outputs, test_golden_figure2_selection,
+        test_golden_selection_gap,
         test_golden_group_sum_selection, test_selection_ties_go_to_lower_index,
         test_window_of_one_returns_own_value, test_golden_softmax_two_keys,
         lambda: test_selected_branch_keeping_every_block_is_dense_causal(64),
