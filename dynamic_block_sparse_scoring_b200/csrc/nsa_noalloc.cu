@@ -11,17 +11,20 @@
 // The scratch array below is a file-scope __device__ array, so every GPU that
 // loads the library holds NOALLOC_SCRATCH_BYTES of device memory until the
 // process exits.  Its host-side name is only a stand-in for the symbol: the
-// device address is looked up with cudaGetSymbolAddress, once per device, on
-// the first call made with that device current, and cached.
+// device address is looked up with cudaGetSymbolAddress on every call, with
+// the caller's device current (a host-side lookup; nothing is cached, so a
+// cudaDeviceReset or another context on the same device cannot leave a stale
+// address behind).
 //
-// All calls share the one array and it keeps the last call's contents.  The
-// array holds the selected block ids, which the selection kernel overwrites
-// completely (every slot, -1 padding included) before the attention reads
-// them, so nothing in it has to start at zero.  Calls whose work overlaps on
-// the GPU (different streams, or different host threads without ordering)
-// race on the array: order them, e.g. by issuing them on one stream.
-#include <mutex>
-
+// All calls share the one array and it keeps the last call's contents.  It is
+// handed to nsa_sparse_attn_fwd as a workspace of NOALLOC_SCRATCH_BYTES bytes,
+// so it holds whatever scratch the plan for that size uses: the selected block
+// ids always, and the plan's index lists and partial results when the
+// problem's full workspace fits.  Every plan writes or clears what it reads
+// before reading it, so nothing in the array has to start at zero.  Calls
+// whose work overlaps on the GPU (different streams, or different host
+// threads without ordering) race on the array: order them, e.g. by issuing
+// them on one stream.
 #include "common.cuh"
 
 namespace {
@@ -30,22 +33,11 @@ constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(32) << 20;   // 32 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-constexpr int MAX_DEVICES = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[MAX_DEVICES] = {nullptr};
-
-// Device address of g_noalloc_scratch on the current device.
+// Device address of g_noalloc_scratch in the current context.
 nsa_status scratch_address(void** addr) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_CUDA;
-    if (dev < 0 || dev >= MAX_DEVICES) return NSA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return NSA_ERR_CUDA;
+    *addr = p;
     return NSA_OK;
 }
 

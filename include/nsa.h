@@ -188,10 +188,13 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
  * device.
  * Limit: problems with nsa_workspace_size_min() > 32 MiB return NSA_ERR_WORKSPACE
  * (e.g. 65536 queries x 4 selection units x top-16 need 16 MiB).
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it.  Every call uses the same array, which keeps
- * the previous call's contents (nothing in it needs to start at zero); calls
- * whose GPU work overlaps race on it, so order them (e.g. one stream).
+ * Every call looks up the array's device address on the current device (a
+ * host-side lookup, nothing cached) and passes the array as a workspace of
+ * 32 MiB, so it holds whatever scratch the plan for that size uses (the block
+ * ids, plus the plan's lists and partials when the full workspace fits).
+ * Every call uses the same array, which keeps the previous call's contents
+ * (nothing in it needs to start at zero); calls whose GPU work overlaps race
+ * on it, so order them (e.g. one stream).
  */
 nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, const void* k,
                                        const void* v, const float* kbar, const void* kcmp,

@@ -101,3 +101,27 @@ def check_out(gpu: np.ndarray, ora: np.ndarray, what=""):
     assert err.max() <= OUT_MAX_ABS, f"{what}: max abs err {err.max():.3e}"
     assert err.mean() <= OUT_MEAN_ABS, f"{what}: mean abs err {err.mean():.3e}"
     return float(err.max()), float(err.mean())
+
+
+def check_selection_all_rows(run: "GpuRun", chunk: int = 2048):
+    """Both GPU selections (stand-alone and inside the forward call) against the
+    oracle's selection on every query row of every sequence, in row chunks.
+
+    Returns the number of rows (per unit) resolved differently at a near-tie."""
+    wl = run.wl
+    nb_all = -(-wl.seqlen_kv // wl.sel_block)
+    ties = 0
+    for b in range(wl.batch):
+        Kbar = O.pool_block_keys(f64(run.x["k"][b]), wl.sel_block)
+        for r0 in range(0, wl.seqlen_q, chunk):
+            rows = np.arange(r0, min(wl.seqlen_q, r0 + chunk))
+            pos = rows + wl.q_pos0
+            rows_t = torch.as_tensor(rows, device=run.x["q"].device)
+            q = f64(run.x["q"][b].index_select(0, rows_t))
+            s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
+                               wl.per_head_select, nb_all)
+            ora_idx, gap = O.select_blocks(s, pos, wl.sel_block, wl.top_k)
+            for got in (run.idx, run.idx_fwd):
+                gpu_idx = got[b].index_select(1, rows_t).cpu().numpy()
+                ties += check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
+    return ties

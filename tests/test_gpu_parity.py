@@ -1,8 +1,9 @@
 """GPU parity: the C-ABI CUDA path against the fp64 oracle, element by element.
 
-Small problems are compared on every row; the full-size workloads on sampled
-rows (first rows, evenly strided rows, block boundaries, the last row) and,
-for decode, on sampled sequences.  Tolerances are stated in tests/parity.py.
+Small problems are compared on every row.  The full-size prefills have their
+selected block ids compared on every row, and their outputs on sampled rows
+(first rows, evenly strided rows, block boundaries, the last row); the decode
+batch is compared on every sequence.  Tolerances are stated in tests/parity.py.
 """
 import numpy as np
 import pytest
@@ -15,8 +16,8 @@ from oracle import nsa_oracle as O
 pytestmark = pytest.mark.gpu
 
 from dynamic_block_sparse_scoring_b200 import abi
-from tests.parity import (GpuRun, check_idx, check_out, f64, OUT_MAX_ABS, OUT_MEAN_ABS,
-                          SCORE_ATOL, SCORE_RTOL)
+from tests.parity import (GpuRun, check_idx, check_out, check_selection_all_rows, f64,
+                          OUT_MAX_ABS, OUT_MEAN_ABS, SCORE_ATOL, SCORE_RTOL)
 
 TINY = WORKLOADS["tiny"]
 
@@ -198,8 +199,10 @@ SAMPLED["bm_two_chunks"] = WORKLOADS["nsa64k"].with_(name="bm_two_chunks", seqle
 
 @pytest.mark.parametrize("name", sorted(SAMPLED))
 def test_full_size_prefill_sampled_rows(name):
+    """Selected ids on every row against the oracle; outputs on sampled rows."""
     wl = SAMPLED[name]
     run = GpuRun(wl)
+    check_selection_all_rows(run)
     T = wl.seqlen_q
     extra = [wl.sel_block - 1, wl.sel_block, wl.sel_block + 1, 511, 512, 513, T // 2, T - 2]
     extra += [r for r in (8190, 8191, 8192, 8193) if r < T]
@@ -219,10 +222,10 @@ def test_full_size_prefill_sampled_rows(name):
         assert bool(ascending.all())                                   # ascending, no repeats
 
 
-def test_decode_sampled_sequences():
+def test_decode_every_sequence():
     wl = WORKLOADS["decode64x64k"]
     run = GpuRun(wl)
-    compare_run(run, [0], seqs=[0, 31, 63])
+    compare_run(run, [0], seqs=range(wl.batch))
 
 
 @pytest.mark.parametrize("name", ["nsa_small", "bm_g8_ragged"])

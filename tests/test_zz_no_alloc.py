@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 
 OUT_MAX_ABS = 2e-2
 OUT_MEAN_ABS = 2e-3
+NOALLOC_BYTES = 32 << 20     # size of the library's scratch array
 
 
 def _forward_pair(wl, seed):
@@ -52,6 +53,36 @@ def test_noalloc_matches_regular_entry_point_twice_in_a_row(name):
         assert np.isfinite(got).all()
         err = np.abs(got - ref)
         assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS
+
+
+def test_noalloc_takes_the_small_workspace_plan_when_the_full_one_does_not_fit():
+    """Selected ids fit the 32 MiB array but the fastest plan's lists and partials
+    do not: the no-alloc call runs the plan a workspace of that size gets, which is
+    the plan of the minimal workspace, and matches the regular call given exactly
+    nsa_workspace_size_min() bytes."""
+    wl = WORKLOADS["nsa64k"].with_(name="nsa_tail4k", seqlen_q=4096, seqlen_kv=16384,
+                                   q_pos0=16384 - 4096)
+    cfg = abi.config(wl)
+    wmin, wfull = abi.nsa_workspace_size_min(cfg), abi.nsa_workspace_size(cfg)
+    assert wmin <= NOALLOC_BYTES < wfull
+    assert abi.nsa_attn_plan(cfg, True, NOALLOC_BYTES) == abi.nsa_attn_plan(cfg, True, wmin)
+    x = make_inputs(wl, device="cuda")
+    pooled = abi.alloc_pooled(cfg, "cuda")
+    abi.nsa_pool_kv(cfg, x["k"], x["v"], pooled["kbar"], pooled["kcmp"], pooled["vcmp"])
+    ws = torch.empty(wmin, dtype=torch.uint8, device="cuda")
+    ref = torch.empty(wl.batch, wl.seqlen_q, wl.h_q, wl.d_v, dtype=torch.bfloat16, device="cuda")
+    abi.nsa_sparse_attn_fwd(cfg, x["q"], x["k"], x["v"], pooled["kbar"], pooled["kcmp"],
+                            pooled["vcmp"], x["gates"], None, ref, ws, wmin)
+    for _ in range(2):
+        got = torch.full_like(ref, float("nan"))
+        status = abi.lib.nsa_sparse_attn_fwd_noalloc(
+            ctypes.byref(cfg), x["q"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(),
+            pooled["kbar"].data_ptr(), pooled["kcmp"].data_ptr(), pooled["vcmp"].data_ptr(),
+            x["gates"].data_ptr(), got.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert status == 0, abi.nsa_status_string(status)
+        torch.cuda.synchronize()
+        # same plan, same kernels, same inputs: the same bits
+        assert torch.equal(got, ref)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
