@@ -367,6 +367,28 @@ def stage_rooflines(wl: Workload, path: str, stage_ms: dict, idx: torch.Tensor, 
     return out
 
 
+SELECTED_STAGES = ("index", "sel_bm", "sel_merge", "expand")
+
+
+def selected_roofline(wl: Workload, path: str, stage_ms: dict, pk: dict):
+    """The selected branch's algorithmic FLOPs over the time of every stage that serves
+    only that branch (block-major plans: the inverted index, the block-major attention
+    and the partial merge; the selection itself is counted separately, as "select").
+    None when the plan computes the selected branch inside another kernel."""
+    if not wl.branches & 2 or path != "block-major":
+        return None
+    parts = {k: v for k, v in stage_ms.items() if k in SELECTED_STAGES}
+    if "sel_bm" not in parts:
+        return None
+    ms = sum(parts.values())
+    work = algorithmic_flops(wl)["sel"] * wl.batch
+    ach = work / (ms / 1e3) / 1e12
+    return {"stages": sorted(parts), "ms": ms, "bound": "tensor", "unit": "TFLOP/s",
+            "flops_per_step": work, "achieved": ach, "peak": pk["bf16_tflops"],
+            "frac": ach / pk["bf16_tflops"],
+            "peak_source": "measured dense bf16 (burst, cuBLAS)"}
+
+
 def e2e_steps(pf: Prefill, steps: int, warmup: int, world: int):
     """Same step through the public API with pinned host inputs: every step copies its
     own inputs host->device, runs the forward (pool + select + attention) and reads its
@@ -437,11 +459,14 @@ def cpu_baseline(wl: Workload, x, budget_s: float = 15.0, rows_per_step=None):
                 top_k=wl.top_k, window=wl.window, cmp_block=wl.cmp_block,
                 cmp_stride=wl.cmp_stride, scale=wl.scale, branches=wl.branches,
                 per_head_select=wl.per_head_select)
+    # One Python process walks the rows; only numpy's BLAS products inside a row may
+    # run on more threads.  Report the process as one core and the BLAS pool beside it.
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        blas_threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        cores = 1
+        blas_threads = 1
+    cores = 1
     K, V = f64(x["k"][0]), f64(x["v"][0])
     T = wl.seqlen_q
     t0 = time.perf_counter()
@@ -466,6 +491,9 @@ def cpu_baseline(wl: Workload, x, budget_s: float = 15.0, rows_per_step=None):
         rng_rows = np.linspace(done_rows % 7, T - 1, num=n).astype(np.int64)
     total = spent + t_pool
     return {"value": flops / total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "parallelism": f"one Python process (row loop single-threaded; numpy BLAS products "
+                           f"may use up to {blas_threads} threads of the {os.cpu_count()} host "
+                           f"cores)",
             "sample": f"{done_rows} evenly strided query rows of {wl.name} sequence 0 "
                       f"(all selection units, all branches, K/V pooling included: "
                       f"{t_pool:.1f} s pooling + {spent:.1f} s rows)",
@@ -525,7 +553,50 @@ def run_decode(world: int, steps: int, warmup: int):
             "bytes_per_step": nbytes, "frac": gbs / world / pk["hbm_gbs"],
             "peak_gbs": pk["hbm_gbs"], "path": path, "timing": "CUDA graph replay",
             "ms_per_step_stream": ms_stream,
+            "frac_stream": job_rate(nbytes, world, ms_stream) / 1e9 / world / pk["hbm_gbs"],
+            "frac_note": "frac: the step replayed as one CUDA graph; frac_stream: the same "
+                         "kernels launched one by one on the stream (host launch gaps included)",
             "stage_ms": dec_stages}
+
+
+def config_of(wl: Workload, world: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen_q,
+            "h_q": wl.h_q, "h_kv": wl.h_kv, "d_qk": wl.d_qk, "d_v": wl.d_v,
+            "sel_block": wl.sel_block, "top_k": wl.top_k, "window": wl.window,
+            "cmp": [wl.cmp_block, wl.cmp_stride],
+            "parallelism": f"independent sequences x{world}",
+            "l2": "256 MB flush before every step; inputs > L2"}
+
+
+def run_config(name: str, steps: int, warmup: int, world: int, rank: int):
+    """One prefill workload through the same step as the headline: mean step time,
+    tokens/s, algorithmic TFLOP/s and the stage rooflines."""
+    wl = WORKLOADS[name]
+    pf = Prefill(wl, seed=rank_seed(rank))
+    per, _, stage_ms = timed_steps(pf, steps, warmup, world)
+    ms = max_over_ranks(float(per.sum(axis=1).mean()), world)
+    fl = algorithmic_flops(wl)
+    pk, _ = peaks()
+    pf.attn_launches()
+    stages = stage_rooflines(wl, pf.path, stage_ms, pf.selected_ids(), pk)
+    launches = pf.launches_per_step
+    status = pf.abi.nsa_get_device_status()
+    res = {"workload": name, "batch": wl.batch, "seq_len": wl.seqlen_q, "h_q": wl.h_q,
+           "h_kv": wl.h_kv, "d_qk": wl.d_qk, "d_v": wl.d_v, "sel_block": wl.sel_block,
+           "top_k": wl.top_k, "per_head_select": wl.per_head_select, "steps": steps,
+           "ms_per_step": ms, "tokens_per_s": job_rate(wl.seqlen_q * wl.batch, world, ms),
+           "value": job_rate(fl["total"] * wl.batch, world, ms) / 1e12, "unit": "TFLOP/s",
+           "algorithmic_flops_per_step": fl["total"] * wl.batch, "path": pf.path,
+           "kernels_per_step": launches,
+           "stages": {k: {"ms": v["ms"], "achieved": v["achieved"], "unit": v["unit"],
+                          "frac": v["frac"], "bound": v["bound"]} for k, v in stages.items()},
+           "roofline_selected": selected_roofline(wl, pf.path, stage_ms, pk)}
+    del pf
+    torch.cuda.empty_cache()
+    if status != 0:
+        raise SystemExit(f"device status {status} on {name}: a kernel's bounded wait timed out")
+    return res
 
 
 def run_ours(args):
@@ -560,7 +631,8 @@ def run_ours(args):
     d["achieved"] *= d["ms"] / stage_ms_all[dom]       # slowest rank
     d["frac"] = d["achieved"] / d["peak"]
     kernel, source = STAGE_KERNELS[dom]
-    roof = {"kernel": kernel, "stage": dom, "bound": d["bound"], "achieved": d["achieved"],
+    roof = {"what": "dominant stage: the longest stage of the step",
+            "kernel": kernel, "stage": dom, "bound": d["bound"], "achieved": d["achieved"],
             "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
             "traffic": traffic_for(kernel, source),
             "peak_source": f"{src} " + ("dense bf16 (burst, cuBLAS)" if d["bound"] == "tensor"
@@ -571,6 +643,7 @@ def run_ours(args):
             "path": pf.path,
             "stages": {k: {"ms": v["ms"], "achieved": v["achieved"], "unit": v["unit"],
                            "frac": v["frac"], "bound": v["bound"]} for k, v in stages.items()}}
+    sel_roof = selected_roofline(wl, pf.path, {k: stage_ms_all[k] for k in stage_ms_all}, pk)
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_steps(pf, max(4, args.steps), 2, world)
@@ -588,23 +661,24 @@ def run_ours(args):
     del pf
     torch.cuda.empty_cache()
     decode = None if args.no_decode else run_decode(world, args.steps, args.warmup)
+    others = {}
+    if not args.no_configs:
+        for name in ("tiny", "moba32k", "nsa128k_planted"):
+            if name != wl.name:
+                others[name] = run_config(name, min(args.steps, 5), args.warmup, world, rank)
     cpu = cpu_baseline(wl, x_cpu) if x_cpu is not None else None
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16, sigmoid gates)",
-                "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen_q,
-                           "h_q": wl.h_q, "h_kv": wl.h_kv, "d_qk": wl.d_qk, "d_v": wl.d_v,
-                           "sel_block": wl.sel_block, "top_k": wl.top_k, "window": wl.window,
-                           "cmp": [wl.cmp_block, wl.cmp_stride],
-                           "parallelism": f"independent sequences x{world}",
-                           "l2": "256 MB flush before every step; inputs > L2"},
+                "config": config_of(wl, world),
                 "tokens_per_s": tokens, "algorithmic_flops_per_step": fl_all,
                 "stage_ms": {"pool": float(per[:, 0].mean()), "select": stage_ms.get("select", 0.0),
                              "attn": float(per[:, 2].mean()) - stage_ms.get("select", 0.0)},
-                "roofline": roof, "peaks": src, "cpu_baseline": cpu, "e2e": e2e,
-                "decode": decode, "gpu_launches": launches, "clocks": clk,
+                "roofline": roof, "roofline_selected": sel_roof, "peaks": src,
+                "cpu_baseline": cpu, "e2e": e2e,
+                "decode": decode, "configs": others, "gpu_launches": launches, "clocks": clk,
                 "wall_s_timed_region": wall}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -632,9 +706,10 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen_q},
+            "config": config_of(wl, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"],
-                             "kind": "oracle", "sample": res["sample"] + " per step"},
+                             "kind": "oracle", "parallelism": res["parallelism"],
+                             "sample": res["sample"] + " per step"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -650,6 +725,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other prefill workloads (tiny, moba32k, nsa128k_planted)")
     ap.add_argument("--seqlen", type=int, default=0, help="override the prefill length (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling)")
     args = ap.parse_args()
