@@ -1,0 +1,162 @@
+// Merge of the block-major selected-branch partials into one output per
+// (query, head): o_sel = sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M).
+//
+// Each slot's partial is a softmax over one kept block (Zhang Xiaojun #94
+// transcript (bidclub.ai), §4 "Inside Native Sparse Attention": the selected
+// branch is one softmax over every token of the kept blocks); weighting the
+// per-block results by their normalisers recovers that single softmax.
+//
+// HBM-bound: a thread owns 8 output columns of one (query, head) and issues
+// all of its slots' 16-byte partial loads (after one read of the query's
+// block ids) before combining them.
+#include "common.cuh"
+
+namespace nsa {
+
+namespace {
+
+constexpr int MG_MAXK = 16;   // slots per query handled here (the block-major path needs top_k <= 16)
+
+__global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
+                                                        const __nv_bfloat16* __restrict__ part_o,
+                                                        const float* __restrict__ part_lse,
+                                                        __nv_bfloat16* __restrict__ o_sel) {
+    // one CTA per query: the query's slot count and its (slot, head) log-sum-exps
+    // are staged once in shared memory (one coalesced read), so that every thread
+    // issues only its 16-byte partial loads
+    __shared__ float lse_s[MG_MAXK * 16];
+    __shared__ int nvalid_s;
+    const int hpt = s.heads_per_unit, c8n = s.dv / 8;
+    const int qi = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
+    const int h = threadIdx.x / c8n, c8 = threadIdx.x % c8n;
+    const size_t prow0 = ((size_t)(b * s.Hsel + u) * s.Tq + qi) * s.topk;
+    if (threadIdx.x < 32) {
+        // the kept blocks fill the first slots (ascending, -1 padded)
+        const int blk = threadIdx.x < s.topk ? idx[prow0 + threadIdx.x] : -1;
+        const int nv = __popc(__ballot_sync(0xffffffffu, blk >= 0));
+        if (threadIdx.x == 0) nvalid_s = nv;
+    }
+    for (int e = threadIdx.x; e < s.topk * hpt; e += blockDim.x)
+        lse_s[e] = __ldcs(part_lse + prow0 * hpt + e);
+    __syncthreads();
+    if (h >= hpt) return;
+    const int nvalid = nvalid_s;
+    uint4 raw[MG_MAXK];
+#pragma unroll
+    for (int sl = 0; sl < MG_MAXK; ++sl)              // every load of the row issued at once
+        if (sl < nvalid)
+            raw[sl] = __ldcs(reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8));
+    float m = -INFINITY;
+#pragma unroll
+    for (int sl = 0; sl < MG_MAXK; ++sl)
+        if (sl < nvalid) m = fmaxf(m, lse_s[sl * hpt + h]);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float wsum = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < MG_MAXK; ++sl) {
+        if (sl >= nvalid) break;
+        const float w = exp2f(lse_s[sl * hpt + h] - m);
+        wsum += w;
+        float f[8];
+        unpack8(raw[sl], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= inv;
+    const int hq = s.per_head ? u : u * s.G + h;
+    *reinterpret_cast<uint4*>(o_sel + (((size_t)b * s.Tq + qi) * s.Hq + hq) * s.dv + c8 * 8) =
+        pack8(acc);
+}
+
+// Selected branch alone with one head per unit (MoBA's per-head selection;
+// Zhang Xiaojun #94 transcript (bidclub.ai), §7: every head keeps its own
+// blocks and the output is that branch alone).  A kept block reaches here as
+// its 64-key sub-blocks, each one slot with its own partial; the merge is the
+// same normaliser-weighted sum, taken in batches of MO_BATCH slots whose loads
+// are issued together (running maximum rescaled between batches), and the
+// result is written to out with the branch's gate.  One thread per 8 output
+// columns of a (query, head).
+constexpr int MO_BATCH = 8;
+
+__global__ void __launch_bounds__(256) sel_merge_out_kernel(Shape s, const int32_t* __restrict__ idx,
+                                                            const __nv_bfloat16* __restrict__ part_o,
+                                                            const float* __restrict__ part_lse,
+                                                            const float* __restrict__ gates,
+                                                            __nv_bfloat16* __restrict__ out) {
+    const int c8n = s.dv / 8;
+    const size_t total = (size_t)s.B * s.Tq * s.Hq * c8n;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int c8 = (int)(e % c8n);
+        const size_t row = e / c8n;                     // (b, query, head) of out
+        const int hq = (int)(row % s.Hq);
+        const int qi = (int)((row / s.Hq) % s.Tq);
+        const int b = (int)(row / ((size_t)s.Hq * s.Tq));
+        const size_t prow0 = ((size_t)(b * s.Hsel + hq) * s.Tq + qi) * s.topk;   // unit = head
+        // the kept sub-blocks fill the first slots (-1 padded)
+        int nvalid = 0;
+        while (nvalid < s.topk && idx[prow0 + nvalid] >= 0) ++nvalid;
+        float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f, m = -INFINITY;
+        for (int kb = 0; kb < nvalid; kb += MO_BATCH) {
+            float lse[MO_BATCH];
+            uint4 raw[MO_BATCH];
+#pragma unroll
+            for (int k = 0; k < MO_BATCH; ++k) {
+                lse[k] = -INFINITY;
+                if (kb + k < nvalid) {
+                    lse[k] = __ldcs(part_lse + prow0 + kb + k);
+                    raw[k] = __ldcs(reinterpret_cast<const uint4*>(part_o + (prow0 + kb + k) * s.dv + c8 * 8));
+                }
+            }
+            float mb = m;
+#pragma unroll
+            for (int k = 0; k < MO_BATCH; ++k) mb = fmaxf(mb, lse[k]);
+            if (mb == -INFINITY) continue;             // nothing visible so far
+            const float sc = m == -INFINITY ? 0.f : exp2f(m - mb);
+            wsum *= sc;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) o[q] *= sc;
+            m = mb;
+#pragma unroll
+            for (int k = 0; k < MO_BATCH; ++k) {
+                if (kb + k >= nvalid) break;
+                const float w = exp2f(lse[k] - m);
+                wsum += w;
+                float f[8];
+                unpack8(raw[k], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) o[q] = fmaf(w, f[q], o[q]);
+            }
+        }
+        const float g = gates ? gates[row * 3 + 1] : 1.f;
+        const float scale = wsum > 0.f ? g / wsum : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[q] *= scale;
+        *reinterpret_cast<uint4*>(out + row * s.dv + c8 * 8) = pack8(o);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_sel_merge_out(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
+                                 const float* part_lse, const float* gates, __nv_bfloat16* out,
+                                 cudaStream_t st) {
+    const size_t total = (size_t)s.B * s.Tq * s.Hq * (s.dv / 8);
+    if (total == 0) return cudaSuccess;
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
+    sel_merge_out_kernel<<<grid, 256, 0, st>>>(s, idx, part_o, part_lse, gates, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
+                             const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st) {
+    // one CTA per query row: heads x 16-byte columns threads (<= 16 x 16)
+    const int threads = ((s.heads_per_unit * (s.dv / 8) + 31) / 32) * 32;
+    dim3 grid(s.Tq, s.Hsel, s.B);
+    sel_merge_kernel<<<grid, std::max(threads, 32), 0, st>>>(s, idx, part_o, part_lse, o_sel);
+    return cudaGetLastError();
+}
+
+}  // namespace nsa
