@@ -130,19 +130,94 @@ def block_scores(q_rows: np.ndarray, positions: np.ndarray, Kbar: np.ndarray, h_
     return out
 
 
-def select_blocks(scores: np.ndarray, positions: np.ndarray, sel_block: int, top_k: int):
+def block_scores_prob(q_rows: np.ndarray, positions: np.ndarray, Kbar: np.ndarray, h_q: int,
+                      h_kv: int, sel_block: int, scale: float, per_head: bool, n_blocks: int):
+    """Selection-score variant: each head's block probabilities, summed over the unit.
+
+    Transcript #94, §4 (GQA discussion): the group's heads add up their block
+    scores.  This variant reads "score" as the normalised score of §2 (after
+    the softmax) instead of the raw scaled dot product: per head h, the
+    softmax of scale * q_h . Kbar_b over the row's candidate blocks b < c(t),
+    then the sum over the unit's heads.  Shapes and -inf marking as in
+    ``block_scores``.
+    """
+    R = q_rows.shape[0]
+    units = selection_units(h_q, h_kv, per_head)
+    out = np.full((len(units), R, n_blocks), NEG_INF)
+    cur = positions // sel_block
+    nb_full = Kbar.shape[1]
+    for u, (hk, heads) in enumerate(units):
+        for r in range(R):
+            c = min(int(cur[r]), nb_full)
+            if c == 0:
+                continue
+            total = np.zeros(c)
+            for h in heads:
+                logits = scale * (Kbar[hk, :c] @ q_rows[r, h, :])
+                p = np.exp(logits - logits.max())
+                total += p / p.sum()
+            out[u, r, :c] = total
+    return out
+
+
+def block_scores_from_compressed(q_rows: np.ndarray, positions: np.ndarray, Kc: np.ndarray,
+                                 h_q: int, h_kv: int, sel_block: int, cmp_block: int,
+                                 cmp_stride: int, scale: float, per_head: bool, n_blocks: int):
+    """Selection-score variant: block scores taken from the compressed branch.
+
+    Transcript #94, §4: when the selection blocks and the compressed tokens
+    are cut differently, the selection score of a block has to be gathered
+    from the compressed tokens that overlap it (the "corner case").  Read
+    plainly: per head h, p_j = softmax over the visible compressed tokens
+    (j * stride + cmp_block - 1 <= t) of scale * q_h . Kc_j (the compressed
+    branch's attention weights); block b's score is sum_j p_j * w_jb with
+    w_jb = |[j*stride, j*stride + cmp_block) ∩ [b*sel_block, (b+1)*sel_block)|
+    / cmp_block, the share of token j's window inside block b; the unit sums
+    its heads.  Candidates are the past blocks b < c(t) as in ``block_scores``.
+    """
+    R = q_rows.shape[0]
+    units = selection_units(h_q, h_kv, per_head)
+    out = np.full((len(units), R, n_blocks), NEG_INF)
+    n_cmp = Kc.shape[1]
+    for u, (hk, heads) in enumerate(units):
+        for r in range(R):
+            t = int(positions[r])
+            c = t // sel_block
+            if c == 0:
+                continue
+            js = compressed_keys(t, n_cmp, cmp_block, cmp_stride)
+            total = np.zeros(c)
+            if len(js):
+                lo, hi = js * cmp_stride, js * cmp_stride + cmp_block
+                for h in heads:
+                    logits = scale * (Kc[hk, js] @ q_rows[r, h, :])
+                    p = np.exp(logits - logits.max())
+                    p /= p.sum()
+                    for b in range(c):
+                        ov = np.clip(np.minimum(hi, (b + 1) * sel_block) - np.maximum(lo, b * sel_block),
+                                     0, None)
+                        total[b] += float((p * ov).sum()) / cmp_block
+            out[u, r, :c] = total
+    return out
+
+
+def select_blocks(scores: np.ndarray, positions: np.ndarray, sel_block: int, top_k: int,
+                  n_sink: int = 0):
     """Top-k block sets from candidate scores.
 
     scores [n_units, R, n_blocks] (-inf for non-candidates).  For each row the
     current block c = pos // sel_block is always kept (LateTalk #103, §13:
-    MoBA's static part), plus the top (top_k - 1) past blocks by score, equal
-    scores going to the lower block index (transcript #94, §4, Figure 2:
-    keep the k highest-scoring blocks).  Returns
+    MoBA's static part), and so are the first ``n_sink`` blocks when they lie
+    before it (transcript #94, §4: the attention sink at the start of the
+    sequence, read as leading blocks kept like the current one); the rest of
+    the top_k places go to the best remaining past blocks by score, equal
+    scores going to the lower block index (transcript #94, §4, Figure 2: keep
+    the k highest-scoring blocks).  Returns
 
     * idx [n_units, R, top_k] int32, ascending, -1 padded;
     * gap [n_units, R]: the fp32-rounded difference between the last kept and
-      the first dropped past score (inf when every candidate is kept), which
-      says how close the row's selection is to a tie.
+      the first dropped scored past block (inf when every candidate is kept),
+      which says how close the row's selection is to a tie.
     """
     U, R, nb = scores.shape
     idx = np.full((U, R, top_k), -1, dtype=np.int32)
@@ -151,16 +226,18 @@ def select_blocks(scores: np.ndarray, positions: np.ndarray, sel_block: int, top
         for r in range(R):
             c = int(positions[r]) // sel_block
             n_cand = min(c, nb)
-            s = scores[u, r, :n_cand]
+            forced = list(range(min(n_sink, n_cand)))
+            free = top_k - 1 - len(forced)            # places left for scored blocks
+            rest = np.arange(len(forced), n_cand)
+            s = scores[u, r, rest]
             # stable sort on -s: equal scores keep ascending block order
             order = np.argsort(-s, kind="stable")
-            keep = order[:min(top_k - 1, n_cand)]
-            chosen = sorted([int(b) for b in keep] + [c])
+            keep = rest[order[:max(0, min(free, len(rest)))]]
+            chosen = sorted(forced + [int(b) for b in keep] + [c])
             idx[u, r, :len(chosen)] = chosen
-            if n_cand > top_k - 1:
+            if free >= 1 and len(rest) > free:
                 s32 = s.astype(np.float32).astype(np.float64)
-                gap[u, r] = s32[order[top_k - 2]] - s32[order[top_k - 1]] if top_k >= 2 \
-                    else np.inf
+                gap[u, r] = s32[order[free - 1]] - s32[order[free]]
     return idx, gap
 
 
@@ -213,12 +290,38 @@ def pooled_inputs(K, V, sel_block, cmp_block, cmp_stride):
             "Vc": compress(V, cmp_block, cmp_stride)}
 
 
+def opt(cfg, name, default):
+    """Optional configuration entry (mapping or attribute)."""
+    if isinstance(cfg, dict):
+        return cfg.get(name, default)
+    return getattr(cfg, name, default)
+
+
+def selection_scores(cfg, q_rows, positions, pooled, n_blocks):
+    """Block scores of the configured kind: "dot" (the scaled dot product with the
+    pooled key, summed over the unit; the default), "prob" (``block_scores_prob``)
+    or "cmp" (``block_scores_from_compressed``)."""
+    mode = opt(cfg, "score_mode", "dot")
+    h_q, h_kv, sel_block = opt(cfg, "h_q", 0), opt(cfg, "h_kv", 0), opt(cfg, "sel_block", 0)
+    scale, per_head = opt(cfg, "scale", 1.0), bool(opt(cfg, "per_head_select", False))
+    if mode == "prob":
+        return block_scores_prob(q_rows, positions, pooled["Kbar"], h_q, h_kv, sel_block, scale,
+                                 per_head, n_blocks)
+    if mode == "cmp":
+        return block_scores_from_compressed(q_rows, positions, pooled["Kc"], h_q, h_kv, sel_block,
+                                            opt(cfg, "cmp_block", 0), opt(cfg, "cmp_stride", 1),
+                                            scale, per_head, n_blocks)
+    return block_scores(q_rows, positions, pooled["Kbar"], h_q, h_kv, sel_block, scale, per_head,
+                        n_blocks)
+
+
 def nsa_rows(cfg, q_rows, positions, K, V, gates_rows=None, idx=None, pooled=None):
     """Gated NSA output for a set of query rows of one sequence.
 
     cfg: mapping or object with h_q, h_kv, d_qk, sel_block, top_k, window,
     cmp_block, cmp_stride, scale, branches (1 cmp | 2 sel | 4 win),
-    per_head_select, gated.
+    per_head_select, gated, and optionally score_mode ("dot", "prob", "cmp")
+    and sink_blocks (leading blocks always kept).
     q_rows [R, H_q, d_qk], positions [R], K [H_kv, T_kv, d_qk],
     V [H_kv, T_kv, d_v], gates_rows [R, H_q, 3] (cmp, sel, win) or None,
     idx: optional externally chosen [n_units, R, top_k] block sets,
@@ -242,15 +345,14 @@ def nsa_rows(cfg, q_rows, positions, K, V, gates_rows=None, idx=None, pooled=Non
     n_blocks = -(-T_kv // sel_block)
 
     if pooled is None:
-        pooled = pooled_inputs(K, V, sel_block, cmp_block if branches & 1 else 0,
-                               cmp_stride if branches & 1 else 1)
+        need_cmp = branches & 1 or opt(cfg, "score_mode", "dot") == "cmp"
+        pooled = pooled_inputs(K, V, sel_block, cmp_block if need_cmp else 0,
+                               cmp_stride if need_cmp else 1)
     gap = np.full((len(units), R), np.inf)
     if branches & 2:
         if idx is None:
-            Kbar = pooled["Kbar"]
-            s = block_scores(q_rows, positions, Kbar, h_q, h_kv, sel_block, scale, per_head,
-                             n_blocks)
-            idx, gap = select_blocks(s, positions, sel_block, top_k)
+            s = selection_scores(cfg, q_rows, positions, pooled, n_blocks)
+            idx, gap = select_blocks(s, positions, sel_block, top_k, opt(cfg, "sink_blocks", 0))
     if branches & 1:
         Kc, Vc = pooled["Kc"], pooled["Vc"]
         n_cmp = Kc.shape[1]

@@ -445,6 +445,151 @@ def test_external_idx_is_used():
 # Planted mistakes: each must make at least one pin above fail.
 # ---------------------------------------------------------------------------
 
+# ---------------------------------------------------------------------------
+# Selection-score variants and forced leading blocks
+# ---------------------------------------------------------------------------
+
+def test_golden_prob_selection():
+    """Probability-sum scores on a hand-computed 2-head example; the raw sum picks otherwise."""
+    gd = golden("prob_selection.json")
+    Kbar = np.array(gd["Kbar"])[None]                  # [1, nb_full, d]
+    q = np.array(gd["q"])[None]                        # [1 row, heads, d]
+    pos = np.array([gd["position"]])
+    args = (q, pos, Kbar, gd["h_q"], gd["h_kv"], gd["sel_block"], gd["scale"], False, 4)
+    s = O.block_scores_prob(*args)
+    np.testing.assert_allclose(s[0, 0, :3], gd["expected_scores"], atol=1e-7)
+    idx, _ = O.select_blocks(s, pos, gd["sel_block"], gd["top_k"])
+    assert idx[0, 0].tolist() == gd["expected_blocks"]
+    idx_raw, _ = O.select_blocks(O.block_scores(*args), pos, gd["sel_block"], gd["top_k"])
+    assert idx_raw[0, 0].tolist() == gd["expected_blocks_raw_sum"]
+
+
+def test_prob_scores_sum_to_the_number_of_heads():
+    """Each head's probabilities over the candidates sum to 1."""
+    cfg = cfg_of(h_q=8, h_kv=2, d_qk=32, d_v=16, sel_block=16, top_k=4)
+    q, K, V, _ = rand_problem(cfg, 200, seed=11)
+    pos = np.arange(200)
+    Kbar = O.pool_block_keys(K, 16)
+    s = O.block_scores_prob(q, pos, Kbar, 8, 2, 16, cfg["scale"], False, 13)
+    for r in range(200):
+        c = r // 16
+        if c:
+            np.testing.assert_allclose(s[:, r, :c].sum(axis=-1), 4.0, rtol=1e-12)
+
+
+def test_prob_selection_equals_raw_selection_for_single_head_units():
+    """Softmax is strictly increasing, so one head's probabilities rank blocks like its scores."""
+    cfg = cfg_of(h_q=4, h_kv=4, d_qk=32, d_v=16, sel_block=16, top_k=5)
+    q, K, V, _ = rand_problem(cfg, 300, seed=12)
+    pos = np.arange(300)
+    Kbar = O.pool_block_keys(K, 16)
+    args = (q, pos, Kbar, 4, 4, 16, cfg["scale"], True, 19)
+    a, _ = O.select_blocks(O.block_scores_prob(*args), pos, 16, 5)
+    b, _ = O.select_blocks(O.block_scores(*args), pos, 16, 5)
+    assert np.array_equal(a, b)
+
+
+def test_golden_compressed_aggregation():
+    """Uniform compressed probabilities spread over the overlapped blocks, by hand."""
+    gd = golden("cmp_aggregation.json")
+    rng = np.random.default_rng(13)
+    T = gd["position"] + 1
+    Kc = rng.standard_normal((1, O.n_compressed(T, gd["cmp_block"], gd["cmp_stride"]), 8))
+    q = np.zeros((1, gd["h_q"], 8))
+    pos = np.array([gd["position"]])
+    s = O.block_scores_from_compressed(q, pos, Kc, gd["h_q"], gd["h_kv"], gd["sel_block"],
+                                       gd["cmp_block"], gd["cmp_stride"], 1.0, False, 4)
+    np.testing.assert_allclose(s[0, 0, :3], gd["expected_scores"], rtol=1e-12)
+    idx, _ = O.select_blocks(s, pos, gd["sel_block"], gd["top_k"])
+    assert idx[0, 0].tolist() == gd["expected_blocks"]
+
+
+def test_compressed_aggregation_by_source_tokens():
+    """Brute force at the token level: every compressed token's probability is spread
+    evenly over its source tokens, and a block's score sums its tokens' shares."""
+    rng = np.random.default_rng(14)
+    h_q, h_kv, d, bs, lc, sc, T = 4, 2, 16, 16, 8, 4, 150
+    K = rng.standard_normal((h_kv, T, d))
+    Kc = O.compress(K, lc, sc)
+    q = rng.standard_normal((T, h_q, d))
+    pos = np.arange(T)
+    nb = -(-T // bs)
+    s = O.block_scores_from_compressed(q, pos, Kc, h_q, h_kv, bs, lc, sc, 0.3, False, nb)
+    G = h_q // h_kv
+    for r in range(0, T, 7):
+        c = r // bs
+        vis = [j for j in range(Kc.shape[1]) if j * sc + lc - 1 <= r]
+        for g in range(h_kv):
+            share = np.zeros(T + lc)
+            for h in range(g * G, (g + 1) * G):
+                if not vis:
+                    continue
+                lg = np.array([0.3 * float(q[r, h] @ Kc[g, j]) for j in vis])
+                w = np.exp(lg - lg.max())
+                w /= w.sum()
+                for wj, j in zip(w, vis):
+                    share[j * sc:j * sc + lc] += wj / lc
+            want = [share[b * bs:(b + 1) * bs].sum() for b in range(c)]
+            np.testing.assert_allclose(s[g, r, :c], want, rtol=1e-10, atol=1e-14)
+
+
+def test_compressed_aggregation_with_aligned_blocks_is_the_compressed_probability():
+    """cmp_block = cmp_stride = sel_block: token j is block j, so a block's score is the
+    unit's summed compressed-branch weight of that token."""
+    rng = np.random.default_rng(15)
+    h_q, h_kv, d, bs, T = 2, 1, 8, 8, 80
+    K = rng.standard_normal((h_kv, T, d))
+    Kc = O.compress(K, bs, bs)
+    q = rng.standard_normal((T, h_q, d))
+    pos = np.arange(T)
+    s = O.block_scores_from_compressed(q, pos, Kc, h_q, h_kv, bs, bs, bs, 1.0, False, T // bs)
+    for r in range(bs, T):
+        c = r // bs
+        vis = np.arange((r - bs + 1) // bs + 1)
+        want = np.zeros(c)
+        for h in range(h_q):
+            lg = Kc[0, vis] @ q[r, h]
+            w = np.exp(lg - lg.max())
+            want += (w / w.sum())[:c]
+        np.testing.assert_allclose(s[0, r, :c], want, rtol=1e-12)
+
+
+def brute_force_selection_with_sinks(s, c, k, n_sink):
+    forced = list(range(min(n_sink, c)))
+    rest = [b for b in range(len(forced), c)]
+    kept = []
+    for b in rest:
+        beaten_by = sum(1 for b2 in rest if s[b2] > s[b] or (s[b2] == s[b] and b2 < b))
+        if beaten_by < k - 1 - len(forced):
+            kept.append(b)
+    return sorted(forced + kept + [c])
+
+
+@pytest.mark.parametrize("n_sink", [1, 2, 3])
+def test_sink_blocks_match_brute_force(n_sink):
+    rng = np.random.default_rng(20 + n_sink)
+    T, b_s, k = 400, 16, 4
+    scores = np.full((2, T, 25), -np.inf)
+    for r in range(T):
+        c = r // b_s
+        scores[:, r, :c] = rng.integers(0, 4, size=(2, c))
+    idx, _ = O.select_blocks(scores, np.arange(T), b_s, k, n_sink)
+    for u in range(2):
+        for r in range(T):
+            c = r // b_s
+            got = [x for x in idx[u, r].tolist() if x >= 0]
+            assert got == brute_force_selection_with_sinks(scores[u, r], c, k, n_sink)
+            assert len(got) == min(k, c + 1)
+            assert all(b in got for b in range(min(n_sink, c)))
+
+
+def test_sinks_filling_every_free_place_keep_the_leading_blocks():
+    scores = np.random.default_rng(30).standard_normal((1, 1, 20))
+    idx, gap = O.select_blocks(scores, np.array([19 * 4]), 4, 5, n_sink=4)
+    assert idx[0, 0].tolist() == [0, 1, 2, 3, 19]
+    assert gap[0, 0] == np.inf
+
+
 def _mut_window_off_by_one(t, window):
     return np.arange(max(0, t - window + 2), t + 1, dtype=np.int64)
 
@@ -471,7 +616,7 @@ def _mut_pool_drops_last(K, sel_block):
     return out
 
 
-def _mut_select_higher_index_on_tie(scores, positions, sel_block, top_k):
+def _mut_select_higher_index_on_tie(scores, positions, sel_block, top_k, n_sink=0):
     U, R, nb = scores.shape
     idx = np.full((U, R, top_k), -1, dtype=np.int32)
     gap = np.full((U, R), np.inf)
@@ -485,7 +630,7 @@ def _mut_select_higher_index_on_tie(scores, positions, sel_block, top_k):
     return idx, gap
 
 
-def _mut_gap_one_place_late(scores, positions, sel_block, top_k):
+def _mut_gap_one_place_late(scores, positions, sel_block, top_k, n_sink=0):
     """Tie gap measured between the first and second dropped scores."""
     U, R, nb = scores.shape
     idx = np.full((U, R, top_k), -1, dtype=np.int32)
@@ -525,6 +670,43 @@ def _mut_softmax_no_max(q, k, v, scale):
     return (p / p.sum(axis=1, keepdims=True).clip(min=1.0)) @ v
 
 
+def _mut_prob_over_all_blocks(q_rows, positions, Kbar, h_q, h_kv, sel_block, scale, per_head,
+                              n_blocks):
+    """Probability-sum scores normalised over every pooled block, current and later ones too."""
+    R = q_rows.shape[0]
+    units = O.selection_units(h_q, h_kv, per_head)
+    out = np.full((len(units), R, n_blocks), -np.inf)
+    nb_full = Kbar.shape[1]
+    for u, (hk, heads) in enumerate(units):
+        for r in range(R):
+            c = min(int(positions[r]) // sel_block, nb_full)
+            if c == 0:
+                continue
+            total = np.zeros(nb_full)
+            for h in heads:
+                lg = scale * (Kbar[hk] @ q_rows[r, h])
+                p = np.exp(lg - lg.max())
+                total += p / p.sum()
+            out[u, r, :c] = total[:c]
+    return out
+
+
+def _mut_cmp_weight_in_tokens(q_rows, positions, Kc, h_q, h_kv, sel_block, cmp_block, cmp_stride,
+                              scale, per_head, n_blocks):
+    """Compressed aggregation weighted by overlapping tokens, not by the share of the window."""
+    return O_REAL_CMP(q_rows, positions, Kc, h_q, h_kv, sel_block, cmp_block, cmp_stride, scale,
+                      per_head, n_blocks) * cmp_block
+
+
+def _mut_sinks_outside_k(scores, positions, sel_block, top_k, n_sink=0):
+    """Sink blocks added on top of k - 1 scored blocks."""
+    return O_REAL_SELECT(scores, positions, sel_block, top_k + min(n_sink, 1) * n_sink, 0)
+
+
+O_REAL_CMP = O.block_scores_from_compressed
+O_REAL_SELECT = O.select_blocks
+
+
 MUTATIONS = {
     "window off by one": ("window_keys", _mut_window_off_by_one),
     "selected keys exclude self": ("selected_keys", _mut_selected_strict_causal),
@@ -534,10 +716,15 @@ MUTATIONS = {
     "tie gap one place late": ("select_blocks", _mut_gap_one_place_late),
     "group max instead of sum": ("block_scores", _mut_scores_max_not_sum),
     "softmax normaliser clipped": ("softmax_attention", _mut_softmax_no_max),
+    "probabilities normalised over later blocks": ("block_scores_prob", _mut_prob_over_all_blocks),
+    "compressed weights in tokens": ("block_scores_from_compressed", _mut_cmp_weight_in_tokens),
+    "sinks kept outside k": ("select_blocks", _mut_sinks_outside_k),
 }
 
 PINS = [test_golden_uniform_query_outputs, test_golden_figure2_selection,
-        test_golden_selection_gap,
+        test_golden_selection_gap, test_golden_prob_selection, test_prob_scores_sum_to_the_number_of_heads,
+        test_golden_compressed_aggregation, test_compressed_aggregation_by_source_tokens,
+        lambda: test_sink_blocks_match_brute_force(2),
         test_golden_group_sum_selection, test_selection_ties_go_to_lower_index,
         test_window_of_one_returns_own_value, test_golden_softmax_two_keys,
         lambda: test_selected_branch_keeping_every_block_is_dense_causal(64),
