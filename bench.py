@@ -213,6 +213,36 @@ class Prefill:
         self.ws_bytes = abi.nsa_workspace_size(self.cfg)
         self.ws = torch.empty(max(self.ws_bytes, 1), dtype=torch.uint8, device="cuda")
         self.launches_per_step = 0
+        self.append = None
+
+    def enable_append(self, seed: int):
+        """Decode: each step first appends the query's own token to the cache
+        (nsa_append_kv at the query position, refreshing the pooled tokens it completes)
+        instead of pooling the whole cache."""
+        wl = self.wl
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed)
+        self.append = {
+            "cfg": self.abi.config(wl, seqlen_q=1, q_pos0=wl.q_pos0),
+            "k": torch.randn(wl.batch, wl.h_kv, 1, wl.d_qk, generator=g, device="cuda").to(torch.bfloat16),
+            "v": torch.randn(wl.batch, wl.h_kv, 1, wl.d_v, generator=g, device="cuda").to(torch.bfloat16)}
+
+    def append_bytes(self) -> float:
+        """Bytes one append moves: the new rows, the keys of the selection block and the
+        K/V window of the compressed token it completes (if any), and their pooled tokens."""
+        wl, t = self.wl, self.wl.q_pos0
+        rows = wl.batch * wl.h_kv
+        n = rows * (wl.d_qk + wl.d_v) * 2                              # new K/V rows written
+        if (t + 1) % wl.sel_block == 0:
+            n += rows * (wl.sel_block * wl.d_qk * 2 + wl.d_qk * 4)     # block keys read, mean written
+        if t + 1 >= wl.cmp_block and (t + 1 - wl.cmp_block) % wl.cmp_stride == 0:
+            n += rows * (wl.cmp_block + 1) * (wl.d_qk + wl.d_v) * 2    # window read, token written
+        return float(n)
+
+    def append_launches(self) -> int:
+        wl, t = self.wl, self.wl.q_pos0
+        return 1 + int((t + 1) % wl.sel_block == 0) + \
+            int(t + 1 >= wl.cmp_block and (t + 1 - wl.cmp_block) % wl.cmp_stride == 0)
 
     def attn_launches(self) -> int:
         """Kernels nsa_sparse_attn_fwd launches with the selection inside (the library
@@ -226,7 +256,11 @@ class Prefill:
         n = 0
         if ev:
             ev[0].record()
-        if pool:
+        if pool and self.append is not None:
+            ap = self.append
+            a.nsa_append_kv(ap["cfg"], x["k"], x["v"], ap["k"], ap["v"], p["kbar"], p["kcmp"], p["vcmp"])
+            n += self.append_launches()
+        elif pool:
             a.nsa_pool_kv(self.cfg, x["k"], x["v"], p["kbar"], p["kcmp"], p["vcmp"])
             n += int(self.wl.branches & 2 > 0 and self.cfg.seqlen_kv >= self.cfg.sel_block) + \
                 int(self.wl.branches & 1 > 0)
@@ -501,20 +535,21 @@ def cpu_baseline(wl: Workload, x, budget_s: float = 15.0, rows_per_step=None):
 
 
 def graph_steps(pf: Prefill, steps: int, warmup: int, world: int) -> float:
-    """Mean device time of one step without pooling (selection + attention), captured once
-    as a CUDA graph and replayed, so that host launch gaps between the few short kernels of
-    a decode step are not counted.  The 256 MB L2 flush runs before every replay, outside
-    the timed events."""
+    """Mean device time of one decode step (the cache append when enabled, selection,
+    attention), captured once as a CUDA graph and replayed, so that host launch gaps
+    between the few short kernels of a decode step are not counted.  The 256 MB L2 flush
+    runs before every replay, outside the timed events."""
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
+    pool = pf.append is not None                      # decode: the append is part of the step
     with torch.cuda.stream(side):                    # warm-up (and lazy set-up) outside capture
-        pf.step(pool=False)
+        pf.step(pool=pool)
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        pf.step(pool=False)
+        pf.step(pool=pool)
     for _ in range(warmup):
         flush.fill_(1.0)
         g.replay()
@@ -536,23 +571,30 @@ def graph_steps(pf: Prefill, steps: int, warmup: int, world: int) -> float:
 
 def run_decode(world: int, steps: int, warmup: int):
     wl = WORKLOADS["decode64x64k"]
-    pf = Prefill(wl, seed=rank_seed(torch.distributed.get_rank() if world > 1 else 0, decode=True))
-    pf.step()                        # pooled cache built once (cache maintenance, not timed)
+    seed = rank_seed(torch.distributed.get_rank() if world > 1 else 0, decode=True)
+    pf = Prefill(wl, seed=seed)
+    pf.step()                        # the prefilled cache pooled once (before decoding, not timed)
     torch.cuda.synchronize()
-    per, _, dec_stages = timed_steps(pf, steps, warmup, world, pool=False)
+    # a decode step: append the query's own token (pooled tokens refreshed incrementally),
+    # select, attend
+    pf.enable_append(seed + 500)
+    per, _, dec_stages = timed_steps(pf, steps, warmup, world, pool=True)
     pf.attn_launches()
     path = pf.path
-    ms_stream = float(per[:, 1:].sum(axis=1).mean())
+    ms_stream = float(per.sum(axis=1).mean())
+    ms_append = float(per[:, 0].mean())
     ms = max_over_ranks(graph_steps(pf, steps, warmup, world), world)
-    nbytes = decode_bytes(wl, pf.selected_ids())
+    nbytes = decode_bytes(wl, pf.selected_ids()) + pf.append_bytes()
     pk, _ = peaks()
     gbs = job_rate(nbytes, world, ms) / 1e9
+    pf_append_bytes = pf.append_bytes()
     del pf
     torch.cuda.empty_cache()
     return {"workload": wl.name, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
             "bytes_per_step": nbytes, "frac": gbs / world / pk["hbm_gbs"],
             "peak_gbs": pk["hbm_gbs"], "path": path, "timing": "CUDA graph replay",
-            "ms_per_step_stream": ms_stream,
+            "ms_per_step_stream": ms_stream, "append_ms_stream": ms_append,
+            "append_bytes": pf_append_bytes,
             "frac_stream": job_rate(nbytes, world, ms_stream) / 1e9 / world / pk["hbm_gbs"],
             "frac_note": "frac: the step replayed as one CUDA graph; frac_stream: the same "
                          "kernels launched one by one on the stream (host launch gaps included)",

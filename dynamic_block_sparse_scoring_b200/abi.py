@@ -23,6 +23,7 @@ if not os.path.exists(_LIB_PATH):
 lib = ctypes.CDLL(_LIB_PATH)
 
 NSA_BR_CMP, NSA_BR_SEL, NSA_BR_WIN, NSA_PER_HEAD_SELECT = 1, 2, 4, 8
+NSA_SCORE_PROB, NSA_SCORE_CMP, NSA_SINK_SHIFT, NSA_DEBUG_CHECKS = 16, 32, 16, 64
 STATUS = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED", 3: "NSA_ERR_WORKSPACE",
           4: "NSA_ERR_CUDA", 5: "NSA_ERR_TIMEOUT"}
 
@@ -53,14 +54,18 @@ _SIGS = {
     "nsa_workspace_size": [_cfgp, ctypes.POINTER(_sz)],
     "nsa_workspace_size_min": [_cfgp, ctypes.POINTER(_sz)],
     "nsa_pool_kv": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "nsa_append_kv": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "nsa_score_blocks": [_cfgp, _vp, _vp, _vp, _vp],
     "nsa_topk_select": [_cfgp, _vp, _vp, _vp, _vp, _vp],
+    "nsa_score_blocks_ex": [_cfgp, _vp, _vp, _vp, _vp, _vp],
+    "nsa_topk_select_ex": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp],
     "nsa_sparse_attn_fwd": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "nsa_sparse_attn_fwd_noalloc": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "nsa_get_device_status": [ctypes.POINTER(ctypes.c_int32)],
     "nsa_attn_plan": [_cfgp, ctypes.c_int, _sz, ctypes.POINTER(ctypes.c_int32),
                       ctypes.POINTER(ctypes.c_int32)],
     "nsa_timing_enable": [ctypes.c_int32],
+    "nsa_check_bounded_wait": [ctypes.c_uint64, _vp],
     "nsa_timing_read": [ctypes.c_int32, ctypes.POINTER(ctypes.c_float),
                         ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_int32)],
 }
@@ -122,6 +127,10 @@ def nsa_attn_plan(cfg: NsaConfig, select_inside: bool, ws_bytes: int):
     return PATHS[path.value], n.value
 
 
+def nsa_check_bounded_wait(limit_ns: int, stream=None):
+    _check("nsa_check_bounded_wait", lib.nsa_check_bounded_wait(limit_ns, _stream(stream)))
+
+
 def nsa_get_device_status() -> int:
     """Reads and clears the device status word (0 = OK, 5 = a bounded wait timed out)."""
     v = ctypes.c_int32(0)
@@ -161,6 +170,25 @@ def nsa_workspace_size_min(cfg: NsaConfig) -> int:
 def nsa_pool_kv(cfg, k, v, kbar, kcmp=None, vcmp=None, stream=None):
     _check("nsa_pool_kv", lib.nsa_pool_kv(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(kbar),
                                           _ptr(kcmp), _ptr(vcmp), _stream(stream)))
+
+
+def nsa_append_kv(cfg, k, v, k_new, v_new, kbar=None, kcmp=None, vcmp=None, stream=None):
+    """Append cfg.seqlen_q tokens per sequence at KV position cfg.q_pos0 and refresh the
+    pooled tokens they complete (cfg.seqlen_kv = cache rows per plane)."""
+    _check("nsa_append_kv", lib.nsa_append_kv(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(k_new),
+                                              _ptr(v_new), _ptr(kbar), _ptr(kcmp), _ptr(vcmp),
+                                              _stream(stream)))
+
+
+def nsa_score_blocks_ex(cfg, q, kbar, kcmp, scores, stream=None):
+    _check("nsa_score_blocks_ex", lib.nsa_score_blocks_ex(ctypes.byref(cfg), _ptr(q), _ptr(kbar),
+                                                          _ptr(kcmp), _ptr(scores), _stream(stream)))
+
+
+def nsa_topk_select_ex(cfg, q, kbar, kcmp, scores, idx, stream=None):
+    _check("nsa_topk_select_ex", lib.nsa_topk_select_ex(ctypes.byref(cfg), _ptr(q), _ptr(kbar),
+                                                        _ptr(kcmp), _ptr(scores), _ptr(idx),
+                                                        _stream(stream)))
 
 
 def nsa_score_blocks(cfg, q, kbar, scores, stream=None):

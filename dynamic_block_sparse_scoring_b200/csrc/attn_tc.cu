@@ -1041,6 +1041,28 @@ cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o
     return cudaGetLastError();
 }
 
+// Self-test of the failure path shared by the tensor-core kernels: one warp
+// waits, with the same bounded wait, on an mbarrier whose phase nothing ever
+// completes, gives up after `limit_ns` and records NSA_ERR_TIMEOUT in the
+// same status word, exactly as a kernel whose copy or MMA never arrived.
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncwarp();
+    const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar, 0, &abort_flag, limit_ns));
+    if (!ok && threadIdx.x == 0) raise_abort(&abort_flag);
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns);
+    return cudaGetLastError();
+}
+
 int read_and_clear_tc_status() {
     int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, g_tc_status, sizeof(int)) != cudaSuccess) return -1;

@@ -18,6 +18,8 @@ struct Shape {
     int n_cmp;      // compressed tokens
     int Hsel;       // selection units (KV heads or query heads)
     int heads_per_unit;
+    int score_mode; // 0 scaled dot product, 1 probability sums, 2 from the compressed branch
+    int n_sink;     // leading blocks always kept
     bool per_head;
     float scale;
     uint32_t flags;
@@ -75,9 +77,21 @@ namespace nsa {
 cudaError_t launch_pool_kv(const Shape& s, const __nv_bfloat16* k, const __nv_bfloat16* v,
                            float* kbar, __nv_bfloat16* kcmp, __nv_bfloat16* vcmp,
                            cudaStream_t st);
+// pooled tokens of selection blocks [jb0, jb1) and compressed tokens [jc0, jc1)
+cudaError_t launch_pool_range(const Shape& s, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                              float* kbar, __nv_bfloat16* kcmp, __nv_bfloat16* vcmp, int jb0, int jb1,
+                              int jc0, int jc1, cudaStream_t st);
+// rows [t0, t0 + n_new) of every (sequence, KV head) plane of k / v (v may be null)
+cudaError_t launch_append_rows(const Shape& s, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                               __nv_bfloat16* k, __nv_bfloat16* v, int t0, int n_new, cudaStream_t st);
 cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
                               const float* scores_in, float* scores_out, int32_t* idx,
                               cudaStream_t st);
+// selection-score variants (score_mode 1 or 2): scores and/or top-k per row
+bool score_variant_supported(const Shape& s);
+cudaError_t launch_score_variant(const Shape& s, const __nv_bfloat16* q, const float* kbar,
+                                 const __nv_bfloat16* kcmp, float* scores_out, int32_t* idx,
+                                 cudaStream_t st);
 cudaError_t launch_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
                         const __nv_bfloat16* v, const __nv_bfloat16* kcmp,
                         const __nv_bfloat16* vcmp, const float* gates, const int32_t* idx,
@@ -94,6 +108,10 @@ cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o
                                const float* split_lse, const float* gates, __nv_bfloat16* out,
                                cudaStream_t st);
 int read_and_clear_tc_status();
+// the bounded wait's failure path on a barrier nothing completes (attn_tc.cu)
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st);
+// number of invalid rows of a caller-supplied idx into *bad (synchronises st) (sel_index.cu)
+cudaError_t check_idx_rows(const Shape& s, const int32_t* idx, int* bad, cudaStream_t st);
 cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
                              const float* part_lse, __nv_bfloat16* o_sel, cudaStream_t st);
 // selected branch alone, one head per unit: out = g_sel * (merge of the row's

@@ -7,6 +7,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "sel_index.cuh"
 
@@ -23,8 +25,14 @@ bool supported_dv(int d) { return d == 64 || d == 128 || d == 256; }
 nsa_status make_shape(const nsa_config* cfg, Shape* s) {
     if (!cfg || !s) return NSA_ERR_INVALID_ARG;
     const nsa_config& c = *cfg;
-    const uint32_t known = NSA_BR_CMP | NSA_BR_SEL | NSA_BR_WIN | NSA_PER_HEAD_SELECT;
+    const uint32_t known = NSA_BR_CMP | NSA_BR_SEL | NSA_BR_WIN | NSA_PER_HEAD_SELECT | NSA_SCORE_PROB |
+                           NSA_SCORE_CMP | NSA_DEBUG_CHECKS | (0xFFu << NSA_SINK_SHIFT);
     if (c.flags & ~known) return NSA_ERR_INVALID_ARG;
+    if ((c.flags & NSA_SCORE_PROB) && (c.flags & NSA_SCORE_CMP)) return NSA_ERR_INVALID_ARG;
+    // scores from the compressed branch need its compressed tokens
+    if ((c.flags & NSA_SCORE_CMP) && !(c.flags & NSA_BR_CMP)) return NSA_ERR_INVALID_ARG;
+    const int n_sink = (int)((c.flags >> NSA_SINK_SHIFT) & 0xFFu);
+    if (n_sink > 0 && (!(c.flags & NSA_BR_SEL) || n_sink > c.top_k - 1)) return NSA_ERR_INVALID_ARG;
     if (!(c.flags & (NSA_BR_CMP | NSA_BR_SEL | NSA_BR_WIN))) return NSA_ERR_INVALID_ARG;
     if (c.batch < 1 || c.seqlen_q < 0 || c.seqlen_kv < 1 || c.q_pos0 < 0) return NSA_ERR_INVALID_ARG;
     if ((int64_t)c.q_pos0 + c.seqlen_q > c.seqlen_kv) return NSA_ERR_INVALID_ARG;
@@ -71,6 +79,9 @@ nsa_status make_shape(const nsa_config* cfg, Shape* s) {
     s->heads_per_unit = per_head ? 1 : G;
     s->scale = c.scale;
     s->flags = c.flags;
+    s->n_sink = n_sink;
+    s->score_mode = (c.flags & NSA_SCORE_PROB) ? 1 : ((c.flags & NSA_SCORE_CMP) ? 2 : 0);
+    if (s->score_mode != 0 && !nsa::score_variant_supported(*s)) return NSA_ERR_UNSUPPORTED;
     return NSA_OK;
 }
 
@@ -111,7 +122,7 @@ bool use_sub_block_major(const Shape& s) {
 
 // Selection inside nsa_sparse_attn_fwd on the tensor cores: prefill-sized
 // problems (the few-row kernel serves <= 16 rows).
-bool use_score_tc(const Shape& s) { return nsa::score_tc_supported(s) && s.Tq > 16; }
+bool use_score_tc(const Shape& s) { return s.score_mode == 0 && nsa::score_tc_supported(s) && s.Tq > 16; }
 
 // Few query rows per sequence (decode): keys as the MMA M dimension.
 bool use_decode(const Shape& s) { return nsa::attn_dec_supported(s); }
@@ -327,34 +338,97 @@ nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, floa
         need_cmp ? static_cast<__nv_bfloat16*>(vcmp) : nullptr, static_cast<cudaStream_t>(stream)));
 }
 
-nsa_status nsa_score_blocks(const nsa_config* cfg, const void* q, const float* kbar, float* scores,
-                            void* stream) {
+// floor(a / b) for b > 0 and any a
+static int floor_div(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+nsa_status nsa_append_kv(const nsa_config* cfg, void* k, void* v, const void* k_new, const void* v_new,
+                         float* kbar, void* kcmp, void* vcmp, void* stream) {
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    if (s.Tq < 1) return NSA_ERR_INVALID_ARG;
+    if (!k || !v || !k_new || !v_new) return NSA_ERR_INVALID_ARG;
+    const int t0 = s.q0, t1 = s.q0 + s.Tq;      // new rows [t0, t1)
+    // selection blocks ending inside [t0, t1): j * bs + bs - 1 in [t0, t1)
+    const bool sel = (cfg->flags & NSA_BR_SEL) != 0;
+    const int jb0 = t0 / s.bs, jb1 = sel ? std::min(t1 / s.bs, s.nb_full) : jb0;
+    // compressed tokens whose window ends inside [t0, t1): j * sc + lc - 1 in [t0, t1)
+    const bool cmp = (cfg->flags & NSA_BR_CMP) != 0;
+    int jc0 = 0, jc1 = 0;
+    if (cmp && s.n_cmp > 0) {
+        jc0 = std::max(0, floor_div(t0 - s.lc + s.sc, s.sc));
+        jc1 = std::min(s.n_cmp, std::max(0, floor_div(t1 - s.lc, s.sc) + 1));
+        jc1 = std::max(jc1, jc0);
+    }
+    if ((jb1 > jb0 && !kbar) || (jc1 > jc0 && (!kcmp || !vcmp))) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(kbar) ||
+        !aligned16(kcmp) || !aligned16(vcmp))
+        return NSA_ERR_INVALID_ARG;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    __nv_bfloat16* kb = static_cast<__nv_bfloat16*>(k);
+    __nv_bfloat16* vb = static_cast<__nv_bfloat16*>(v);
+    st = cuda_status(nsa::launch_append_rows(s, static_cast<const __nv_bfloat16*>(k_new),
+                                             static_cast<const __nv_bfloat16*>(v_new), kb, vb, t0, s.Tq, cs));
+    if (st != NSA_OK) return st;
+    return cuda_status(nsa::launch_pool_range(s, kb, vb, kbar, static_cast<__nv_bfloat16*>(kcmp),
+                                              static_cast<__nv_bfloat16*>(vcmp), jb0, jb1, jc0, jc1, cs));
+}
+
+// The pooled inputs the configured scores read: kbar (scaled dot product,
+// probability sums) or the compressed keys (scores from the compressed branch).
+static bool score_inputs_ok(const Shape& s, const void* q, const float* kbar, const void* kcmp) {
+    if (!q) return false;
+    if (s.score_mode == 2) return s.n_cmp == 0 || kcmp != nullptr;
+    return s.nb_full == 0 || kbar != nullptr;
+}
+
+// Scores (scores_out) and/or selected ids (idx) computed from q and the pooled keys.
+static cudaError_t launch_selection(const Shape& s, const void* q, const float* kbar, const void* kcmp,
+                             float* scores_out, int32_t* idx, cudaStream_t cs) {
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    if (s.score_mode != 0)
+        return nsa::launch_score_variant(s, qb, kbar, static_cast<const __nv_bfloat16*>(kcmp), scores_out,
+                                         idx, cs);
+    return nsa::launch_score_topk(s, qb, kbar, nullptr, scores_out, idx, cs);
+}
+
+nsa_status nsa_score_blocks_ex(const nsa_config* cfg, const void* q, const float* kbar, const void* kcmp,
+                               float* scores, void* stream) {
     Shape s;
     nsa_status st = make_shape(cfg, &s);
     if (st != NSA_OK) return st;
     if (!(cfg->flags & NSA_BR_SEL)) return NSA_ERR_INVALID_ARG;
-    if (!q || !scores || (s.nb_full > 0 && !kbar)) return NSA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(kbar) || !aligned16(scores)) return NSA_ERR_INVALID_ARG;
+    if (!scores || !score_inputs_ok(s, q, kbar, kcmp)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kbar) || !aligned16(kcmp) || !aligned16(scores)) return NSA_ERR_INVALID_ARG;
     if (s.Tq == 0) return NSA_OK;
-    return cuda_status(nsa::launch_score_topk(s, static_cast<const __nv_bfloat16*>(q), kbar,
-                                              nullptr, scores, nullptr,
-                                              static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_selection(s, q, kbar, kcmp, scores, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
-nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kbar,
-                           const float* scores, int32_t* idx, void* stream) {
+nsa_status nsa_score_blocks(const nsa_config* cfg, const void* q, const float* kbar, float* scores,
+                            void* stream) {
+    return nsa_score_blocks_ex(cfg, q, kbar, nullptr, scores, stream);
+}
+
+nsa_status nsa_topk_select_ex(const nsa_config* cfg, const void* q, const float* kbar, const void* kcmp,
+                              const float* scores, int32_t* idx, void* stream) {
     Shape s;
     nsa_status st = make_shape(cfg, &s);
     if (st != NSA_OK) return st;
     if (!(cfg->flags & NSA_BR_SEL)) return NSA_ERR_INVALID_ARG;
     if (!idx) return NSA_ERR_INVALID_ARG;
-    if (!scores && (!q || (s.nb_full > 0 && !kbar))) return NSA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(kbar) || !aligned16(scores) || !aligned16(idx))
+    if (!scores && !score_inputs_ok(s, q, kbar, kcmp)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kbar) || !aligned16(kcmp) || !aligned16(scores) || !aligned16(idx))
         return NSA_ERR_INVALID_ARG;
     if (s.Tq == 0) return NSA_OK;
-    return cuda_status(nsa::launch_score_topk(s, static_cast<const __nv_bfloat16*>(q), kbar,
-                                              scores, nullptr, idx,
-                                              static_cast<cudaStream_t>(stream)));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (scores)
+        return cuda_status(nsa::launch_score_topk(s, nullptr, nullptr, scores, nullptr, idx, cs));
+    return cuda_status(launch_selection(s, q, kbar, kcmp, nullptr, idx, cs));
+}
+
+nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kbar,
+                           const float* scores, int32_t* idx, void* stream) {
+    return nsa_topk_select_ex(cfg, q, kbar, nullptr, scores, idx, stream);
 }
 
 nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void* k, const void* v,
@@ -368,7 +442,7 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
     const bool cmp = (cfg->flags & NSA_BR_CMP) != 0;
     if (!q || !k || !v || !out) return NSA_ERR_INVALID_ARG;
     if (cmp && s.n_cmp > 0 && (!kcmp || !vcmp)) return NSA_ERR_INVALID_ARG;
-    if (sel && !idx && s.nb_full > 0 && !kbar) return NSA_ERR_INVALID_ARG;
+    if (sel && !idx && !score_inputs_ok(s, q, kbar, kcmp)) return NSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kbar) || !aligned16(kcmp) ||
         !aligned16(vcmp) || !aligned16(gates) || !aligned16(idx) || !aligned16(out) ||
         !aligned16(workspace))
@@ -382,6 +456,13 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
     }
     if (s.Tq == 0) return NSA_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (sel && idx && (cfg->flags & NSA_DEBUG_CHECKS)) {
+        // validate the caller's ids before any attention kernel reads them
+        int bad = 0;
+        st = cuda_status(nsa::check_idx_rows(s, idx, &bad, cs));
+        if (st != NSA_OK) return st;
+        if (bad > 0) return NSA_ERR_INVALID_ARG;
+    }
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
@@ -397,7 +478,7 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
                                                   reinterpret_cast<float*>(ws + wl.sc_kh),
                                                   reinterpret_cast<float*>(ws + wl.sc_kl), sel_idx, cs));
         else
-            st = cuda_status(nsa::launch_score_topk(s, qb, kbar, nullptr, nullptr, sel_idx, cs));
+            st = cuda_status(launch_selection(s, q, kbar, kcmp, nullptr, sel_idx, cs));
         if (st != NSA_OK) return st;
     }
     const Plan plan = make_plan(s, false, ws ? ws_bytes : 0, wl);
@@ -477,6 +558,11 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
     g_timing.mark("attn_tc", cs);
     return cuda_status(nsa::launch_attn_tc(s, qb, kb, vb, kcb, vcb, gates, sel_idx, nullptr, 1,
                                            nullptr, nullptr, ob, cs));
+}
+
+nsa_status nsa_check_bounded_wait(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1 || limit_ns > 1000000000ull) return NSA_ERR_INVALID_ARG;
+    return cuda_status(nsa::launch_wait_selftest(limit_ns, static_cast<cudaStream_t>(stream)));
 }
 
 nsa_status nsa_timing_enable(int32_t on) {

@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(SNT, 1)
                 uint32_t pass = 0;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float sc = s.scale * __uint_as_float(v[j]);
+                    // forced leading (sink) blocks score +inf: always kept
+                    const float sc = blk0 + j < s.n_sink ? INFINITY : s.scale * __uint_as_float(v[j]);
                     if (blk0 + j < ncand && sc > thr) {
                         pass |= 1u << j;
                         cand[r * 33 + j] = sc;

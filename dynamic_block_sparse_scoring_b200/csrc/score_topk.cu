@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
                     const int jj = bg + 16 * m;
                     const int blk = b0 + jj;
                     const bool valid = (r < nrows) && (jj < nk) && (blk < cr);
-                    const float val = s.scale * acc[i][m];
+                    // forced leading (sink) blocks score +inf: always kept, like the own block
+                    const float val = blk < s.n_sink ? INFINITY : s.scale * acc[i][m];
                     if (MODE == MODE_SCORES) {
                         if (r < nrows && jj < nk) {
                             float w = blk < cr ? val : (blk == cr ? INFINITY : -INFINITY);
@@ -221,7 +222,8 @@ __global__ void __launch_bounds__(ST_NT, 2) score_topk_kernel(Shape s, const __n
                 if (r < nrows && jj < nk) {
                     const int cr = (s.q0 + i0 + r) / s.bs;
                     if (blk < cr)
-                        val = scores_in[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + blk];
+                        val = blk < s.n_sink ? INFINITY   // forced leading blocks
+                                             : scores_in[(((size_t)b * s.Hsel + u) * s.Tq + i0 + r) * s.nb_all + blk];
                 }
                 ss[r * (ST_KC + 1) + jj] = val;
             }
@@ -377,7 +379,10 @@ __global__ void __launch_bounds__(SR_NT, 2)
 #pragma unroll
         for (int rr = 0; rr < RPS; ++rr)
             if (lane == rr) mine = part[rr];
-        if (lane < nr) sc[w0 + c * RPS + lane] = s.scale * mine;
+        if (lane < nr) {
+            const int blk = w0 + c * RPS + lane;
+            sc[blk] = blk < s.n_sink ? INFINITY : s.scale * mine;      // forced leading blocks
+        }
     }
     // a copy that never landed only records an error (the row's ids are then invalid)
     if (!ok) atomicExch(&g_select_status, (int)NSA_ERR_TIMEOUT);
@@ -413,6 +418,237 @@ __global__ void __launch_bounds__(SR_NT, 2)
         if (lane == 0) dst[npast] = cr;
         if (lane > npast && lane < s.topk) dst[lane] = -1;
     }
+}
+
+// Selection-score variants (the probability sums of the unit's heads, or
+// block scores gathered from the compressed branch's probabilities), one CTA
+// per (query row, unit, sequence).  Both need every candidate's score before
+// any is known (a softmax over the candidates), so the row is scored twice:
+// pass 1 finds each head's softmax normaliser (online max and sum per thread,
+// then combined across the CTA), pass 2 writes the normalised scores to
+// shared memory.  The row is then written to `scores` and/or its top-(k-1)
+// selected from shared memory (per-warp lists merged as a tree, as above).
+//   VMODE 1: per head h, p_h(b) = softmax_b(scale q_h . kbar_b) over the
+//            candidates b < c(t); score(b) = sum_h p_h(b).
+//   VMODE 2: per head h, p_h(j) = softmax_j(scale q_h . kcmp_j) over the
+//            visible compressed tokens (j * sc + lc - 1 <= t);
+//            score(b) = sum_j (sum_h p_h(j)) |window_j ∩ block_b| / lc.
+// One thread per candidate (block or compressed token) with the unit's query
+// heads broadcast from shared memory; fp32 throughout.
+constexpr int SV_NT = 256;
+constexpr int SV_NW = SV_NT / 32;
+constexpr int SV_MAXH = 16;
+constexpr int SV_MAXC = 16384;          // candidate blocks / visible compressed tokens per row
+
+template <int VMODE, int D>
+__global__ void __launch_bounds__(SV_NT) score_variant_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
+                                                              const float* __restrict__ kbar,
+                                                              const __nv_bfloat16* __restrict__ kcmp,
+                                                              float* __restrict__ scores_out,
+                                                              int32_t* __restrict__ idx) {
+    extern __shared__ __align__(16) float sv_smem[];
+    float* qs = sv_smem;                          // [nh][D]
+    float* red_m = qs + SV_MAXH * D;              // [NW][MAXH]
+    float* red_l = red_m + SV_NW * SV_MAXH;       // [NW][MAXH]
+    float* hm = red_l + SV_NW * SV_MAXH;          // [MAXH] per-head max
+    float* hl = hm + SV_MAXH;                     // [MAXH] per-head 1 / sum
+    float* sc = hl + SV_MAXH;                     // [SV_MAXC] block scores
+    float* pj = sc + SV_MAXC;                     // [SV_MAXC] compressed-token weights (VMODE 2)
+    unsigned long long* lists = reinterpret_cast<unsigned long long*>(pj + (VMODE == 2 ? SV_MAXC : 0));
+    const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int kvh = s.per_head ? u / s.G : u;
+    const int h0 = s.per_head ? u : u * s.G;
+    const int nh = s.heads_per_unit;
+    const int t = s.q0 + i;
+    const int cr = t / s.bs;
+    const int ncand = min(cr, s.nb_full);
+    // the candidates the softmax runs over: blocks, or visible compressed tokens
+    const int nvis = t >= s.lc - 1 ? min(s.n_cmp, (t - s.lc + 1) / s.sc + 1) : 0;
+    const int nsm = VMODE == 1 ? ncand : nvis;
+    const __nv_bfloat16* qrow = q + (((size_t)b * s.Tq + i) * s.Hq + h0) * D;
+    for (int e = tid; e < nh * D; e += SV_NT) qs[e] = bf2f(qrow[e]);
+    __syncthreads();
+    const float* kb = kbar + (size_t)(b * s.Hkv + kvh) * s.nb_full * D;
+    const __nv_bfloat16* kc = kcmp + (size_t)(b * s.Hkv + kvh) * s.n_cmp * D;
+    // scale * q_h . x for every head of the unit, x = candidate e's key row
+    auto logits = [&](int e, float* lg) {
+#pragma unroll
+        for (int h = 0; h < SV_MAXH; ++h) lg[h] = 0.f;
+        for (int c = 0; c < D; c += 8) {
+            float x[8];
+            if (VMODE == 1) {
+                const float4 a = *reinterpret_cast<const float4*>(kb + (size_t)e * D + c);
+                const float4 bq = *reinterpret_cast<const float4*>(kb + (size_t)e * D + c + 4);
+                x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+                x[4] = bq.x; x[5] = bq.y; x[6] = bq.z; x[7] = bq.w;
+            } else {
+                unpack8(*reinterpret_cast<const uint4*>(kc + (size_t)e * D + c), x);
+            }
+#pragma unroll
+            for (int h = 0; h < SV_MAXH; ++h) {
+                if (h < nh) {
+                    const float4 qa = *reinterpret_cast<const float4*>(qs + h * D + c);
+                    const float4 qb = *reinterpret_cast<const float4*>(qs + h * D + c + 4);
+                    float acc = lg[h];
+                    acc = fmaf(qa.x, x[0], acc); acc = fmaf(qa.y, x[1], acc);
+                    acc = fmaf(qa.z, x[2], acc); acc = fmaf(qa.w, x[3], acc);
+                    acc = fmaf(qb.x, x[4], acc); acc = fmaf(qb.y, x[5], acc);
+                    acc = fmaf(qb.z, x[6], acc); acc = fmaf(qb.w, x[7], acc);
+                    lg[h] = acc;
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < SV_MAXH; ++h) lg[h] *= s.scale;
+    };
+    // pass 1: per-head online max / sum over this thread's candidates, then the CTA's
+    float m[SV_MAXH], l[SV_MAXH];
+#pragma unroll
+    for (int h = 0; h < SV_MAXH; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+    }
+    for (int e = tid; e < nsm; e += SV_NT) {
+        float lg[SV_MAXH];
+        logits(e, lg);
+#pragma unroll
+        for (int h = 0; h < SV_MAXH; ++h) {
+            const float mn = fmaxf(m[h], lg[h]);
+            l[h] = l[h] * expf(m[h] - mn) + expf(lg[h] - mn);
+            m[h] = mn;
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < SV_MAXH; ++h) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
+            const float lo = __shfl_xor_sync(0xffffffffu, l[h], off);
+            const float mn = fmaxf(m[h], mo);
+            l[h] = (m[h] == -INFINITY ? 0.f : l[h] * expf(m[h] - mn)) +
+                   (mo == -INFINITY ? 0.f : lo * expf(mo - mn));
+            m[h] = mn;
+        }
+        if (lane == 0) {
+            red_m[warp * SV_MAXH + h] = m[h];
+            red_l[warp * SV_MAXH + h] = l[h];
+        }
+    }
+    __syncthreads();
+    if (tid < SV_MAXH) {
+        float mm = -INFINITY, ll = 0.f;
+        for (int w = 0; w < SV_NW; ++w) {
+            const float mo = red_m[w * SV_MAXH + tid], lo = red_l[w * SV_MAXH + tid];
+            const float mn = fmaxf(mm, mo);
+            ll = (mm == -INFINITY ? 0.f : ll * expf(mm - mn)) + (mo == -INFINITY ? 0.f : lo * expf(mo - mn));
+            mm = mn;
+        }
+        hm[tid] = mm;
+        hl[tid] = ll > 0.f ? 1.f / ll : 0.f;
+    }
+    __syncthreads();
+    // pass 2: the unit's summed probabilities per candidate
+    float* dst2 = VMODE == 1 ? sc : pj;
+    for (int e = tid; e < nsm; e += SV_NT) {
+        float lg[SV_MAXH];
+        logits(e, lg);
+        float p = 0.f;
+#pragma unroll
+        for (int h = 0; h < SV_MAXH; ++h)
+            if (h < nh) p += expf(lg[h] - hm[h]) * hl[h];
+        dst2[e] = p;
+    }
+    __syncthreads();
+    if (VMODE == 2) {
+        // block b: the compressed tokens whose window [j sc, j sc + lc) overlaps it
+        const float inv_lc = 1.f / (float)s.lc;
+        for (int bb = tid; bb < ncand; bb += SV_NT) {
+            const int lo_t = bb * s.bs, hi_t = (bb + 1) * s.bs;
+            int j0 = lo_t - s.lc + 1;
+            j0 = j0 <= 0 ? 0 : (j0 + s.sc - 1) / s.sc;
+            const int j1 = min(nvis - 1, (hi_t - 1) / s.sc);
+            float acc = 0.f;
+            for (int j = j0; j <= j1; ++j) {
+                const int ov = min(j * s.sc + s.lc, hi_t) - max(j * s.sc, lo_t);
+                if (ov > 0) acc = fmaf(pj[j], (float)ov * inv_lc, acc);
+            }
+            sc[bb] = acc;
+        }
+        __syncthreads();
+    }
+    // forced leading blocks
+    for (int bb = tid; bb < min(s.n_sink, ncand); bb += SV_NT) sc[bb] = INFINITY;
+    __syncthreads();
+    if (scores_out) {
+        float* row = scores_out + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.nb_all;
+        for (int bb = tid; bb < s.nb_all; bb += SV_NT)
+            row[bb] = bb < ncand ? sc[bb] : (bb == cr ? INFINITY : -INFINITY);
+    }
+    if (!idx) return;
+    const int K1 = s.topk - 1;
+    unsigned long long key = 0ull, thr = 0ull;
+    const int per = (ncand + SV_NW - 1) / SV_NW;
+    const int w0 = min(ncand, warp * per), nw = min(ncand, w0 + per) - w0;
+    if (K1 > 0) {
+        for (int e0 = 0; e0 < nw; e0 += 32) {
+            const int e = e0 + lane;
+            const unsigned long long ck = e < nw ? score_key(sc[w0 + e], w0 + e) : 0ull;
+            warp_list_merge(key, thr, ck, K1, lane);
+        }
+    }
+    lists[warp * 32 + lane] = key;
+    __syncthreads();
+    for (int step = 1; step < SV_NW; step <<= 1) {
+        if ((warp & (2 * step - 1)) == 0 && K1 > 0) {
+            warp_list_merge(key, thr, lists[(warp + step) * 32 + lane], K1, lane);
+            lists[warp * 32 + lane] = key;
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+        const bool have = lane < K1 && key != 0ull;
+        const int blk = have ? key_block(key) : 0x7fffffff;
+        const int npast = __popc(__ballot_sync(0xffffffffu, have));
+        int rank = 0;
+        for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, blk, o) < blk) ? 1 : 0;
+        int32_t* dst = idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
+        if (have) dst[rank] = blk;
+        if (lane == 0) dst[npast] = cr;
+        if (lane > npast && lane < s.topk) dst[lane] = -1;
+    }
+}
+
+template <int VMODE, int D>
+void launch_variant(const Shape& s, const __nv_bfloat16* q, const float* kbar, const __nv_bfloat16* kcmp,
+                    float* scores_out, int32_t* idx, cudaStream_t st) {
+    const int smem = (SV_MAXH * D + 2 * SV_NW * SV_MAXH + 2 * SV_MAXH + SV_MAXC * (VMODE == 2 ? 2 : 1)) * 4 +
+                     SV_NW * 32 * 8;
+    cudaFuncSetAttribute(score_variant_kernel<VMODE, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    score_variant_kernel<VMODE, D><<<dim3(s.Tq, s.Hsel, s.B), SV_NT, smem, st>>>(s, q, kbar, kcmp, scores_out,
+                                                                               idx);
+}
+
+bool score_variant_supported(const Shape& s) {
+    return s.heads_per_unit <= SV_MAXH && s.nb_full <= SV_MAXC && s.n_cmp <= SV_MAXC &&
+           (s.dqk == 64 || s.dqk == 128 || s.dqk == 192 || s.dqk == 256);
+}
+
+cudaError_t launch_score_variant(const Shape& s, const __nv_bfloat16* q, const float* kbar,
+                                 const __nv_bfloat16* kcmp, float* scores_out, int32_t* idx,
+                                 cudaStream_t st) {
+#define NSA_SV_CASE(DD)                                                                          \
+    if (s.dqk == DD) {                                                                           \
+        if (s.score_mode == 1) launch_variant<1, DD>(s, q, kbar, kcmp, scores_out, idx, st);    \
+        else launch_variant<2, DD>(s, q, kbar, kcmp, scores_out, idx, st);                      \
+        return cudaGetLastError();                                                               \
+    }
+    NSA_SV_CASE(64)
+    NSA_SV_CASE(128)
+    NSA_SV_CASE(192)
+    NSA_SV_CASE(256)
+#undef NSA_SV_CASE
+    return cudaErrorInvalidValue;
 }
 
 template <int D>

@@ -151,7 +151,49 @@ __global__ void expand_kernel(const int32_t* __restrict__ idx, int32_t* __restri
     }
 }
 
+// Debug check of a caller-supplied idx: a row is valid when its ids lie in
+// [0, c(t)] and below nb_all, are strictly ascending, are followed only by -1,
+// and include the own block c(t).  Reads idx only; counts the invalid rows.
+__device__ int g_idx_bad = 0;
+
+__global__ void check_idx_kernel(const int32_t* __restrict__ idx, size_t rows, int Tq, int q0, int topk,
+                                 int bs, int nb_all) {
+    for (size_t r = (size_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows;
+         r += (size_t)gridDim.x * blockDim.x) {
+        const int c = (q0 + (int)(r % Tq)) / bs;
+        const int32_t* row = idx + r * topk;
+        bool bad = false, pad = false, own = false;
+        int prev = -1;
+        for (int e = 0; e < topk; ++e) {
+            const int v = row[e];
+            if (v == -1) {
+                pad = true;
+                continue;
+            }
+            if (pad || v < 0 || v > c || v >= nb_all || v <= prev) bad = true;
+            own |= v == c;
+            prev = v;
+        }
+        if (bad || !own) atomicAdd(&g_idx_bad, 1);
+    }
+}
+
 }  // namespace
+
+cudaError_t check_idx_rows(const Shape& s, const int32_t* idx, int* bad, cudaStream_t st) {
+    const size_t rows = (size_t)s.B * s.Hsel * s.Tq;
+    static const int zero = 0;
+    *bad = 0;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_idx_bad, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<size_t>((rows + 255) / 256, 148 * 8);
+    check_idx_kernel<<<grid, 256, 0, st>>>(idx, rows, s.Tq, s.q0, s.topk, s.bs, s.nb_all);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbolAsync(bad, g_idx_bad, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(st);
+}
 
 cudaError_t launch_sel_expand(const Shape& s, const int32_t* idx, int32_t* idx_sub, cudaStream_t st) {
     const size_t rows = (size_t)s.B * s.Hsel * s.Tq;

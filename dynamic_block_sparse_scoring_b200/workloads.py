@@ -23,6 +23,9 @@ BR_CMP = 1
 BR_SEL = 2
 BR_WIN = 4
 PER_HEAD_SELECT = 8
+SCORE_PROB = 16
+SCORE_CMP = 32
+SINK_SHIFT = 16
 
 
 @dataclass(frozen=True)
@@ -52,6 +55,9 @@ class Workload:
     gated: bool                 # False: enabled branches are summed with weight 1
     planted: bool = False       # keys from a block-run Gaussian mixture
     seed: int = 0
+    score_mode: str = "dot"     # block scores: "dot" (summed scaled dot products), "prob"
+                                # (summed per-head probabilities), "cmp" (from the compressed branch)
+    sink_blocks: int = 0        # leading blocks always kept
 
     @property
     def scale(self) -> float:
@@ -67,7 +73,9 @@ class Workload:
 
     @property
     def flags(self) -> int:
-        return self.branches | (PER_HEAD_SELECT if self.per_head_select else 0)
+        mode = {"dot": 0, "prob": SCORE_PROB, "cmp": SCORE_CMP}[self.score_mode]
+        return (self.branches | (PER_HEAD_SELECT if self.per_head_select else 0) | mode |
+                (self.sink_blocks << SINK_SHIFT))
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

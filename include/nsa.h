@@ -71,6 +71,21 @@ typedef enum {
 #define NSA_BR_SEL 2u            /* selected-block branch */
 #define NSA_BR_WIN 4u            /* sliding-window branch */
 #define NSA_PER_HEAD_SELECT 8u   /* MoBA: every query head selects its own blocks */
+/* Selection-score variants (default: the scaled dot product with the pooled
+ * block key, summed over the unit's heads).  At most one of the two. */
+#define NSA_SCORE_PROB 16u       /* per head, softmax of the block scores over the row's
+                                    candidates; the unit sums its heads' probabilities */
+#define NSA_SCORE_CMP 32u        /* per head, the compressed branch's softmax weights over the
+                                    visible compressed tokens, gathered to each selection
+                                    block by the share of the token's window inside it; the
+                                    unit sums its heads (needs NSA_BR_CMP) */
+/* Debug mode: nsa_sparse_attn_fwd validates a caller-supplied idx before any
+ * attention kernel reads it (see there). */
+#define NSA_DEBUG_CHECKS 64u
+/* Forced leading blocks ("attention sink"): blocks 0 .. n-1 before the
+ * query's own block are always kept, like the own block; n <= top_k - 1. */
+#define NSA_SINK_SHIFT 16
+#define NSA_SINK_BLOCKS(n) ((uint32_t)(n) << NSA_SINK_SHIFT)
 
 typedef struct {
     int32_t batch;       /* B: independent sequences */
@@ -87,7 +102,7 @@ typedef struct {
     int32_t cmp_block;   /* tokens per compressed token */
     int32_t cmp_stride;  /* distance between compressed tokens */
     float scale;         /* logit scale, normally 1/sqrt(d_qk) */
-    uint32_t flags;      /* NSA_BR_* | NSA_PER_HEAD_SELECT */
+    uint32_t flags;      /* NSA_BR_* | NSA_PER_HEAD_SELECT | NSA_SCORE_* | NSA_SINK_BLOCKS(n) */
 } nsa_config;
 
 /*
@@ -122,6 +137,32 @@ nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, floa
                        void* kcmp, void* vcmp, void* stream);
 
 /*
+ * Incremental cache update for decoding (transcript #94 §6 "Why Sparse
+ * Attention Wins": decoding is memory-bound and costs the KV bytes it reads,
+ * so a step must not re-read the whole cache to refresh its pooled tokens).
+ *
+ * The cache has room for cfg->seqlen_kv tokens per (sequence, KV head); the
+ * call appends cfg->seqlen_q new tokens per sequence at KV positions
+ * [q_pos0, q_pos0 + seqlen_q):
+ *   k_new [B, Hkv, seqlen_q, d_qk] bf16, v_new [B, Hkv, seqlen_q, d_v] bf16
+ * are copied into k and v (layouts as above), then every pooled token that the
+ * new rows complete is recomputed from the cache:
+ *   kbar[j] for each selection block with j*sel_block + sel_block - 1 in the
+ *   new range (NSA_BR_SEL), and kcmp/vcmp[j] for each compressed token with
+ *   j*cmp_stride + cmp_block - 1 in it (NSA_BR_CMP),
+ * with the same arithmetic as nsa_pool_kv, so after appending tokens one call
+ * at a time the pooled tensors equal nsa_pool_kv of the filled cache bit for
+ * bit.  Nothing else is read or written.  A decode step then calls
+ * nsa_topk_select / nsa_sparse_attn_fwd with seqlen_kv = the cache size and
+ * q_pos0 = the newest position: every branch is causal, so cache rows after
+ * the query are never attended, but they must hold finite values (e.g.
+ * zeros), because masked keys still enter the value products with weight 0.
+ * kbar / kcmp / vcmp may be NULL when the call completes none of their tokens.
+ */
+nsa_status nsa_append_kv(const nsa_config* cfg, void* k, void* v, const void* k_new,
+                         const void* v_new, float* kbar, void* kcmp, void* vcmp, void* stream);
+
+/*
  * Block selection scores (transcript #94 §4: one score per query and block;
  * group heads add theirs).  scores[b,u,i,j] =
  *   scale * sum_{h in unit u} q[b,i,h,:] . kbar[b,kv(u),j,:]   for j < c(t),
@@ -130,6 +171,24 @@ nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, floa
  */
 nsa_status nsa_score_blocks(const nsa_config* cfg, const void* q, const float* kbar,
                             float* scores, void* stream);
+
+/*
+ * nsa_score_blocks for every score kind: kcmp [B, Hkv, n_cmp, d_qk] is read
+ * by NSA_SCORE_CMP (kbar may then be NULL); the other kinds read kbar (kcmp
+ * may be NULL).  Variant scores (NSA_SCORE_PROB, NSA_SCORE_CMP):
+ *   PROB: sum over the unit's heads h of softmax_b(scale * q_h . kbar_b),
+ *         the softmax over the row's candidates b < c(t);
+ *   CMP:  sum over h and visible compressed tokens j (j*cmp_stride +
+ *         cmp_block - 1 <= t) of softmax_j(scale * q_h . kcmp_j) * w(j, b),
+ *         w(j, b) = |[j*cmp_stride, j*cmp_stride + cmp_block) ∩ block b| / cmp_block
+ * (transcript #94 §4: the normalised score of §2; the "corner case" of
+ * selection blocks cut differently from the compressed tokens), computed in
+ * fp32.  Forced leading blocks (NSA_SINK_BLOCKS) score +INFINITY like the
+ * own block, in every kind.  Limits: <= 16 heads per unit, <= 16384 blocks
+ * and compressed tokens (NSA_ERR_UNSUPPORTED otherwise).
+ */
+nsa_status nsa_score_blocks_ex(const nsa_config* cfg, const void* q, const float* kbar,
+                               const void* kcmp, float* scores, void* stream);
 
 /*
  * Top-k block sets (transcript #94 §4 Figure 2: keep the k best blocks;
@@ -143,6 +202,15 @@ nsa_status nsa_score_blocks(const nsa_config* cfg, const void* q, const float* k
  */
 nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kbar,
                            const float* scores, int32_t* idx, void* stream);
+
+/*
+ * nsa_topk_select for every score kind (kcmp as in nsa_score_blocks_ex).
+ * With NSA_SINK_BLOCKS(n) the first n blocks before the own block are kept
+ * and the remaining top_k - 1 - n places go to the best other past blocks.
+ * With `scores` given, forced blocks are kept whatever their entries hold.
+ */
+nsa_status nsa_topk_select_ex(const nsa_config* cfg, const void* q, const float* kbar,
+                              const void* kcmp, const float* scores, int32_t* idx, void* stream);
 
 /*
  * Gated sparse attention forward (transcript #94 §4 Figure 2).  For each
@@ -170,6 +238,12 @@ nsa_status nsa_topk_select(const nsa_config* cfg, const void* q, const float* kb
  * kernel over the 64-key sub-blocks of the kept blocks and writes out from
  * their merge directly.
  * kcmp/vcmp are read only with NSA_BR_CMP.
+ * A caller-supplied idx must hold, per row, block ids in [0, c(t)] (and
+ * below nb_all), strictly ascending, then -1 padding, the own block c(t)
+ * included.  These rules are trusted, not checked, unless cfg->flags has
+ * NSA_DEBUG_CHECKS: then a read-only kernel checks every row first, the call
+ * synchronises its stream, and a row that breaks them makes the call return
+ * NSA_ERR_INVALID_ARG with nothing else launched (out untouched).
  */
 nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void* k,
                                const void* v, const float* kbar, const void* kcmp,
@@ -208,6 +282,15 @@ nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, con
  * all work on the current device first.  Not for use inside stream capture.
  */
 nsa_status nsa_get_device_status(int32_t* status);
+
+/*
+ * Self-test of the device-side failure path (the pages have no counterpart):
+ * one warp runs the tensor-core kernels' bounded wait on a barrier that
+ * nothing ever completes, gives up after limit_ns (1 .. 1e9 ns) and records
+ * NSA_ERR_TIMEOUT in the same status word, which nsa_get_device_status then
+ * returns.  The GPU context stays usable.  Asynchronous on `stream`.
+ */
+nsa_status nsa_check_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* Organisations of nsa_sparse_attn_fwd (same results, different speed). */
 #define NSA_PATH_ROWWISE 0       /* shapes outside the tensor-core kernels' limits */

@@ -39,7 +39,19 @@ def oracle_cfg(wl: Workload) -> dict:
     return dict(h_q=wl.h_q, h_kv=wl.h_kv, d_qk=wl.d_qk, d_v=wl.d_v, sel_block=wl.sel_block,
                 top_k=wl.top_k, window=wl.window, cmp_block=wl.cmp_block,
                 cmp_stride=wl.cmp_stride, scale=wl.scale, branches=wl.branches,
-                per_head_select=wl.per_head_select, gated=wl.gated)
+                per_head_select=wl.per_head_select, gated=wl.gated, score_mode=wl.score_mode,
+                sink_blocks=wl.sink_blocks)
+
+
+def oracle_selection(wl: Workload, q: np.ndarray, pos: np.ndarray, K: np.ndarray, V=None):
+    """(scores, idx, gap) of the oracle's selection for query rows q [R, Hq, d] at `pos`."""
+    nb_all = -(-wl.seqlen_kv // wl.sel_block)
+    pooled = {"Kbar": O.pool_block_keys(K, wl.sel_block)}
+    if wl.score_mode == "cmp":
+        pooled["Kc"] = O.compress(K, wl.cmp_block, wl.cmp_stride)
+    s = O.selection_scores(oracle_cfg(wl), q, pos, pooled, nb_all)
+    idx, gap = O.select_blocks(s, pos, wl.sel_block, wl.top_k, wl.sink_blocks)
+    return s, idx, gap
 
 
 class GpuRun:
@@ -56,7 +68,8 @@ class GpuRun:
         if wl.branches & abi.NSA_BR_SEL:
             self.idx = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, wl.top_k, dtype=torch.int32,
                                    device="cuda")
-            abi.nsa_topk_select(self.cfg, self.x["q"], self.pooled["kbar"], None, self.idx)
+            abi.nsa_topk_select_ex(self.cfg, self.x["q"], self.pooled["kbar"], self.pooled["kcmp"],
+                                   None, self.idx)
         # the forward with the selection inside the call; it leaves its selected ids at
         # the start of the workspace
         ws = torch.empty(max(abi.nsa_workspace_size(self.cfg), 1), dtype=torch.uint8, device="cuda")
@@ -95,7 +108,7 @@ def tie_margin(ora_idx: np.ndarray, scores: np.ndarray, rows=None) -> np.ndarray
 
 
 def check_idx(gpu_idx: np.ndarray, ora_idx: np.ndarray, gap: np.ndarray, scores: np.ndarray,
-              positions: np.ndarray, sel_block: int, top_k: int):
+              positions: np.ndarray, sel_block: int, top_k: int, n_sink: int = 0):
     """gpu_idx/ora_idx [U, R, k], gap [U, R], scores [U, R, nb] (oracle, -inf non-candidates)."""
     differ = (gpu_idx != ora_idx).any(axis=-1)
     margin = tie_margin(ora_idx, scores, np.nonzero(differ))
@@ -117,8 +130,11 @@ def check_idx(gpu_idx: np.ndarray, ora_idx: np.ndarray, gap: np.ndarray, scores:
         got = [int(b) for b in gpu_idx[u, r] if b >= 0]
         # strictly ascending (no repeated id), own block kept, right size
         assert got == sorted(set(got)) and c in got and len(got) == min(top_k, c + 1)
-        past = [b for b in got if b != c]
-        dropped = [b for b in range(c) if b not in past]
+        # forced leading blocks are kept; the scored places compare like a plain top-k
+        forced = list(range(min(n_sink, c)))
+        assert all(b in got for b in forced)
+        past = [b for b in got if b != c and b not in forced]
+        dropped = [b for b in range(c) if b not in past and b not in forced]
         if past and dropped:
             s = scores[u, r]
             assert min(s[past]) >= max(s[dropped]) - margin[u, r]
@@ -139,19 +155,17 @@ def check_selection_all_rows(run: "GpuRun", chunk: int = 2048):
 
     Returns the number of rows (per unit) resolved differently at a near-tie."""
     wl = run.wl
-    nb_all = -(-wl.seqlen_kv // wl.sel_block)
     ties = 0
     for b in range(wl.batch):
-        Kbar = O.pool_block_keys(f64(run.x["k"][b]), wl.sel_block)
+        K = f64(run.x["k"][b])
         for r0 in range(0, wl.seqlen_q, chunk):
             rows = np.arange(r0, min(wl.seqlen_q, r0 + chunk))
             pos = rows + wl.q_pos0
             rows_t = torch.as_tensor(rows, device=run.x["q"].device)
             q = f64(run.x["q"][b].index_select(0, rows_t))
-            s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
-                               wl.per_head_select, nb_all)
-            ora_idx, gap = O.select_blocks(s, pos, wl.sel_block, wl.top_k)
+            s, ora_idx, gap = oracle_selection(wl, q, pos, K, None)
             for got in (run.idx, run.idx_fwd):
                 gpu_idx = got[b].index_select(1, rows_t).cpu().numpy()
-                ties += check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
+                ties += check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k,
+                                  wl.sink_blocks)
     return ties

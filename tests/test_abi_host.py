@@ -92,7 +92,7 @@ def test_workspace_sizes(abi):
     (dict(seqlen_kv=0), 1),
     (dict(q_pos0=1), 1),               # q_pos0 + Tq > Tkv
     (dict(flags=0), 1),
-    (dict(flags=64 | 7), 1),
+    (dict(flags=128 | 7), 1),          # unknown flag bit
     (dict(top_k=0), 1),
     (dict(window=0), 1),
     (dict(cmp_stride=0), 1),
@@ -174,3 +174,48 @@ def test_sub_block_path_conditions(abi):
     # the workspace holds one partial row per sub-block slot
     small = abi.nsa_workspace_size(abi.config(moba.with_(sel_block=64, top_k=3)))
     assert abi.nsa_workspace_size(abi.config(moba)) > 4 * small
+
+
+def test_append_kv_rejects_bad_arguments_on_host(abi):
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
+    wl = WORKLOADS["decode64x64k"]
+    fake = 1 << 20
+    L = abi.lib
+    ok = abi.config(wl, seqlen_q=1, q_pos0=63)          # completes block 0 and compressed token 2
+    # no new token, past the cache, null cache or source
+    assert L.nsa_append_kv(abi.config(wl, seqlen_q=0, q_pos0=10), fake, fake, fake, fake, fake, fake,
+                           fake, None) == 1
+    assert L.nsa_append_kv(abi.config(wl, seqlen_q=2, q_pos0=wl.seqlen_kv - 1), fake, fake, fake, fake,
+                           fake, fake, fake, None) == 1
+    assert L.nsa_append_kv(ok, None, fake, fake, fake, fake, fake, fake, None) == 1
+    assert L.nsa_append_kv(ok, fake, fake, None, fake, fake, fake, fake, None) == 1
+    # a completed block needs kbar, a completed compressed token needs kcmp and vcmp
+    assert L.nsa_append_kv(ok, fake, fake, fake, fake, None, fake, fake, None) == 1
+    assert L.nsa_append_kv(ok, fake, fake, fake, fake, fake, None, fake, None) == 1
+    # misaligned
+    assert L.nsa_append_kv(ok, fake + 2, fake, fake, fake, fake, fake, fake, None) == 1
+
+
+def test_bounded_wait_self_test_rejects_bad_limits_on_host(abi):
+    assert abi.lib.nsa_check_bounded_wait(0, None) == 1
+    assert abi.lib.nsa_check_bounded_wait(2_000_000_000, None) == 1
+
+
+def test_score_variant_flags_validated_on_host(abi):
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
+    wl = WORKLOADS["tiny"]
+    n = ctypes.c_size_t(0)
+    L = abi.lib
+    both = abi.config(wl, flags=wl.flags | abi.NSA_SCORE_PROB | abi.NSA_SCORE_CMP)
+    assert L.nsa_workspace_size(ctypes.byref(both), ctypes.byref(n)) == 1
+    no_cmp = abi.config(wl, flags=abi.NSA_BR_SEL | abi.NSA_SCORE_CMP)       # needs the compressed branch
+    assert L.nsa_workspace_size(ctypes.byref(no_cmp), ctypes.byref(n)) == 1
+    too_many_sinks = abi.config(wl, flags=wl.flags | (wl.top_k << abi.NSA_SINK_SHIFT))
+    assert L.nsa_workspace_size(ctypes.byref(too_many_sinks), ctypes.byref(n)) == 1
+    ok = abi.config(wl, flags=wl.flags | abi.NSA_SCORE_PROB | ((wl.top_k - 1) << abi.NSA_SINK_SHIFT))
+    assert L.nsa_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == 0
+    # the compressed-branch scores read kcmp: the plain entry points cannot serve them
+    cmp_mode = abi.config(wl, flags=wl.flags | abi.NSA_SCORE_CMP)
+    fake = 1 << 20
+    assert L.nsa_score_blocks(ctypes.byref(cmp_mode), fake, fake, fake, None) == 1
+    assert L.nsa_topk_select(ctypes.byref(cmp_mode), fake, fake, None, fake, None) == 1

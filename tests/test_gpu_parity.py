@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 from dynamic_block_sparse_scoring_b200 import abi
 from tests.parity import (GpuRun, check_idx, check_out, check_selection_all_rows, f64,
-                          OUT_MAX_ABS, OUT_MEAN_ABS, SCORE_ATOL, SCORE_RTOL)
+                          oracle_selection, OUT_MAX_ABS, OUT_MEAN_ABS, SCORE_ATOL, SCORE_RTOL)
 
 TINY = WORKLOADS["tiny"]
 
@@ -87,6 +87,27 @@ EDGE = {
                                             q_pos0=1700, h_q=16, h_kv=1),
     "bm_batch2": WORKLOADS["nsa64k"].with_(name="bm_batch2", batch=2, seqlen_q=700, seqlen_kv=700,
                                            h_q=32, h_kv=2, d_qk=64, d_v=64),
+    # selection-score variants and forced leading blocks, on every selection kernel:
+    # the variant kernel (prefill, decode, block-major), the FFMA / tensor-core / few-row
+    # fused selections with sinks, per-head selection with sinks
+    "prob_tiny": TINY.with_(name="prob_tiny", score_mode="prob"),
+    "cmp_tiny": TINY.with_(name="cmp_tiny", score_mode="cmp", cmp_block=32, cmp_stride=16),
+    "sinks_tiny": TINY.with_(name="sinks_tiny", sink_blocks=2),
+    "prob_sinks_nsa_small": WORKLOADS["nsa64k"].with_(name="prob_sinks_nsa_small", seqlen_q=2048,
+                                                      seqlen_kv=2048, h_q=16, h_kv=1,
+                                                      score_mode="prob", sink_blocks=1),
+    "cmp_nsa_small": WORKLOADS["nsa64k"].with_(name="cmp_nsa_small", seqlen_q=2048, seqlen_kv=2048,
+                                               h_q=16, h_kv=1, score_mode="cmp"),
+    "sinks_nsa_small": WORKLOADS["nsa64k"].with_(name="sinks_nsa_small", seqlen_q=2048,
+                                                 seqlen_kv=2048, h_q=16, h_kv=1, sink_blocks=3),
+    "dec_sinks": WORKLOADS["decode64x64k"].with_(name="dec_sinks", batch=2, seqlen_kv=3000,
+                                                 q_pos0=2999, sink_blocks=2),
+    "dec_prob": WORKLOADS["decode64x64k"].with_(name="dec_prob", batch=2, seqlen_kv=3000,
+                                                q_pos0=2999, score_mode="prob"),
+    "dec_cmp": WORKLOADS["decode64x64k"].with_(name="dec_cmp", batch=2, seqlen_kv=3000,
+                                               q_pos0=2999, score_mode="cmp"),
+    "moba_small_sinks": WORKLOADS["moba32k"].with_(name="moba_small_sinks", seqlen_q=4096,
+                                                   seqlen_kv=4096, h_q=4, h_kv=4, sink_blocks=1),
 }
 
 
@@ -101,16 +122,12 @@ def compare_run(run: GpuRun, rows_per_seq, seqs=None):
             K = f64(run.x["k"][b])
             rows_t = torch.as_tensor(rows, device="cuda")
             q = f64(run.x["q"][b].index_select(0, rows_t))
-            Kbar = O.pool_block_keys(K, wl.sel_block)
-            nb_all = -(-wl.seqlen_kv // wl.sel_block)
-            s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
-                               wl.per_head_select, nb_all)
-            ora_idx, gap = O.select_blocks(s, pos, wl.sel_block, wl.top_k)
+            s, ora_idx, gap = oracle_selection(wl, q, pos, K)
             # the stand-alone selection and the one inside the forward call
             gpu_idx = run.idx[b].index_select(1, rows_t).cpu().numpy()
-            check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
+            check_idx(gpu_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k, wl.sink_blocks)
             fwd_idx = run.idx_fwd[b].index_select(1, rows_t).cpu().numpy()
-            check_idx(fwd_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k)
+            check_idx(fwd_idx, ora_idx, gap, s, pos, wl.sel_block, wl.top_k, wl.sink_blocks)
             idx_for_out = fwd_idx
         else:
             idx_for_out = None
@@ -151,14 +168,15 @@ def test_pool_kv_matches_oracle():
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged_77", "gqa_per_head", "chunked_prefill",
-                                  "nsa_small"])
+                                  "nsa_small", "prob_tiny", "cmp_tiny", "sinks_tiny",
+                                  "prob_sinks_nsa_small"])
 def test_materialised_scores_and_select_from_scores(name):
     wl = EDGE[name]
     run = GpuRun(wl)
     cfg = run.cfg
     nb_all = -(-wl.seqlen_kv // wl.sel_block)
     scores = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, nb_all, device="cuda")
-    abi.nsa_score_blocks(cfg, run.x["q"], run.pooled["kbar"], scores)
+    abi.nsa_score_blocks_ex(cfg, run.x["q"], run.pooled["kbar"], run.pooled["kcmp"], scores)
     idx2 = torch.empty_like(run.idx)
     abi.nsa_topk_select(cfg, None, None, scores, idx2)
     torch.cuda.synchronize()
@@ -167,14 +185,14 @@ def test_materialised_scores_and_select_from_scores(name):
     pos = np.arange(wl.seqlen_q) + wl.q_pos0
     for b in range(wl.batch):
         q = f64(run.x["q"][b])
-        Kbar = O.pool_block_keys(f64(run.x["k"][b]), wl.sel_block)
-        s = O.block_scores(q, pos, Kbar, wl.h_q, wl.h_kv, wl.sel_block, wl.scale,
-                           wl.per_head_select, nb_all)
+        s, _, _ = oracle_selection(wl, q, pos, f64(run.x["k"][b]))
         got = scores[b].cpu().double().numpy()
         cur = pos // wl.sel_block
         for r in range(wl.seqlen_q):
             c = cur[r]
-            np.testing.assert_allclose(got[:, r, :c], s[:, r, :c], rtol=SCORE_RTOL,
+            ns = min(wl.sink_blocks, c)
+            assert np.all(got[:, r, :ns] == np.inf)          # forced leading blocks
+            np.testing.assert_allclose(got[:, r, ns:c], s[:, r, ns:c], rtol=SCORE_RTOL,
                                        atol=SCORE_ATOL)
             assert np.all(got[:, r, c] == np.inf)
             assert np.all(got[:, r, c + 1:] == -np.inf)
