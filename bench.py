@@ -705,7 +705,7 @@ def run_ours(args):
     decode = None if args.no_decode else run_decode(world, args.steps, args.warmup)
     others = {}
     if not args.no_configs:
-        for name in ("tiny", "moba32k", "nsa128k_planted"):
+        for name in ("tiny", "moba32k", "moba32k_full", "nsa128k_planted"):
             if name != wl.name:
                 others[name] = run_config(name, min(args.steps, 5), args.warmup, world, rank)
     cpu = cpu_baseline(wl, x_cpu) if x_cpu is not None else None
@@ -768,7 +768,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
-                    help="skip the other prefill workloads (tiny, moba32k, nsa128k_planted)")
+                    help="skip the other prefill workloads (tiny, moba32k, moba32k_full, "
+                         "nsa128k_planted)")
     ap.add_argument("--seqlen", type=int, default=0, help="override the prefill length (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling)")
     args = ap.parse_args()

@@ -62,7 +62,7 @@ struct ItemMeta {
     int new_block;      // first item on this K/V stage load
     int last_of_block;  // last item using this K/V stage load
     int pad[2];
-    int tok[MT];        // query * 32 + slot
+    int tok[MT];        // query * SEL_SLOTS + slot
 };
 
 struct BmArgs {
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int e = lane; e < m.n * L::QC; e += 32) {
                         const int tt = e / L::QC, c = e % L::QC;
                         tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
-                                             &map_qg, bar.q_full(qs), 64 * c, h0, m.tok[tt] >> 5, b,
+                                             &map_qg, bar.q_full(qs), 64 * c, h0, pair_query(m.tok[tt]), b,
                                              q_policy);
                     }
                 } else {
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         int r[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            r[k] = qrow0 + (toks[min(4 * g4 + k, m.n - 1)] >> 5) * a.s.Hq;
+                            r[k] = qrow0 + pair_query(toks[min(4 * g4 + k, m.n - 1)]) * a.s.Hq;
                         tc::tma_gather4_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + 4 * g4 * 128, &map_qg,
                                              bar.q_full(qs), 64 * c, r[0], r[1], r[2], r[3], q_policy);
                     }
@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!valid) break;
             const bool row_valid = tt < n;
             const int j = lidx % nb_all;
-            const int t = a.s.q0 + (tokr >> 5);
+            const int t = a.s.q0 + pair_query(tokr);
             const int sb = li & 1;
             if (!bm_warp_wait(bar.s_full(sb), (li >> 1) & 1, abort_flag)) {
                 ok = false;
@@ -591,12 +591,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const bool row_valid = tt < n;
             const int bu = (lidx / nb_all) % bhsel;
             const float m = row_m[sb * BM + r], l = row_l[sb * BM + r];
-            const size_t prow = (((size_t)bu * a.s.Tq + (tokr >> 5)) * a.s.topk + (tokr & 31)) * a.hpt + hl;
+            const size_t prow = (((size_t)bu * a.s.Tq + pair_query(tokr)) * a.s.topk + pair_slot(tokr)) * a.hpt + hl;
             // first partial row of each query this lane stores (issuer warp)
             int prow_q[NG];
 #pragma unroll
             for (int g = 0; g < NG; ++g)
-                prow_q[g] = (int)((((size_t)bu * a.s.Tq + (tok_lane[g] >> 5)) * a.s.topk + (tok_lane[g] & 31)) * a.hpt);
+                prow_q[g] = (int)((((size_t)bu * a.s.Tq + pair_query(tok_lane[g])) * a.s.topk + pair_slot(tok_lane[g])) *
+                                  a.hpt);
 #pragma unroll 1
             for (int c = 0; c < DV; c += 64, ++halves) {
                 uint32_t o[64];
@@ -743,10 +744,11 @@ bool sel_bm_supported(const Shape& s) {
     if (s.dv != 64 && s.dv != 128) return false;
     if (s.bs != BLK) return false;
     const int hpt = s.heads_per_unit;
-    // a slot is 5 bits of a list entry; the merge of groups takes up to 16 slots
+    // a slot is SEL_SLOT_BITS of a list entry; the merge of groups takes up to 16 slots
     // (one head per query: q rows are gathered by a 32-bit row index)
     const bool shape_ok = ((hpt == 8 || hpt == 16) && s.topk <= 16) ||
-                          (hpt == 1 && s.topk <= 32 && (size_t)s.B * s.Tq * s.Hq < (size_t(1) << 31));
+                          (hpt == 1 && s.topk <= SEL_SLOTS && (size_t)s.B * s.Tq * s.Hq < (size_t(1) << 31));
+    if (s.Tq >= (1 << (31 - SEL_SLOT_BITS))) return false;       // list entries are int32
     // partial rows are addressed by 32-bit TMA coordinates
     return shape_ok && sel_partial_rows(s) < (size_t(1) << 31);
 }

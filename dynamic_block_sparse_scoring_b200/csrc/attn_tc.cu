@@ -949,7 +949,11 @@ bool attn_tc_supported(const Shape& s) {
     if (s.dqk != 64 && s.dqk != 128 && s.dqk != 192) return false;
     if (s.dv != 64 && s.dv != 128) return false;
     const int hpt = s.heads_per_unit;
-    if (hpt < 4 || hpt > 16 || (BM % hpt) != 0) return false;   // tokens per tile <= 32
+    if (hpt > 16 || (BM % hpt) != 0) return false;
+    // the selected branch's per-segment membership masks hold 32 tokens per tile;
+    // the window and compressed branches alone take one or two heads per unit too
+    // (up to 128 tokens per tile: MHA, or full causal attention as a window >= Tkv)
+    if ((s.flags & NSA_BR_SEL) && hpt < 4) return false;
     if ((s.flags & NSA_BR_SEL) && (s.bs % SEG != 0)) return false;
     if ((s.flags & NSA_BR_SEL) && (BM / hpt) * s.topk > MAX_UNION / 2) return false;
     return true;

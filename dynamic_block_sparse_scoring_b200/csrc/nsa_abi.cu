@@ -116,7 +116,7 @@ Shape sub_block_shape(const Shape& s) {
 bool use_sub_block_major(const Shape& s) {
     if (!(s.flags & NSA_BR_SEL) || (s.flags & (NSA_BR_CMP | NSA_BR_WIN))) return false;
     if (s.heads_per_unit != 1 || s.bs % 64 != 0 || s.Tq < 256) return false;
-    if (s.topk * (s.bs / 64) > 32) return false;
+    if (s.topk * (s.bs / 64) > nsa::SEL_SLOTS) return false;
     return nsa::sel_bm_supported(sub_block_shape(s));
 }
 

@@ -113,7 +113,7 @@ __global__ void fill_pairs_kernel(const int32_t* __restrict__ idx, int32_t* __re
         const int rem = (int)(e % ((size_t)Tq * topk));
         const int qi = rem / topk, slot = rem % topk;
         const int pos = atomicAdd(&cursor[list_of(e, blk, BHsel, Tq, topk, nb_all)], 1);
-        list[pos] = qi * 32 + slot;
+        list[pos] = qi * SEL_SLOTS + slot;
     }
 }
 

@@ -14,7 +14,7 @@ struct SelIndex {
     int32_t* off;       // [L + 1] list offsets (exclusive scan); off[L] = pairs
     int32_t* item_off;  // [L + 1] first work item of each list; item_off[L] = items
     int32_t* cursor;    // [L] fill cursors
-    int32_t* list;      // [pairs] query * 32 + slot, grouped by list
+    int32_t* list;      // [pairs] query * SEL_SLOTS + slot, grouped by list
     int4* items;        // [items] (list id, first pair, pair count, 0)
 };
 
@@ -26,6 +26,12 @@ struct SelIndex {
 // (block-major kernel 8.0 ms against 8.4 at 2048, 9.4 at 1024, 7.9 at one
 // chunk whose index build costs 0.3 ms more).
 constexpr int SEL_CHUNK = 8192;
+// A list entry is query * SEL_SLOTS + slot: up to 64 kept (sub-)blocks per query
+// row, queries below 2^25.
+constexpr int SEL_SLOT_BITS = 6;
+constexpr int SEL_SLOTS = 1 << SEL_SLOT_BITS;
+__host__ __device__ __forceinline__ int pair_query(int e) { return e >> SEL_SLOT_BITS; }
+__host__ __device__ __forceinline__ int pair_slot(int e) { return e & (SEL_SLOTS - 1); }
 inline int sel_chunks(const Shape& s) { return (s.Tq + SEL_CHUNK - 1) / SEL_CHUNK; }
 inline size_t sel_lists_per_chunk(const Shape& s) { return (size_t)s.B * s.Hsel * s.nb_all; }
 

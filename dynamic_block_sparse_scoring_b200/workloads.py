@@ -88,7 +88,8 @@ def _prefill(name, T, **kw):
 # The five workloads.  Sizes are the ones the method is discussed at: a tiny
 # single-group case, MoBA-style per-head selection, NSA prefill at 64k, NSA
 # decode against 64 caches of 64k tokens, and a 128k prefill whose keys carry
-# planted block structure so that the top-k is far from uniform.
+# planted block structure so that the top-k is far from uniform; plus the
+# full-attention layers of MoBA's hybrid at the MoBA shapes.
 WORKLOADS = {
     "tiny": _prefill("tiny", 1024, h_q=4, h_kv=1, d_qk=64, d_v=64, sel_block=64, top_k=4,
                      window=128, cmp_block=32, cmp_stride=32,
@@ -104,6 +105,11 @@ WORKLOADS = {
                              top_k=16, window=512, cmp_block=32, cmp_stride=16,
                              branches=BR_CMP | BR_SEL | BR_WIN, per_head_select=False,
                              gated=True),
+    # MoBA's hybrid: the layers that switch back to full attention (same shapes as
+    # moba32k), i.e. dense causal attention, run as a window covering the whole cache
+    "moba32k_full": _prefill("moba32k_full", 32768, h_q=16, h_kv=16, d_qk=128, d_v=128,
+                             sel_block=512, top_k=3, window=32768, cmp_block=0, cmp_stride=0,
+                             branches=BR_WIN, per_head_select=False, gated=False),
     "nsa128k_planted": _prefill("nsa128k_planted", 131072, h_q=64, h_kv=4, d_qk=192, d_v=128,
                                 sel_block=64, top_k=16, window=512, cmp_block=32, cmp_stride=16,
                                 branches=BR_CMP | BR_SEL | BR_WIN, per_head_select=False,

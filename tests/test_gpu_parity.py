@@ -108,6 +108,22 @@ EDGE = {
                                                q_pos0=2999, score_mode="cmp"),
     "moba_small_sinks": WORKLOADS["moba32k"].with_(name="moba_small_sinks", seqlen_q=4096,
                                                    seqlen_kv=4096, h_q=4, h_kv=4, sink_blocks=1),
+    # per-head selection on the sub-block path with up to 64 sub-blocks per query
+    # (1024-key blocks; 512-key blocks x top-8; 256-key blocks x top-16)
+    "sub_bs1024": WORKLOADS["moba32k"].with_(name="sub_bs1024", seqlen_q=3000, seqlen_kv=3000,
+                                             h_q=2, h_kv=2, sel_block=1024, top_k=3),
+    "sub_bs512_top8": WORKLOADS["moba32k"].with_(name="sub_bs512_top8", seqlen_q=2000,
+                                                 seqlen_kv=5000, q_pos0=3000, h_q=2, h_kv=2,
+                                                 top_k=8),
+    "sub_bs256_top16": WORKLOADS["moba32k"].with_(name="sub_bs256_top16", seqlen_q=4200,
+                                                  seqlen_kv=4200, h_q=2, h_kv=1, sel_block=256,
+                                                  top_k=16),
+    # full causal attention (MoBA's hybrid layers) on the tensor cores with one head per
+    # unit, and window + compressed branches with two heads per unit
+    "full_attn_mha": WORKLOADS["moba32k_full"].with_(name="full_attn_mha", seqlen_q=2000,
+                                                     seqlen_kv=2000, window=2000, h_q=4, h_kv=4),
+    "win_cmp_g2": TINY.with_(name="win_cmp_g2", seqlen_q=900, seqlen_kv=900, h_q=4, h_kv=2,
+                             branches=BR_CMP | BR_WIN),
 }
 
 
@@ -198,6 +214,17 @@ def test_materialised_scores_and_select_from_scores(name):
             assert np.all(got[:, r, c + 1:] == -np.inf)
 
 
+def test_full_attention_layer_is_dense_causal_attention():
+    """MoBA's full-attention layers (a window covering the cache) against library SDPA (fp32)."""
+    wl = EDGE["full_attn_mha"]
+    run = GpuRun(wl)
+    assert abi.nsa_attn_plan(run.cfg, False, abi.nsa_workspace_size(run.cfg))[0] in ("query-major", "split-k")
+    q = run.x["q"][0].float().permute(1, 0, 2)
+    ref = F.scaled_dot_product_attention(q, run.x["k"][0].float(), run.x["v"][0].float(),
+                                         is_causal=True, scale=wl.scale).permute(1, 0, 2)
+    check_out(run.out[0].double().cpu().numpy(), ref.double().cpu().numpy(), "full attention")
+
+
 def test_every_block_kept_is_dense_causal_attention():
     """Library SDPA (fp32) as an independent check of the special case."""
     wl = EDGE["every_block"].with_(h_q=8, h_kv=2)
@@ -209,7 +236,7 @@ def test_every_block_kept_is_dense_causal_attention():
     check_out(run.out[0].double().cpu().numpy(), ref.double().cpu().numpy(), "dense causal")
 
 
-SAMPLED = {name: WORKLOADS[name] for name in ["moba32k", "nsa64k", "nsa128k_planted"]}
+SAMPLED = {name: WORKLOADS[name] for name in ["moba32k", "nsa64k", "nsa128k_planted", "moba32k_full"]}
 # block-major work items cross the 8192-query chunk boundary (ragged second chunk)
 SAMPLED["bm_two_chunks"] = WORKLOADS["nsa64k"].with_(name="bm_two_chunks", seqlen_q=9000,
                                                      seqlen_kv=9000, h_q=16, h_kv=1)
@@ -220,12 +247,15 @@ def test_full_size_prefill_sampled_rows(name):
     """Selected ids on every row against the oracle; outputs on sampled rows."""
     wl = SAMPLED[name]
     run = GpuRun(wl)
-    check_selection_all_rows(run)
+    if wl.branches & BR_SEL:
+        check_selection_all_rows(run)
     T = wl.seqlen_q
     extra = [wl.sel_block - 1, wl.sel_block, wl.sel_block + 1, 511, 512, 513, T // 2, T - 2]
     extra += [r for r in (8190, 8191, 8192, 8193) if r < T]
     rows = row_sample(T, stride=max(1, T // 384), head=128, extra=extra)
     compare_run(run, rows)
+    if not wl.branches & BR_SEL:
+        return
     # every row of both selections: structural invariants
     for idx in (run.idx[0], run.idx_fwd[0]):
         t = torch.arange(T, device="cuda") + wl.q_pos0
