@@ -374,3 +374,87 @@ def nsa_rows(cfg, q_rows, positions, K, V, gates_rows=None, idx=None, pooled=Non
                 ks = window_keys(t, window)
                 out[r, heads] += weight(2) * softmax_attention(q, K[hk, ks], V[hk, ks], scale)
     return out, idx, gap
+
+
+# ---------------------------------------------------------------------------
+# Backward pass
+# ---------------------------------------------------------------------------
+
+def softmax_attention_grad(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                           d_o: np.ndarray):
+    """Gradients of o = softmax(scale * q k^T) v with respect to q, k and v.
+
+    Transcript #94, §2: the output is the softmax-weighted sum of the values.
+    The chain rule through it, with P the weights and dO the output gradient:
+    dV = P^T dO; dP = dO V^T; dS = P * (dP - rowsum(dP * P)) (the softmax
+    Jacobian); dq = scale * dS k; dk = scale * dS^T q.  q [n, d], k [m, d],
+    v [m, dv], d_o [n, dv]; no keys: zero gradients.
+    """
+    if k.shape[0] == 0:
+        return np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    logits = scale * (q @ k.T)
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    dv = p.T @ d_o
+    dp = d_o @ v.T
+    ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def nsa_rows_backward(cfg, q_rows, positions, K, V, gates_rows, idx, d_out):
+    """Gradients of the gated output of ``nsa_rows`` for fixed selected blocks.
+
+    The top-k choice is discrete and passes no gradient (transcript #94, §6:
+    the compressed branch is what carries gradient to the block
+    representations), so ``idx`` [n_units, R, top_k] is an input.  The
+    compressed tokens are means of K/V windows (§4, Figure 2; mean pooling,
+    §7), so their gradients reach every token of the window with weight
+    1 / cmp_block.  Returns (dq [R, H_q, d_qk], dK [H_kv, T_kv, d_qk],
+    dV [H_kv, T_kv, d_v], dg [R, H_q, 3] or None) for the loss
+    sum(d_out * out), d_out [R, H_q, d_v].
+    """
+    get = (lambda name: cfg[name]) if isinstance(cfg, dict) else (lambda name: getattr(cfg, name))
+    h_q, h_kv = get("h_q"), get("h_kv")
+    sel_block, window = get("sel_block"), get("window")
+    cmp_block, cmp_stride = get("cmp_block"), get("cmp_stride")
+    scale, branches, per_head = get("scale"), get("branches"), bool(get("per_head_select"))
+    positions = np.asarray(positions, dtype=np.int64)
+    units = selection_units(h_q, h_kv, per_head)
+    R = q_rows.shape[0]
+    dq = np.zeros_like(q_rows)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dg = None if gates_rows is None else np.zeros((R, h_q, 3))
+    if branches & 1:
+        Kc, Vc = compress(K, cmp_block, cmp_stride), compress(V, cmp_block, cmp_stride)
+        dKc, dVc = np.zeros_like(Kc), np.zeros_like(Vc)
+        n_cmp = Kc.shape[1]
+    for r in range(R):
+        t = int(positions[r])
+        for u, (hk, heads) in enumerate(units):
+            q = q_rows[r, heads, :]
+            for br in (0, 1, 2):
+                if not branches & (1 << br):
+                    continue
+                if br == 0:
+                    js = compressed_keys(t, n_cmp, cmp_block, cmp_stride)
+                    kk, vv = Kc[hk, js], Vc[hk, js]
+                else:
+                    ks = selected_keys(idx[u, r], t, sel_block) if br == 1 else window_keys(t, window)
+                    kk, vv = K[hk, ks], V[hk, ks]
+                g = gates_rows[r, heads, br] if gates_rows is not None else np.ones(len(heads))
+                if dg is not None:
+                    dg[r, heads, br] = (d_out[r, heads] * softmax_attention(q, kk, vv, scale)).sum(axis=1)
+                gq, gk, gv = softmax_attention_grad(q, kk, vv, scale, g[:, None] * d_out[r, heads])
+                dq[r, heads] += gq
+                if br == 0:
+                    dKc[hk, js] += gk
+                    dVc[hk, js] += gv
+                else:
+                    np.add.at(dK[hk], ks, gk)
+                    np.add.at(dV[hk], ks, gv)
+    if branches & 1:
+        for j in range(n_cmp):
+            dK[:, j * cmp_stride:j * cmp_stride + cmp_block] += dKc[:, j:j + 1] / cmp_block
+            dV[:, j * cmp_stride:j * cmp_stride + cmp_block] += dVc[:, j:j + 1] / cmp_block
+    return dq, dK, dV, dg

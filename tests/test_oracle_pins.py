@@ -590,6 +590,68 @@ def test_sinks_filling_every_free_place_keep_the_leading_blocks():
     assert gap[0, 0] == np.inf
 
 
+# ---------------------------------------------------------------------------
+# Backward pass
+# ---------------------------------------------------------------------------
+
+def _bwd_problem(seed=0, T=40):
+    rng = np.random.default_rng(seed)
+    cfg = dict(h_q=4, h_kv=2, d_qk=8, d_v=4, sel_block=8, top_k=3, window=10, cmp_block=8,
+               cmp_stride=4, scale=8 ** -0.5, branches=7, per_head_select=False)
+    q = rng.standard_normal((T, 4, 8))
+    K = rng.standard_normal((2, T, 8))
+    V = rng.standard_normal((2, T, 4))
+    g = rng.uniform(0.2, 1.0, (T, 4, 3))
+    return rng, cfg, q, K, V, g
+
+
+def test_backward_matches_finite_differences():
+    """Central differences of the loss sum(d_out * out) in fp64, blocks held fixed."""
+    rng, cfg, q, K, V, g = _bwd_problem()
+    pos = np.arange(q.shape[0])
+    out, idx, _ = O.nsa_rows(cfg, q, pos, K, V, g)
+    d_out = rng.standard_normal(out.shape)
+    grads = O.nsa_rows_backward(cfg, q, pos, K, V, g, idx, d_out)
+
+    def loss():
+        return float((O.nsa_rows(cfg, q, pos, K, V, g, idx=idx)[0] * d_out).sum())
+
+    h = 1e-6
+    for arr, grad in zip((q, K, V, g), grads):
+        flat, gflat = arr.reshape(-1), grad.reshape(-1)
+        for i in rng.choice(flat.size, 24, replace=False):
+            old = flat[i]
+            flat[i] = old + h
+            lp = loss()
+            flat[i] = old - h
+            lm = loss()
+            flat[i] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - gflat[i]) <= 1e-7 + 1e-6 * abs(fd), (fd, gflat[i])
+
+
+def test_backward_of_dense_causal_attention_is_autograd():
+    """Window covering the sequence, gates (0, 0, 1): the gradients are those of dense
+    causal softmax attention, computed by torch autograd in float64 (K/V shared by each
+    group of two heads, so their gradients sum over the group)."""
+    rng, cfg, q, K, V, _ = _bwd_problem(seed=1, T=30)
+    cfg = dict(cfg, window=30, branches=4)
+    T = q.shape[0]
+    pos = np.arange(T)
+    d_out = rng.standard_normal((T, 4, 4))
+    dq, dK, dV, _ = O.nsa_rows_backward(cfg, q, pos, K, V, None, None, d_out)
+    qt = torch.tensor(q, requires_grad=True)
+    Kt = torch.tensor(K, requires_grad=True)
+    Vt = torch.tensor(V, requires_grad=True)
+    o = F.scaled_dot_product_attention(qt.permute(1, 0, 2), Kt.repeat_interleave(2, 0),
+                                       Vt.repeat_interleave(2, 0), is_causal=True,
+                                       scale=cfg["scale"]).permute(1, 0, 2)
+    (o * torch.tensor(d_out)).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK, Kt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dV, Vt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
 def _mut_window_off_by_one(t, window):
     return np.arange(max(0, t - window + 2), t + 1, dtype=np.int64)
 
@@ -707,6 +769,29 @@ O_REAL_CMP = O.block_scores_from_compressed
 O_REAL_SELECT = O.select_blocks
 
 
+def _mut_softmax_grad_no_rowsum(q, k, v, scale, d_o):
+    """Softmax gradient without the row-sum (normaliser) term."""
+    if k.shape[0] == 0:
+        return np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    lg = scale * (q @ k.T)
+    p = np.exp(lg - lg.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    ds = p * (d_o @ v.T)
+    return scale * (ds @ k), scale * (ds.T @ q), p.T @ d_o
+
+
+def _mut_bwd_cmp_not_averaged(cfg, q_rows, positions, K, V, gates_rows, idx, d_out):
+    """Compressed-token gradients added to every window token undivided."""
+    dq, dK, dV, dg = O_REAL_BWD(cfg, q_rows, positions, K, V, gates_rows, idx, d_out)
+    c = dict(cfg, branches=1)
+    _, dK1, dV1, _ = O_REAL_BWD(c, q_rows, positions, K, V, gates_rows, idx, d_out)
+    l = cfg["cmp_block"]
+    return dq, dK + (l - 1) * dK1, dV + (l - 1) * dV1, dg
+
+
+O_REAL_BWD = O.nsa_rows_backward
+
+
 MUTATIONS = {
     "window off by one": ("window_keys", _mut_window_off_by_one),
     "selected keys exclude self": ("selected_keys", _mut_selected_strict_causal),
@@ -719,12 +804,14 @@ MUTATIONS = {
     "probabilities normalised over later blocks": ("block_scores_prob", _mut_prob_over_all_blocks),
     "compressed weights in tokens": ("block_scores_from_compressed", _mut_cmp_weight_in_tokens),
     "sinks kept outside k": ("select_blocks", _mut_sinks_outside_k),
+    "softmax gradient without the normaliser term": ("softmax_attention_grad", _mut_softmax_grad_no_rowsum),
+    "compressed gradient not averaged over its window": ("nsa_rows_backward", _mut_bwd_cmp_not_averaged),
 }
 
 PINS = [test_golden_uniform_query_outputs, test_golden_figure2_selection,
         test_golden_selection_gap, test_golden_prob_selection, test_prob_scores_sum_to_the_number_of_heads,
         test_golden_compressed_aggregation, test_compressed_aggregation_by_source_tokens,
-        lambda: test_sink_blocks_match_brute_force(2),
+        lambda: test_sink_blocks_match_brute_force(2), test_backward_matches_finite_differences,
         test_golden_group_sum_selection, test_selection_ties_go_to_lower_index,
         test_window_of_one_returns_own_value, test_golden_softmax_two_keys,
         lambda: test_selected_branch_keeping_every_block_is_dense_causal(64),
