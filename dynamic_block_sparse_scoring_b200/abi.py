@@ -66,6 +66,9 @@ _SIGS = {
                       ctypes.POINTER(ctypes.c_int32)],
     "nsa_timing_enable": [ctypes.c_int32],
     "nsa_check_bounded_wait": [ctypes.c_uint64, _vp],
+    "nsa_bwd_workspace_size": [_cfgp, ctypes.POINTER(_sz)],
+    "nsa_sparse_attn_bwd": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                            _sz, _vp],
     "nsa_timing_read": [ctypes.c_int32, ctypes.POINTER(ctypes.c_float),
                         ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_int32)],
 }
@@ -125,6 +128,21 @@ def nsa_attn_plan(cfg: NsaConfig, select_inside: bool, ws_bytes: int):
     _check("nsa_attn_plan", lib.nsa_attn_plan(ctypes.byref(cfg), int(select_inside), ws_bytes,
                                               ctypes.byref(path), ctypes.byref(n)))
     return PATHS[path.value], n.value
+
+
+def nsa_bwd_workspace_size(cfg: NsaConfig) -> int:
+    n = _sz(0)
+    _check("nsa_bwd_workspace_size", lib.nsa_bwd_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def nsa_sparse_attn_bwd(cfg, q, k, v, kcmp, vcmp, gates, idx, d_out, dq, dk, dv, dgates=None,
+                        workspace=None, ws_bytes=0, stream=None):
+    _check("nsa_sparse_attn_bwd",
+           lib.nsa_sparse_attn_bwd(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(kcmp),
+                                   _ptr(vcmp), _ptr(gates), _ptr(idx), _ptr(d_out), _ptr(dq),
+                                   _ptr(dk), _ptr(dv), _ptr(dgates), _ptr(workspace), ws_bytes,
+                                   _stream(stream)))
 
 
 def nsa_check_bounded_wait(limit_ns: int, stream=None):

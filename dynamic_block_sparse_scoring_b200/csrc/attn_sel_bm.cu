@@ -44,7 +44,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BLK = 64;             // keys per block (the path requires sel_block == 64)
-constexpr int NTHREADS = 448;      // producer, MMA, 2 softmax warpgroups, epilogue warpgroup
+constexpr int NTHREADS = 480;      // producer, MMA, 2 softmax warpgroups, epilogue warpgroup, Q loader
 constexpr int NM = 8;               // item descriptors in flight
 constexpr int CHUNK_Q = 16384;      // 128 rows x 64 columns bf16
 constexpr int CHUNK_KV = 8192;      // 64 rows x 64 columns bf16
@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int i = 0; i < NM; ++i) {
             tc::mbar_init(bar.meta_full(i), 1);
-            tc::mbar_init(bar.meta_empty(i), 9);   // MMA lane + owning softmax WG + epilogue WG
+            // MMA lane + owning softmax WG + epilogue WG (+ the Q-loader warp, groups of heads)
+            tc::mbar_init(bar.meta_empty(i), MT <= 32 ? 10 : 9);
         }
         tc::mbar_init(bar.drain(), 1);
         *abort_flag = 0;
@@ -161,6 +162,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 1) {
         tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tc::prefetch_map(&map_qg);
+        tc::prefetch_map(&map_k);
+        tc::prefetch_map(&map_v);
+        tc::prefetch_map(&map_po);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -261,23 +268,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 m.kvs = kvs;
                 if constexpr (MT <= 32) {
+                    // the Q-loader warp gathers the item's query rows from the metadata
                     const int tokv = list_at(it.y, m.n);
                     for (int tt = 0; tt < MT; ++tt) m.tok[tt] = __shfl_sync(0xffffffffu, tokv, tt);
-                    const int qs = li % NQ;
-                    if (!bm_warp_wait(bar.q_empty(qs), ((li / NQ) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), m.n * L::QC * a.hpt * 128);
-                    __syncwarp();
-                    // one TMA per (query, 64-column chunk), spread over the lanes; the
-                    // query rows are reused by the chunk's other blocks, so keep them in L2
-                    for (int e = lane; e < m.n * L::QC; e += 32) {
-                        const int tt = e / L::QC, c = e % L::QC;
-                        tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
-                                             &map_qg, bar.q_full(qs), 64 * c, h0, pair_query(m.tok[tt]), b,
-                                             q_policy);
-                    }
                 } else {
                     // more queries than lanes: they go straight into the item's
                     // metadata slot, which the Q loads then read back
@@ -317,7 +310,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                              bar.q_full(qs), 64 * c, r[0], r[1], r[2], r[3], q_policy);
                     }
                 }
-                ++q_loads;
+                if constexpr (MT > 32) ++q_loads;
                 ++i;
             } else {
                 ++ends;    // two end markers: each softmax warpgroup sees one
@@ -356,6 +349,57 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (q_loads > s) {
                 const uint32_t last = s + ((q_loads - 1 - s) / NQ) * NQ;
                 tc::mbar_wait(bar.q_full(s), (last / NQ) & 1, &never, WAIT_NS);
+            }
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------------------ Q loader (groups of
+        // heads): one TMA per (query, 64-column chunk) of every item, spread over the
+        // lanes, into the item's Q stage.  Issuing these 3 x TOK boxes per item from
+        // the producer warp made it the slowest role, so they have their own warp.
+        if constexpr (MT <= 32) {
+            bool ok = true;
+            uint32_t q_loads = 0;
+            const uint64_t q_policy = tc::l2_policy_evict_last();
+            for (int li = 0; ok; ++li) {
+                const int slot = li % NM;
+                if (!bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const ItemMeta& mref = metas[slot];
+                const int valid = mref.valid, lidx = mref.lidx, n = mref.n;
+                const int tokl = lane < MT ? mref.tok[lane] : 0;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
+                if (!valid) break;
+                const int bu = (lidx / nb_all) % bhsel;
+                const int b = bu / a.s.Hsel, u = bu % a.s.Hsel;
+                const int h0 = a.s.per_head ? u : u * a.s.G;
+                const int qs = li % NQ;
+                if (!bm_warp_wait(bar.q_empty(qs), ((li / NQ) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar.q_full(qs), n * L::QC * a.hpt * 128);
+                __syncwarp();
+                for (int e0 = 0; e0 < n * L::QC; e0 += 32) {
+                    const int e = e0 + lane;
+                    const int tt = e / L::QC, c = e % L::QC;
+                    const int qtok = __shfl_sync(0xffffffffu, tokl, tt & 31);
+                    if (e < n * L::QC)
+                        tc::tma_load_4d_hint(sm + L::Q_OFF + (qs * L::QC + c) * CHUNK_Q + tt * a.hpt * 128,
+                                             &map_qg, bar.q_full(qs), 64 * c, h0, pair_query(qtok), b, q_policy);
+                }
+                ++q_loads;
+            }
+            if (!ok) bm_abort(abort_flag);
+            // wait for every copy still in flight before the CTA may exit
+            volatile int never = 0;
+            for (uint32_t s = 0; s < NQ; ++s) {
+                if (q_loads > s) {
+                    const uint32_t last = s + ((q_loads - 1 - s) / NQ) * NQ;
+                    tc::mbar_wait(bar.q_full(s), (last / NQ) & 1, &never, WAIT_NS);
+                }
             }
         }
     } else if (warp == 1) {
@@ -436,7 +480,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
         }
         __syncwarp();
-    } else if (warp < 10) {
+    } else if (warp >= 2 && warp < 10) {
         // ------------------------------------------------------------ softmax (warps 2-5 and
         // 6-9, alternate items; S/P double-buffered in TMEM)
         const int wg = (warp - 2) >> 2;          // softmax warpgroup 0 / 1 takes items li % 2 == wg
@@ -533,7 +577,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0) tc::mbar_arrive(bar.p_full(sb));
         }
         if (!ok) bm_abort(abort_flag);
-    } else {
+    } else if (warp >= 10 && warp < 14) {
         // ------------------------------------------------------------ epilogue (warps 10-13,
         // every item): o = P V (already divided by l) -> bf16 partial rows, staged in
         // shared memory in the 128-byte-swizzled layout and written by TMA stores

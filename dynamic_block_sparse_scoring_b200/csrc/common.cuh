@@ -87,6 +87,12 @@ cudaError_t launch_append_rows(const Shape& s, const __nv_bfloat16* k_new, const
 cudaError_t launch_score_topk(const Shape& s, const __nv_bfloat16* q, const float* kbar,
                               const float* scores_in, float* scores_out, int32_t* idx,
                               cudaStream_t st);
+// backward pass for fixed block sets (attn_bwd.cu)
+bool bwd_supported(const Shape& s);
+cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const __nv_bfloat16* kcmp, const __nv_bfloat16* vcmp,
+                            const float* gates, const int32_t* idx, const __nv_bfloat16* d_out, float* dq,
+                            float* dk, float* dv, float* dgates, float* dkc, float* dvc, cudaStream_t st);
 // selection-score variants (score_mode 1 or 2): scores and/or top-k per row
 bool score_variant_supported(const Shape& s);
 cudaError_t launch_score_variant(const Shape& s, const __nv_bfloat16* q, const float* kbar,

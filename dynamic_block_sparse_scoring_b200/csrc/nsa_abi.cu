@@ -560,6 +560,52 @@ nsa_status nsa_sparse_attn_fwd(const nsa_config* cfg, const void* q, const void*
                                            nullptr, nullptr, ob, cs));
 }
 
+static size_t bwd_ws_bytes(const Shape& s) {
+    if (!(s.flags & NSA_BR_CMP) || s.n_cmp == 0) return 0;
+    return round_up((size_t)s.B * s.Hkv * s.n_cmp * s.dqk * 4, 256) +
+           round_up((size_t)s.B * s.Hkv * s.n_cmp * s.dv * 4, 256);
+}
+
+nsa_status nsa_bwd_workspace_size(const nsa_config* cfg, size_t* bytes) {
+    if (!bytes) return NSA_ERR_INVALID_ARG;
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    *bytes = bwd_ws_bytes(s);
+    return NSA_OK;
+}
+
+nsa_status nsa_sparse_attn_bwd(const nsa_config* cfg, const void* q, const void* k, const void* v,
+                               const void* kcmp, const void* vcmp, const float* gates, const int32_t* idx,
+                               const void* d_out, float* dq, float* dk, float* dv, float* dgates,
+                               void* workspace, size_t ws_bytes, void* stream) {
+    Shape s;
+    nsa_status st = make_shape(cfg, &s);
+    if (st != NSA_OK) return st;
+    const bool sel = (cfg->flags & NSA_BR_SEL) != 0;
+    const bool cmp = (cfg->flags & NSA_BR_CMP) != 0 && s.n_cmp > 0;
+    if (!q || !k || !v || !d_out || !dq || !dk || !dv) return NSA_ERR_INVALID_ARG;
+    if ((sel && !idx) || (cmp && (!kcmp || !vcmp))) return NSA_ERR_INVALID_ARG;
+    if (gates && !dgates) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kcmp) || !aligned16(vcmp) ||
+        !aligned16(gates) || !aligned16(idx) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !aligned16(dgates) || !aligned16(workspace))
+        return NSA_ERR_INVALID_ARG;
+    if (!nsa::bwd_supported(s)) return NSA_ERR_UNSUPPORTED;
+    const size_t need = bwd_ws_bytes(s);
+    if (need && (!workspace || ws_bytes < need)) return NSA_ERR_WORKSPACE;
+    if (s.Tq == 0) return NSA_OK;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* dkc = need ? reinterpret_cast<float*>(ws) : nullptr;
+    float* dvc = need ? reinterpret_cast<float*>(ws + round_up((size_t)s.B * s.Hkv * s.n_cmp * s.dqk * 4, 256))
+                      : nullptr;
+    return cuda_status(nsa::launch_attn_bwd(
+        s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(kcmp),
+        static_cast<const __nv_bfloat16*>(vcmp), gates, idx, static_cast<const __nv_bfloat16*>(d_out), dq, dk,
+        dv, dgates, dkc, dvc, static_cast<cudaStream_t>(stream)));
+}
+
 nsa_status nsa_check_bounded_wait(uint64_t limit_ns, void* stream) {
     if (limit_ns < 1 || limit_ns > 1000000000ull) return NSA_ERR_INVALID_ARG;
     return cuda_status(nsa::launch_wait_selftest(limit_ns, static_cast<cudaStream_t>(stream)));

@@ -220,8 +220,17 @@ nsa_status nsa_topk_select_ex(const nsa_config* cfg, const void* q, const float*
  *   o_sel = softmax attention over the tokens u <= t of the blocks in idx (NSA_BR_SEL)
  *   o_win = softmax attention over keys max(0, t-window+1) .. t           (NSA_BR_WIN)
  *   out   = g0*o_cmp + g1*o_sel + g2*o_win   (gates NULL: weight 1 each)
- * A branch with no visible key contributes 0.  Softmax and accumulation run in
- * fp32; out is rounded to bf16 once.
+ * A branch with no visible key contributes 0.  Precision: bf16 inputs; scores,
+ * softmax and accumulation in fp32; out rounded to bf16.  On the query-major,
+ * split-k and decode plans (nsa_attn_plan) that is the only rounding.  The
+ * block-major plan keeps each kept block's partial result o = (P V) / l in
+ * bf16 (one rounding per (query, head, block), relative error <= 2^-9),
+ * merges a query's partials in fp32 and, when other branches follow, hands
+ * the merged o_sel to the query-major kernel in bf16 (a second rounding of
+ * the selected branch) before the gated sum is rounded once more; with the
+ * selected branch alone the merge writes g_sel * o_sel to out directly.  The
+ * extra roundings add at most about 2 * 2^-9 * g_sel * max|o_sel| to an
+ * output element (measured on the 64k workload: see the parity tests).
  * idx may be NULL, in which case the blocks are selected as nsa_topk_select
  * does (needs q, kbar and at least nsa_workspace_size_min() bytes of
  * workspace; with nsa_workspace_size() bytes and more than 16 query rows the
@@ -274,6 +283,32 @@ nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, con
                                        const void* v, const float* kbar, const void* kcmp,
                                        const void* vcmp, const float* gates, void* out,
                                        void* stream);
+
+/*
+ * Backward pass for fixed block sets (transcript #94 §6: the top-k choice is
+ * discrete and passes no gradient, the compressed branch carries gradient to
+ * the keys and values it pools; §2: each branch is a softmax-weighted sum).
+ * For the loss sum(d_out * out), with out as nsa_sparse_attn_fwd computes it
+ * from the same q, k, v, kcmp, vcmp, gates and the blocks in idx:
+ *   dq     [B, Tq, Hq, d_qk]  fp32, overwritten
+ *   dk, dv [B, Hkv, Tkv, d]   fp32, overwritten (every key's gradient, summed
+ *                             over queries and heads; a compressed token's
+ *                             gradient reaches each token of its window
+ *                             divided by cmp_block)
+ *   dgates [B, Tq, Hq, 3]     fp32, d_out . o_branch (NULL when gates is NULL)
+ * d_out [B, Tq, Hq, d_v] bf16; idx as returned by the selection (required
+ * with NSA_BR_SEL); kcmp/vcmp as nsa_pool_kv writes them (with NSA_BR_CMP).
+ * Needs nsa_bwd_workspace_size() bytes of workspace (the compressed tokens'
+ * gradients).  Plain fp32 CUDA-core arithmetic with atomic accumulation of
+ * dk / dv (summation order varies between runs).  Limits: d_qk <= 256, at
+ * most 16384 keys per branch and row (NSA_ERR_UNSUPPORTED otherwise).
+ */
+nsa_status nsa_bwd_workspace_size(const nsa_config* cfg, size_t* bytes);
+nsa_status nsa_sparse_attn_bwd(const nsa_config* cfg, const void* q, const void* k,
+                               const void* v, const void* kcmp, const void* vcmp,
+                               const float* gates, const int32_t* idx, const void* d_out,
+                               float* dq, float* dk, float* dv, float* dgates,
+                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Reads and clears the device-side status word of the tensor-core kernels:

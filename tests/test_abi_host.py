@@ -221,3 +221,23 @@ def test_score_variant_flags_validated_on_host(abi):
     fake = 1 << 20
     assert L.nsa_score_blocks(ctypes.byref(cmp_mode), fake, fake, fake, None) == 1
     assert L.nsa_topk_select(ctypes.byref(cmp_mode), fake, fake, None, fake, None) == 1
+
+
+def test_backward_validates_on_host(abi):
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
+    wl = WORKLOADS["tiny"]
+    cfg = abi.config(wl)
+    fake = 1 << 20
+    L = abi.lib
+    n = ctypes.c_size_t(0)
+    assert L.nsa_bwd_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == 0
+    n_cmp = (wl.seqlen_kv - wl.cmp_block) // wl.cmp_stride + 1
+    assert n.value >= n_cmp * (wl.d_qk + wl.d_v) * 4 * wl.h_kv
+    args = [fake] * 12          # q, k, v, kcmp, vcmp, gates, idx, d_out, dq, dk, dv, dgates
+    # the selected branch needs the forward's ids; gates need a gate gradient buffer
+    a = list(args); a[6] = None
+    assert L.nsa_sparse_attn_bwd(ctypes.byref(cfg), *a, fake, n.value, None) == 1
+    a = list(args); a[11] = None
+    assert L.nsa_sparse_attn_bwd(ctypes.byref(cfg), *a, fake, n.value, None) == 1
+    # workspace too small
+    assert L.nsa_sparse_attn_bwd(ctypes.byref(cfg), *args, fake, n.value - 256, None) == 3

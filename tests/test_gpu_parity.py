@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 
 from dynamic_block_sparse_scoring_b200 import abi
 from tests.parity import (GpuRun, check_idx, check_out, check_selection_all_rows, f64,
-                          oracle_selection, OUT_MAX_ABS, OUT_MEAN_ABS, SCORE_ATOL, SCORE_RTOL)
+                          oracle_cfg, oracle_selection, OUT_MAX_ABS, OUT_MEAN_ABS, SCORE_ATOL,
+                          SCORE_RTOL)
 
 TINY = WORKLOADS["tiny"]
 
@@ -302,3 +303,36 @@ def test_minimal_workspace_path_matches_oracle(name):
     same = (run.idx[0] == run.idx_fwd[0]).all(dim=0).all(dim=-1).cpu().numpy()
     err = np.abs(f64(out[0]) - f64(run.out[0]))[same]
     assert err.max() <= 2 * OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS
+
+
+@pytest.mark.parametrize("name", ["nsa_small", "bm_g8_ragged"])
+def test_block_major_rounding_budget(name):
+    """The block-major plan rounds each kept block's partial result and the merged
+    selected branch to bf16 before the final rounding (include/nsa.h).  Bound the extra
+    error: against the fp64 oracle it stays within 1e-2 max / 1e-3 mean (half the
+    general tolerance), and it differs from the query-major plan (one rounding) by at
+    most 2 * 2^-9 * g_sel * max|o_sel| plus one bf16 ulp (2^-7 relative) of the output."""
+    wl = EDGE[name]
+    run = GpuRun(wl)
+    assert abi.nsa_attn_plan(run.cfg, True, abi.nsa_workspace_size(run.cfg))[0] == "block-major"
+    rows = np.arange(wl.seqlen_q)
+    ora, _, _ = run.oracle_rows(0, rows, idx=run.idx_fwd[0].cpu().numpy())
+    got = f64(run.out[0])
+    err = np.abs(got - ora)
+    assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+    # the selected branch alone (oracle, fp64) bounds what the extra roundings can move
+    sel_only = dict(oracle_cfg(wl), branches=BR_SEL, gated=False)
+    q = f64(run.x["q"][0])
+    o_sel, _, _ = O.nsa_rows(sel_only, q, rows + wl.q_pos0, f64(run.x["k"][0]), f64(run.x["v"][0]),
+                             None, idx=run.idx_fwd[0].cpu().numpy())
+    g_sel = f64(run.x["gates"][0])[..., 1]
+    bound = 2 * 2.0 ** -9 * g_sel * np.abs(o_sel).max(axis=-1) + 2.0 ** -7 * np.abs(ora).max(axis=-1)
+    ws = torch.empty(abi.nsa_workspace_size_min(run.cfg), dtype=torch.uint8, device="cuda")
+    qm = torch.empty_like(run.out)
+    abi.nsa_sparse_attn_fwd(run.cfg, run.x["q"], run.x["k"], run.x["v"], run.pooled["kbar"],
+                            run.pooled["kcmp"], run.pooled["vcmp"], run.x["gates"], run.idx_fwd,
+                            qm, ws, ws.numel())
+    torch.cuda.synchronize()
+    diff = np.abs(got - f64(qm)).max(axis=-1)
+    assert (diff <= bound + 1e-6).all(), float((diff - bound).max())
+    print(f"{name}: block-major vs oracle max {err.max():.3e} mean {err.mean():.3e}")
