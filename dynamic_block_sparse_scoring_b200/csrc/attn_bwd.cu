@@ -87,7 +87,11 @@ __global__ void __launch_bounds__(BW_NT) bwd_rows_kernel(BwdArgs a) {
     float dq_acc[2] = {0.f, 0.f};         // columns tid and tid + 128 of dq (dqk <= 256)
     const size_t plane = (size_t)b * s.Hkv + kvh;
     for (int br = 0; br < 3; ++br) {
-        if (!(s.flags & (1u << br))) continue;
+        if (!(s.flags & (1u << br))) {
+            // the output does not depend on a disabled branch's gate
+            if (tid == 0 && a.dgates) a.dgates[row * 3 + br] = 0.f;
+            continue;
+        }
         // the branch's keys: e -> (key row, whether it is a compressed token)
         int nkeys = 0, win_lo = 0, nblk = 0;
         if (br == 0) {

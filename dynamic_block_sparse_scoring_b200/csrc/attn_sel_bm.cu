@@ -582,16 +582,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // every item): o = P V (already divided by l) -> bf16 partial rows, staged in
         // shared memory in the 128-byte-swizzled layout and written by TMA stores
         // (one {64 columns x hpt rows} box per query and column half, whole lines
-        // instead of a 256-byte row per lane); lse = m + log2(l) per row.  The four
-        // warps decide every wait together (barrier reduction), so none of them can
-        // be left alone at a named barrier.
+        // instead of a 256-byte row per lane); lse = m + log2(l) per row.  A warp's 32
+        // rows are whole queries, so each warp stores its own queries' rows as soon as
+        // it has staged them (warp-level ordering only; the stores of an item are
+        // spread over the four warps).  The four warps decide every wait together
+        // (barrier reduction), so none of them can be left alone at a named barrier.
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int tt = r / a.hpt, hl = r % a.hpt;
         const float* row_m = reinterpret_cast<const float*>(sm + L::ROW_OFF);
         const float* row_l = row_m + 2 * BM;
-        const bool issuer = warp == 10;           // lane q issues the stores of the item's query q
+        // queries whose rows this warp holds: qpw of them, one store per lane l < qpw
+        // (one head per query: lanes 0..7 store four rows each with one scatter)
+        const int qpw = MT > 32 ? 32 : 32 / a.hpt;
         const uint64_t st_policy = tc::l2_policy_evict_first();
         uint32_t halves = 0;
         bool ok = true;
@@ -599,20 +603,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int slot = li % NM;
             bool okw = bm_warp_wait(bar.meta_full(slot), (li / NM) & 1, abort_flag);
             int valid = 0, lidx = 0, n = 0, tokr = 0;
-            int tok_lane[NG];             // the queries whose stores this lane issues
+            int tok_lane[4];              // the queries whose stores this lane issues
 #pragma unroll
-            for (int g = 0; g < NG; ++g) tok_lane[g] = 0;
+            for (int g = 0; g < 4; ++g) tok_lane[g] = 0;
             if (okw) {
                 const ItemMeta& mref = metas[slot];
                 valid = mref.valid;
                 lidx = mref.lidx;
                 n = mref.n;
                 tokr = tt < MT ? mref.tok[tt] : 0;
-                // (one head per query: lane l stores rows 4l .. 4l + 3, one scatter of four)
+                // lane l of warp quarter w: query w * qpw + l (groups of heads), or
+                // rows 32 w + 4 l .. 32 w + 4 l + 3 (one head per query, lanes 0..7)
 #pragma unroll
-                for (int g = 0; g < NG; ++g) {
-                    const int qi = MT > 32 ? 4 * lane + g : 32 * g + lane;
-                    tok_lane[g] = qi < MT ? mref.tok[qi] : 0;
+                for (int g = 0; g < 4; ++g) {
+                    const int qi = MT > 32 ? 32 * quarter + 4 * lane + g : quarter * qpw + lane;
+                    const bool mine = MT > 32 ? lane < 8 : (g == 0 && lane < qpw);
+                    tok_lane[g] = mine && qi < MT ? mref.tok[qi] : 0;
                 }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar.meta_empty(slot));
@@ -636,10 +642,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int bu = (lidx / nb_all) % bhsel;
             const float m = row_m[sb * BM + r], l = row_l[sb * BM + r];
             const size_t prow = (((size_t)bu * a.s.Tq + pair_query(tokr)) * a.s.topk + pair_slot(tokr)) * a.hpt + hl;
-            // first partial row of each query this lane stores (issuer warp)
-            int prow_q[NG];
+            // first partial row of each query this lane stores
+            int prow_q[4];
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
+            for (int g = 0; g < 4; ++g)
                 prow_q[g] = (int)((((size_t)bu * a.s.Tq + pair_query(tok_lane[g])) * a.s.topk + pair_slot(tok_lane[g])) *
                                   a.hpt);
 #pragma unroll 1
@@ -654,10 +660,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar.o_free(sb));
                 }
-                // staging buffer (halves & 1) was last read by the stores issued two
-                // halves ago; at most the latest group may still be reading
-                if (issuer) tc::bulk_wait_read<1>();
-                tc::named_bar_sync(1, 128);
+                // staging buffer (halves & 1) was last read by the stores this warp
+                // issued two halves ago; at most the latest group may still be reading
+                tc::bulk_wait_read<1>();
+                __syncwarp();
                 uint8_t* rowp = sm + L::STG_OFF + (halves & 1) * (BM * 128) + r * 128;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -669,34 +675,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     *reinterpret_cast<uint4*>(rowp + ((q ^ (r & 7)) << 4)) = u4;
                 }
                 tc::fence_proxy_async_smem();
-                tc::named_bar_sync(1, 128);
-                if (issuer) {
-                    uint8_t* stg = sm + L::STG_OFF + (halves & 1) * (BM * 128);
-                    if constexpr (MT > 32) {
-                        static_assert(NG == 4, "one scatter of four rows per lane");
-                        if (4 * lane + 3 < n) {
-                            tc::tma_scatter4(&map_po, stg + 4 * lane * 128, c, prow_q[0], prow_q[1], prow_q[2],
+                __syncwarp();
+                uint8_t* stg = sm + L::STG_OFF + (halves & 1) * (BM * 128);
+                if constexpr (MT > 32) {
+                    const int r0 = 32 * quarter + 4 * lane;          // this lane's four rows
+                    if (lane < 8) {
+                        if (r0 + 3 < n) {
+                            tc::tma_scatter4(&map_po, stg + r0 * 128, c, prow_q[0], prow_q[1], prow_q[2],
                                              prow_q[3]);
                         } else {
 #pragma unroll
-                            for (int g = 0; g < NG; ++g)
-                                if (4 * lane + g < n)
-                                    tc::tma_store_2d_hint(&map_po, stg + (4 * lane + g) * 128, c, prow_q[g],
-                                                          st_policy);
+                            for (int g = 0; g < 4; ++g)
+                                if (r0 + g < n) tc::tma_store_2d_hint(&map_po, stg + (r0 + g) * 128, c, prow_q[g],
+                                                                      st_policy);
                         }
-                    } else {
-#pragma unroll
-                        for (int g = 0; g < NG; ++g)
-                            if (32 * g + lane < n)
-                                tc::tma_store_2d_hint(&map_po, stg + (32 * g + lane) * a.hpt * 128, c, prow_q[g],
-                                                      st_policy);
                     }
-                    tc::bulk_commit();
+                } else {
+                    const int qi = quarter * qpw + lane;
+                    if (lane < qpw && qi < n)
+                        tc::tma_store_2d_hint(&map_po, stg + qi * a.hpt * 128, c, prow_q[0], st_policy);
                 }
+                tc::bulk_commit();
             }
             if (row_valid) __stcs(a.part_lse + prow, m + __log2f(l));
         }
-        if (issuer) tc::bulk_wait<0>();
+        tc::bulk_wait<0>();
         if (!ok) bm_abort(abort_flag);
     }
 

@@ -156,8 +156,10 @@ nsa_status nsa_pool_kv(const nsa_config* cfg, const void* k, const void* v, floa
  * nsa_topk_select / nsa_sparse_attn_fwd with seqlen_kv = the cache size and
  * q_pos0 = the newest position: every branch is causal, so cache rows after
  * the query are never attended, but they must hold finite values (e.g.
- * zeros), because masked keys still enter the value products with weight 0.
- * kbar / kcmp / vcmp may be NULL when the call completes none of their tokens.
+ * zeros), because masked keys still enter the value products with weight 0;
+ * the same holds for the compressed tokens not yet complete (zero kcmp and
+ * vcmp once when the cache is created).  kbar / kcmp / vcmp may be NULL when
+ * the call completes none of their tokens.
  */
 nsa_status nsa_append_kv(const nsa_config* cfg, void* k, void* v, const void* k_new,
                          const void* v_new, float* kbar, void* kcmp, void* vcmp, void* stream);

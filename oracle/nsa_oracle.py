@@ -297,10 +297,25 @@ def opt(cfg, name, default):
     return getattr(cfg, name, default)
 
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to bfloat16 (8-bit significand), to nearest with ties to even, via
+    float32 (the value is first rounded to float32, as a float32 mean would be).
+    Returned as float64.  Finite inputs only."""
+    f = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (f >> 16) & 1
+    r = ((f + 0x7FFF + lsb) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def selection_scores(cfg, q_rows, positions, pooled, n_blocks):
     """Block scores of the configured kind: "dot" (the scaled dot product with the
     pooled key, summed over the unit; the default), "prob" (``block_scores_prob``)
-    or "cmp" (``block_scores_from_compressed``)."""
+    or "cmp" (``block_scores_from_compressed``).
+
+    The "cmp" scores read the compressed keys as the kernel stores them, rounded
+    to bfloat16: the top-k is an integer decision, taken on both sides from the
+    same stored keys (the fp64 means differ from the stored ones by up to 2^-9
+    relative, enough to reorder blocks whose scores are 1e-4 apart)."""
     mode = opt(cfg, "score_mode", "dot")
     h_q, h_kv, sel_block = opt(cfg, "h_q", 0), opt(cfg, "h_kv", 0), opt(cfg, "sel_block", 0)
     scale, per_head = opt(cfg, "scale", 1.0), bool(opt(cfg, "per_head_select", False))
@@ -308,7 +323,8 @@ def selection_scores(cfg, q_rows, positions, pooled, n_blocks):
         return block_scores_prob(q_rows, positions, pooled["Kbar"], h_q, h_kv, sel_block, scale,
                                  per_head, n_blocks)
     if mode == "cmp":
-        return block_scores_from_compressed(q_rows, positions, pooled["Kc"], h_q, h_kv, sel_block,
+        return block_scores_from_compressed(q_rows, positions, round_bf16(pooled["Kc"]), h_q, h_kv,
+                                            sel_block,
                                             opt(cfg, "cmp_block", 0), opt(cfg, "cmp_stride", 1),
                                             scale, per_head, n_blocks)
     return block_scores(q_rows, positions, pooled["Kbar"], h_q, h_kv, sel_block, scale, per_head,

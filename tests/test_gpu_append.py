@@ -89,7 +89,9 @@ def test_decode_steps_on_the_growing_cache_match_the_oracle():
     g.manual_seed(60)
     k = torch.zeros_like(x["k"])
     v = torch.zeros_like(x["v"])
-    pooled = abi.alloc_pooled(cfg, "cuda")
+    # a new cache: its rows and its pooled tokens start at zero (finite), since masked
+    # keys still enter the value products with weight 0
+    pooled = {name: t.zero_() for name, t in abi.alloc_pooled(cfg, "cuda").items()}
     _append(wl, k, v, pooled, x["k"], x["v"], 0, 2000)
     filled = 2000
     for t in [2000, 2001, 2047, 2048, 2063, 2100]:

@@ -309,9 +309,10 @@ def test_minimal_workspace_path_matches_oracle(name):
 def test_block_major_rounding_budget(name):
     """The block-major plan rounds each kept block's partial result and the merged
     selected branch to bf16 before the final rounding (include/nsa.h).  Bound the extra
-    error: against the fp64 oracle it stays within 1e-2 max / 1e-3 mean (half the
-    general tolerance), and it differs from the query-major plan (one rounding) by at
-    most 2 * 2^-9 * g_sel * max|o_sel| plus one bf16 ulp (2^-7 relative) of the output."""
+    error per (row, head): against the fp64 oracle within half a bf16 ulp of the output
+    plus 2 * 2^-9 * g_sel * max|o_sel| plus 1e-3 (mean <= 1e-3, half the general
+    tolerance), and against the query-major plan (one rounding) within the extra term
+    plus one bf16 ulp (2^-7 relative) of the output."""
     wl = EDGE[name]
     run = GpuRun(wl)
     assert abi.nsa_attn_plan(run.cfg, True, abi.nsa_workspace_size(run.cfg))[0] == "block-major"
@@ -319,14 +320,19 @@ def test_block_major_rounding_budget(name):
     ora, _, _ = run.oracle_rows(0, rows, idx=run.idx_fwd[0].cpu().numpy())
     got = f64(run.out[0])
     err = np.abs(got - ora)
-    assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
     # the selected branch alone (oracle, fp64) bounds what the extra roundings can move
     sel_only = dict(oracle_cfg(wl), branches=BR_SEL, gated=False)
     q = f64(run.x["q"][0])
     o_sel, _, _ = O.nsa_rows(sel_only, q, rows + wl.q_pos0, f64(run.x["k"][0]), f64(run.x["v"][0]),
                              None, idx=run.idx_fwd[0].cpu().numpy())
     g_sel = f64(run.x["gates"][0])[..., 1]
-    bound = 2 * 2.0 ** -9 * g_sel * np.abs(o_sel).max(axis=-1) + 2.0 ** -7 * np.abs(ora).max(axis=-1)
+    extra = 2 * 2.0 ** -9 * g_sel * np.abs(o_sel).max(axis=-1)
+    # against the oracle: the final rounding (half a bf16 ulp, 2^-8 relative), the two
+    # extra roundings, and fp32 accumulation
+    ora_bound = 2.0 ** -8 * np.abs(ora).max(axis=-1) + extra + 1e-3
+    assert (err.max(axis=-1) <= ora_bound).all(), float((err.max(axis=-1) - ora_bound).max())
+    assert err.mean() <= 1e-3, err.mean()
+    bound = extra + 2.0 ** -7 * np.abs(ora).max(axis=-1)
     ws = torch.empty(abi.nsa_workspace_size_min(run.cfg), dtype=torch.uint8, device="cuda")
     qm = torch.empty_like(run.out)
     abi.nsa_sparse_attn_fwd(run.cfg, run.x["q"], run.x["k"], run.x["v"], run.pooled["kbar"],

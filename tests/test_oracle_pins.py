@@ -590,6 +590,16 @@ def test_sinks_filling_every_free_place_keep_the_leading_blocks():
     assert gap[0, 0] == np.inf
 
 
+def test_golden_bf16_rounding():
+    """Round to nearest, ties to even, on hand-derived cases; and torch's bf16 cast."""
+    gd = golden("bf16_rounding.json")
+    for c in gd["cases"]:
+        assert O.round_bf16(np.array([c["x"]]))[0] == c["expected"], c
+    x = np.random.default_rng(40).standard_normal(10000) * 30
+    want = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.round_bf16(x), want)
+
+
 # ---------------------------------------------------------------------------
 # Backward pass
 # ---------------------------------------------------------------------------
