@@ -342,20 +342,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok && pend.plane >= 0 && !issue_v(pend)) ok = false;
         if (!ok) dec_abort(abort_flag);
         // wait for every copy still in flight before the CTA may exit
-        volatile int never = 0;
         for (uint32_t st = 0; st < NKS; ++st)
             if (kcount > st) {
                 const uint32_t last = st + ((kcount - 1 - st) / NKS) * NKS;
-                tc::mbar_wait(bar.k_full(st), (last / NKS) & 1, &never, WAIT_NS);
+                tc::mbar_wait_bounded(bar.k_full(st), (last / NKS) & 1, WAIT_NS);
             }
         for (uint32_t st = 0; st < 2; ++st) {
             if (vcount > st) {
                 const uint32_t last = st + ((vcount - 1 - st) / 2) * 2;
-                tc::mbar_wait(bar.v_full(st), (last >> 1) & 1, &never, WAIT_NS);
+                tc::mbar_wait_bounded(bar.v_full(st), (last >> 1) & 1, WAIT_NS);
             }
             if (qcount > st) {
                 const uint32_t last = st + ((qcount - 1 - st) / 2) * 2;
-                tc::mbar_wait(bar.q_full(st), (last >> 1) & 1, &never, WAIT_NS);
+                tc::mbar_wait_bounded(bar.q_full(st), (last >> 1) & 1, WAIT_NS);
             }
         }
     } else if (warp == 1) {
@@ -430,9 +429,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ++ocount;
             }
             if (!ok) dec_abort(abort_flag);
-            volatile int never = 0;
             // the last epilogue has read O (and every MMA before its commit completed)
-            if (ocount > 0) tc::mbar_wait(bar.o_free(), (ocount - 1) & 1, &never, WAIT_NS);
+            if (ocount > 0) tc::mbar_wait_bounded(bar.o_free(), (ocount - 1) & 1, WAIT_NS);
         }
         __syncwarp();
     } else {

@@ -338,17 +338,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (!ok) bm_abort(abort_flag);
         // wait for every copy still in flight before the CTA may exit
-        volatile int never = 0;
         for (uint32_t s = 0; s < 2; ++s) {
             if (kv_loads > s) {
                 const uint32_t last = s + ((kv_loads - 1 - s) / 2) * 2;
-                tc::mbar_wait(bar.kv_full(s), (last >> 1) & 1, &never, WAIT_NS);
+                tc::mbar_wait_bounded(bar.kv_full(s), (last >> 1) & 1, WAIT_NS);
             }
         }
         for (uint32_t s = 0; s < NQ; ++s) {
             if (q_loads > s) {
                 const uint32_t last = s + ((q_loads - 1 - s) / NQ) * NQ;
-                tc::mbar_wait(bar.q_full(s), (last / NQ) & 1, &never, WAIT_NS);
+                tc::mbar_wait_bounded(bar.q_full(s), (last / NQ) & 1, WAIT_NS);
             }
         }
     } else if (warp == 14) {
@@ -394,11 +393,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) bm_abort(abort_flag);
             // wait for every copy still in flight before the CTA may exit
-            volatile int never = 0;
             for (uint32_t s = 0; s < NQ; ++s) {
                 if (q_loads > s) {
                     const uint32_t last = s + ((q_loads - 1 - s) / NQ) * NQ;
-                    tc::mbar_wait(bar.q_full(s), (last / NQ) & 1, &never, WAIT_NS);
+                    tc::mbar_wait_bounded(bar.q_full(s), (last / NQ) & 1, WAIT_NS);
                 }
             }
         }
@@ -475,9 +473,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 prev_last = last;
             }
             if (!ok) bm_abort(abort_flag);
-            volatile int never = 0;
             tc::mma_commit(bar.drain());
-            tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
+            tc::mbar_wait_bounded(bar.drain(), 0, WAIT_NS);
         }
         __syncwarp();
     } else if (warp >= 2 && warp < 10) {

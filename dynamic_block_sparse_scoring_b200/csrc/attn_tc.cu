@@ -200,9 +200,10 @@ struct Producer {
             const int per_seg = L::QC + L::VC;
             if (e < 2 * per_seg) {
                 const int sg = e / per_seg, c = e % per_seg;
-                if (kt.seg[sg] >= 0) {
-                    if (c < L::QC) tc::tma_prefetch_l2_3d(cmp ? mkc : mk, 64 * c, kt.seg[sg], plane);
-                    else tc::tma_prefetch_l2_3d(cmp ? mvc : mv, 64 * (c - L::QC), kt.seg[sg], plane);
+                const int row = sg ? kt.seg[1] : kt.seg[0];   // (a select keeps kt in registers)
+                if (row >= 0) {
+                    if (c < L::QC) tc::tma_prefetch_l2_3d(cmp ? mkc : mk, 64 * c, row, plane);
+                    else tc::tma_prefetch_l2_3d(cmp ? mvc : mv, 64 * (c - L::QC), row, plane);
                 }
             }
             return true;
@@ -407,14 +408,13 @@ struct Producer {
 
     // Waits for every copy this warp issued (bounded, regardless of abort).
     __device__ void drain(uint32_t q_loads) {
-        volatile int never = 0;
         for (uint32_t s = 0; s < NS && s < gk; ++s) {
             const uint32_t last = s + ((gk - 1 - s) / NS) * NS;   // last key tile on stage s
             const uint32_t ph = (last / NS) & 1;
-            tc::mbar_wait(bar.k_full(s), ph, &never, WAIT_NS);
-            tc::mbar_wait(bar.v_full(s), ph, &never, WAIT_NS);
+            tc::mbar_wait_bounded(bar.k_full(s), ph, WAIT_NS);
+            tc::mbar_wait_bounded(bar.v_full(s), ph, WAIT_NS);
         }
-        if (q_loads > 0) tc::mbar_wait(bar.q_full(), (q_loads - 1) & 1, &never, WAIT_NS);
+        if (q_loads > 0) tc::mbar_wait_bounded(bar.q_full(), (q_loads - 1) & 1, WAIT_NS);
     }
 };
 
@@ -560,9 +560,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) raise_abort(abort_flag);
             // all issued MMAs must finish before TMEM is released
-            volatile int never = 0;
             tc::mma_commit(bar.drain());
-            tc::mbar_wait(bar.drain(), 0, &never, WAIT_NS);
+            tc::mbar_wait_bounded(bar.drain(), 0, WAIT_NS);
         }
         __syncwarp();
     }
@@ -670,12 +669,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc::fence_after_sync();
                 // valid key offsets [lo, hi] of this thread's segment for its row
                 int lo = 0, hi = -1;
-                const int s0 = kt.seg[half];
+                const int s0 = half ? kt.seg[1] : kt.seg[0];
                 if (s0 >= 0 && row_valid) {
                     if (kt.br == BR_CMP) {
                         hi = min(SEG - 1, cmp_cap - s0);
                     } else if (kt.br == BR_SEL) {
-                        if ((kt.member[half] >> tt) & 1u) hi = min(SEG - 1, t - s0);
+                        if (((half ? kt.member[1] : kt.member[0]) >> tt) & 1u) hi = min(SEG - 1, t - s0);
                     } else {
                         lo = max(0, t - a.s.win + 1 - s0);
                         hi = min(SEG - 1, t - s0);

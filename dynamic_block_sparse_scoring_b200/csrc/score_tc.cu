@@ -199,11 +199,10 @@ __global__ void __launch_bounds__(SNT, 1)
                 __syncwarp();
             }
         if (!ok) sc_abort(abort_flag);
-        volatile int never = 0;
         for (uint32_t st = 0; st < 2; ++st)
             if (cnt > st) {
                 const uint32_t last = st + ((cnt - 1 - st) / 2) * 2;
-                tc::mbar_wait(bar.full(st), (last >> 1) & 1, &never, WAIT_NS);
+                tc::mbar_wait_bounded(bar.full(st), (last >> 1) & 1, WAIT_NS);
             }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -244,9 +243,8 @@ __global__ void __launch_bounds__(SNT, 1)
                 tc::mma_commit(bar.s_full(sb));
             }
             if (!ok) sc_abort(abort_flag);
-            volatile int never = 0;
             // every MMA completes before TMEM is released
-            if (n_nt > 0) tc::mbar_wait(bar.s_full((n_nt - 1) & 1), ((n_nt - 1) >> 1) & 1, &never, WAIT_NS);
+            if (n_nt > 0) tc::mbar_wait_bounded(bar.s_full((n_nt - 1) & 1), ((n_nt - 1) >> 1) & 1, WAIT_NS);
         }
         __syncwarp();
     } else {

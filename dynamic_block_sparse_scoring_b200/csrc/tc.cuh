@@ -73,6 +73,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
     }
 }
 
+// The same bounded wait without an abort flag: for the drains that must see
+// in-flight copies and MMAs complete even after another role has aborted.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* b, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(b, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
 // ----------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
