@@ -105,8 +105,8 @@ struct Smem {
     static constexpr int XCH_OFF = UNION_OFF + MAX_UNION * 4;      // row max / sum exchange
     static constexpr int BAR_OFF = XCH_OFF + 6 * BM * 4;
     // barriers: q_full, q_empty, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    // meta_full[NM], meta_empty[NM], s_full[2], p_full[2], pv_done, drain
-    static constexpr int NBAR = 2 + 4 * NS + 2 * NM + 4 + 2;
+    // meta_full[NM], meta_empty[NM], s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int NBAR = 2 + 4 * NS + 2 * NM + 4 + 3;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int BYTES = MISC_OFF + 64;
     static constexpr int ALLOC = BYTES + 1024;   // slack to align the base to 1024 B
@@ -126,8 +126,9 @@ struct Bars {
     __device__ __forceinline__ uint64_t* meta_empty(int i) const { return b + 2 + 4 * NS + NM + i; }
     __device__ __forceinline__ uint64_t* s_full(int i) const { return b + 2 + 4 * NS + 2 * NM + i; }
     __device__ __forceinline__ uint64_t* p_full(int i) const { return b + 4 + 4 * NS + 2 * NM + i; }
-    __device__ __forceinline__ uint64_t* pv_done() const { return b + 6 + 4 * NS + 2 * NM; }
-    __device__ __forceinline__ uint64_t* drain() const { return b + 7 + 4 * NS + 2 * NM; }
+    // P V of key tile k completes pv_done(k & 1)
+    __device__ __forceinline__ uint64_t* pv_done(int i) const { return b + 6 + 4 * NS + 2 * NM + i; }
+    __device__ __forceinline__ uint64_t* drain() const { return b + 8 + 4 * NS + 2 * NM; }
 };
 
 __device__ __forceinline__ Bars make_bars(uint64_t* b) {
@@ -453,7 +454,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc::mbar_init(bar.s_full(i), 1);
             tc::mbar_init(bar.p_full(i), 8);       // 8 softmax warps
         }
-        tc::mbar_init(bar.pv_done(), 1);
+        tc::mbar_init(bar.pv_done(0), 1);
+        tc::mbar_init(bar.pv_done(1), 1);
         tc::mbar_init(bar.drain(), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -549,7 +551,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                        idesc_pv, (prev_first && kk == 0) ? 0u : 1u);
                         }
                         tc::mma_commit(bar.v_empty(pst));
-                        tc::mma_commit(bar.pv_done());
+                        tc::mma_commit(bar.pv_done(prev_gi & 1));
                     }
                     if (br == BR_END) break;
                     have_prev = true;
@@ -580,7 +582,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float* xmax = reinterpret_cast<float*>(sm + L::XCH_OFF);   // [2 parity][2 half][BM]
         float* xsum = xmax + 4 * BM;                                 // [2 half][BM]
         constexpr int DVH = DV / 2;
-        uint32_t gm = 0, gi = 0, npv = 0;
+        uint32_t gm = 0, gi = 0;
+        // P V of key tile k is the (k >> 1)-th completion of pv_done(k & 1).  When
+        // this warp has S of tile k, P V of tile k - 2 has completed (the tensor
+        // pipe runs in order) and that of tile k + 1 cannot have started, so the
+        // parity wait for tile k - 1 is unambiguous however many earlier waits were
+        // skipped.
+        auto wait_pv = [&](uint32_t k) {
+            return warp_wait(bar.pv_done(k & 1), (k >> 1) & 1, abort_flag);
+        };
         bool ok = true;
         for (int work = blockIdx.x; ok && work < a.n_work * a.n_split; work += gridDim.x) {
             const WorkTile w = decode_work(a, work % a.n_work);
@@ -739,26 +749,71 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 };
-                if (__all_sync(0xffffffffu, lo == 0 && hi == SEG - 1))
-                    half_row(std::false_type{});
-                else
-                    half_row(std::true_type{});
+                // Later tiles of a branch try one pass first: the exponentials use the
+                // row's running reference max while the tile's max is taken alongside.
+                // The two passes above would keep that reference unless a score
+                // exceeds it by more than 8 (log2 units), so when no row of this warp
+                // pair does (one barrier vote), the result is theirs; otherwise both
+                // warps redo the tile with them (S is still in TMEM: no P is stored
+                // before the vote).
+                auto one_pass = [&](auto masked_tag) {
+                    constexpr bool MASKED = decltype(masked_tag)::value;
+                    tc::tmem_ld32(tS0 + sb * 128 + lane_off + half * SEG, sv);
+                    tc::tmem_ld32(tS0 + sb * 128 + lane_off + half * SEG + 32, sv + 32);
+                    tc::tmem_wait_ld();
+                    const uint32_t span = (uint32_t)(hi - lo);
+                    const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
+                    float ym[4], ps[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) ym[q] = -INFINITY;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) ps[q] = 0.f;
+#pragma unroll
+                    for (int k = 0; k < SEG; k += 2) {
+                        float x0 = __uint_as_float(sv[k]), x1 = __uint_as_float(sv[k + 1]);
+                        if (MASKED) {
+                            x0 = (uint32_t)(k - lo) <= span ? x0 : -INFINITY;
+                            x1 = (uint32_t)(k + 1 - lo) <= span ? x1 : -INFINITY;
+                        }
+                        const float y0 = fmaf(x0, a.scale_log2, neg_m);
+                        const float y1 = fmaf(x1, a.scale_log2, neg_m);
+                        ym[(k >> 1) & 3] = fmaxf(ym[(k >> 1) & 3], fmaxf(y0, y1));
+                        const float p0 = tc::ex2(y0), p1 = tc::ex2(y1);
+                        ps[(k >> 1) & 7] += p0 + p1;
+                        sv[k >> 1] = tc::pack_bf16x2(p0, p1);     // packed in place: k/2 < k
+                    }
+                    psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                    const float ymax = fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3]));
+                    // a row without a reference yet takes one from its first valid score
+                    return m_ref == -INFINITY ? ymax != -INFINITY : ymax > 8.f;
+                };
+                const bool full_warp = __all_sync(0xffffffffu, lo == 0 && hi == SEG - 1);
+                bool done = false;
+                if (!new_branch) {
+                    const bool over = full_warp ? one_pass(std::false_type{}) : one_pass(std::true_type{});
+                    done = tc::named_bar_and(2 + quarter, 64, !over);
+                    if (done) m_use = m_ref;
+                }
+                if (!done) {
+                    if (full_warp)
+                        half_row(std::false_type{});
+                    else
+                        half_row(std::true_type{});
+                }
                 tc::tmem_st32(tS0 + sb * 128 + lane_off + half * 32, sv);
                 tc::tmem_wait_st();
 
                 // O may be touched only after the previous P V has landed; the wait is
-                // skipped when this tile neither rescales O nor closes a branch (P V of
-                // tile k is the k-th completion of pv_done, so the parity stays known)
+                // skipped when this tile neither rescales O nor closes a branch
                 if (have_prev) {
                     const bool touch_o = (new_branch && cur_br >= 0) || __any_sync(0xffffffffu, rescale);
                     if (touch_o) {
-                        if (!warp_wait(bar.pv_done(), npv & 1, abort_flag)) {
+                        if (!wait_pv(gi - 1)) {
                             ok = false;
                             break;
                         }
                         tc::fence_after_sync();
                     }
-                    ++npv;
                 }
                 if (new_branch && cur_br >= 0) correction(cur_br);
                 if (new_branch) l = 0.f;
@@ -787,11 +842,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) break;
             if (have_prev) {
-                if (!warp_wait(bar.pv_done(), npv & 1, abort_flag)) {
+                if (!wait_pv(gi - 1)) {
                     ok = false;
                     break;
                 }
-                ++npv;
                 tc::fence_after_sync();
                 correction(cur_br);
             }
