@@ -608,6 +608,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int cur_br = -1;
             bool acc_has = false, have_prev = false;
             float m_ref = -INFINITY, l = 0.f;      // l: this half's share of the row sum
+            // the row's gates are read now and o_sel's half-row is brought into L2, so
+            // that neither load's latency lands in a branch end or the epilogue
+            float gate[3] = {1.f, 1.f, 1.f};
+            if (a.gates && row_valid && !split_mode) {
+                const float* grow_gates = a.gates + grow * 3;
+                gate[0] = grow_gates[0];
+                gate[1] = grow_gates[1];
+                gate[2] = grow_gates[2];
+            }
+            if (a.o_sel != nullptr && row_valid && !split_mode)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.o_sel + grow * DV + half * (DV / 2)));
 
             // folds gate * O / l of the finished branch into Acc (warp-uniform); in
             // split mode writes this share's O / l and lse for the row instead
@@ -639,7 +650,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 float wgt = 0.f;
                 if (row_valid && lrow > 0.f) {
-                    const float g = a.gates ? a.gates[grow * 3 + br] : 1.f;
+                    const float g = br == 0 ? gate[0] : br == 1 ? gate[1] : gate[2];
                     wgt = g / lrow;
                 }
 #pragma unroll 1
@@ -859,7 +870,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             // selected branch computed outside: out += g_sel * o_sel
             const bool add_sel = a.o_sel != nullptr && (a.s.flags & NSA_BR_SEL) && row_valid;
-            const float g_sel = add_sel ? (a.gates ? a.gates[grow * 3 + 1] : 1.f) : 0.f;
+            const float g_sel = add_sel ? gate[1] : 0.f;
             // epilogue: this half of the Acc row (+ the selected branch) -> bf16 -> out
 #pragma unroll 1
             for (int c = half * DVH; c < (half + 1) * DVH; c += 32) {
