@@ -7,8 +7,8 @@
 // per-block results by their normalisers recovers that single softmax.
 //
 // HBM-bound: a thread owns 8 output columns of one (query, head) and issues
-// all of its slots' 16-byte partial loads (after one read of the query's
-// block ids) before combining them.
+// its slots' 16-byte partial loads eight at a time (after one read of the
+// query's block ids) before combining them.
 #include "common.cuh"
 
 namespace nsa {
@@ -16,6 +16,7 @@ namespace nsa {
 namespace {
 
 constexpr int MG_MAXK = 16;   // slots per query handled here (the block-major path needs top_k <= 16)
+constexpr int MG_BATCH = 8;
 
 __global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
                                                         const __nv_bfloat16* __restrict__ part_o,
@@ -41,26 +42,33 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_
     __syncthreads();
     if (h >= hpt) return;
     const int nvalid = nvalid_s;
-    uint4 raw[MG_MAXK];
-#pragma unroll
-    for (int sl = 0; sl < MG_MAXK; ++sl)              // every load of the row issued at once
-        if (sl < nvalid)
-            raw[sl] = __ldcs(reinterpret_cast<const uint4*>(part_o + ((prow0 + sl) * hpt + h) * s.dv + c8 * 8));
     float m = -INFINITY;
 #pragma unroll
     for (int sl = 0; sl < MG_MAXK; ++sl)
         if (sl < nvalid) m = fmaxf(m, lse_s[sl * hpt + h]);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     float wsum = 0.f;
+    // slots in batches of MG_BATCH whose loads are issued together (three CTAs of
+    // 256 threads per SM keep enough bytes in flight with half the row at a time,
+    // and the 80-register budget holds a batch without spilling)
 #pragma unroll
-    for (int sl = 0; sl < MG_MAXK; ++sl) {
-        if (sl >= nvalid) break;
-        const float w = exp2f(lse_s[sl * hpt + h] - m);
-        wsum += w;
-        float f[8];
-        unpack8(raw[sl], f);
+    for (int b0 = 0; b0 < MG_MAXK; b0 += MG_BATCH) {
+        if (b0 >= nvalid) break;
+        uint4 raw[MG_BATCH];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        for (int k = 0; k < MG_BATCH; ++k)
+            if (b0 + k < nvalid)
+                raw[k] = __ldcs(reinterpret_cast<const uint4*>(part_o + ((prow0 + b0 + k) * hpt + h) * s.dv + c8 * 8));
+#pragma unroll
+        for (int k = 0; k < MG_BATCH; ++k) {
+            if (b0 + k >= nvalid) break;
+            const float w = exp2f(lse_s[(b0 + k) * hpt + h] - m);
+            wsum += w;
+            float f[8];
+            unpack8(raw[k], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll
