@@ -66,6 +66,7 @@ _SIGS = {
                       ctypes.POINTER(ctypes.c_int32)],
     "nsa_timing_enable": [ctypes.c_int32],
     "nsa_check_bounded_wait": [ctypes.c_uint64, _vp],
+    "nsa_set_wait_limit_ns": [ctypes.c_uint64],
     "nsa_bwd_workspace_size": [_cfgp, ctypes.POINTER(_sz)],
     "nsa_sparse_attn_bwd": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                             _sz, _vp],
@@ -147,6 +148,10 @@ def nsa_sparse_attn_bwd(cfg, q, k, v, kcmp, vcmp, gates, idx, d_out, dq, dk, dv,
 
 def nsa_check_bounded_wait(limit_ns: int, stream=None):
     _check("nsa_check_bounded_wait", lib.nsa_check_bounded_wait(limit_ns, _stream(stream)))
+
+
+def nsa_set_wait_limit_ns(limit_ns: int):
+    _check("nsa_set_wait_limit_ns", lib.nsa_set_wait_limit_ns(limit_ns))
 
 
 def nsa_get_device_status() -> int:

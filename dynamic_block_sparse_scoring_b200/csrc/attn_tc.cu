@@ -103,7 +103,7 @@ struct Smem {
     static constexpr int META_OFF = V_OFF + NS * VC * CHUNK;
     static constexpr int UNION_OFF = META_OFF + NM * (int)sizeof(KeyTile);
     static constexpr int XCH_OFF = UNION_OFF + MAX_UNION * 4;      // row max / sum exchange
-    static constexpr int BAR_OFF = XCH_OFF + 6 * BM * 4;
+    static constexpr int BAR_OFF = XCH_OFF + 6 * BM * 4 + 64;       // + pair status words
     // barriers: q_full, q_empty, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
     // meta_full[NM], meta_empty[NM], s_full[2], p_full[2], pv_done[2], drain
     static constexpr int NBAR = 2 + 4 * NS + 2 * NM + 4 + 3;
@@ -156,16 +156,15 @@ __device__ __forceinline__ WorkTile decode_work(const TcArgs& a, int w) {
     return t;
 }
 
+// Limit of every wait on a copy, an MMA or another role (WAIT_NS unless a test
+// shortened it through nsa_set_wait_limit_ns); the drains before TMEM is freed
+// keep WAIT_NS.
+__constant__ uint64_t c_wait_ns = WAIT_NS;
+
 // Every lane waits (each acquires the barrier); the result is made warp-uniform
 // so that a timeout seen by one lane unwinds the whole warp together.
 __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
-    return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, abort_flag, WAIT_NS));
-}
-
-// Barrier between the two softmax warps that hold the two halves of the same
-// rows (warps w and w + 4 of the softmax warpgroups): named barrier 2 + w % 4.
-__device__ __forceinline__ void named_sync_softmax() {
-    asm volatile("bar.sync %0, 64;" ::"r"(2 + (int)((threadIdx.x >> 5) & 3)) : "memory");
+    return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, abort_flag, c_wait_ns));
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag) {
@@ -498,13 +497,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t gm = 0, gi = 0, wt = 0;
             bool ok = true;
             for (int work = blockIdx.x; ok && work < a.n_work * a.n_split; work += gridDim.x, ++wt) {
-                if (!tc::mbar_wait(bar.q_full(), wt & 1, abort_flag, WAIT_NS)) { ok = false; break; }
+                if (!tc::mbar_wait(bar.q_full(), wt & 1, abort_flag, c_wait_ns)) { ok = false; break; }
                 bool have_prev = false;
                 uint32_t prev_gi = 0;
                 int prev_first = 0;
                 while (true) {
                     const int slot = gm % NM;
-                    if (!tc::mbar_wait(bar.meta_full(slot), (gm / NM) & 1, abort_flag, WAIT_NS)) {
+                    if (!tc::mbar_wait(bar.meta_full(slot), (gm / NM) & 1, abort_flag, c_wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -514,7 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     ++gm;
                     if (br != BR_END) {
                         const int st = gi % NS;
-                        if (!tc::mbar_wait(bar.k_full(st), (gi / NS) & 1, abort_flag, WAIT_NS)) {
+                        if (!tc::mbar_wait(bar.k_full(st), (gi / NS) & 1, abort_flag, c_wait_ns)) {
                             ok = false;
                             break;
                         }
@@ -536,9 +535,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         // O (+)= P V for the previous key tile
                         const int pst = prev_gi % NS;
                         if (!tc::mbar_wait(bar.p_full(prev_gi & 1), (prev_gi >> 1) & 1, abort_flag,
-                                           WAIT_NS) ||
+                                           c_wait_ns) ||
                             !tc::mbar_wait(bar.v_full(pst), (prev_gi / NS) & 1, abort_flag,
-                                           WAIT_NS)) {
+                                           c_wait_ns)) {
                             ok = false;
                             break;
                         }
@@ -581,6 +580,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         float* xmax = reinterpret_cast<float*>(sm + L::XCH_OFF);   // [2 parity][2 half][BM]
         float* xsum = xmax + 4 * BM;                                 // [2 half][BM]
+        int* xstat = reinterpret_cast<int*>(xsum + 2 * BM);          // [2 parity][8 warps]
+        const int sw = warp - 4;                                     // partner warp: sw ^ 4
+        uint32_t pseq = 0;                                           // pair barriers passed
+        // Barrier between the two warps that hold the two halves of the same rows
+        // (named barrier 2 + quarter, 64 threads).  It returns the AND of `pred` over
+        // both warps and sets `fail` when either arrives failed: a warp whose wait
+        // ran out raises the abort flag, arrives here once with failed = true and
+        // leaves, and its partner, at whichever pair barrier it reaches next, learns
+        // of it here and leaves too, so neither is left alone at a barrier.  A warp
+        // can be at most one pair barrier ahead of its partner, so the status words
+        // alternate between two slots.
+        auto pair_sync = [&](bool pred, bool failed, bool& fail) {
+            if (lane == 0) xstat[(pseq & 1) * 8 + sw] = failed ? 1 : 0;
+            const bool all = tc::named_bar_and(2 + quarter, 64, pred && !failed);
+            fail = failed || xstat[(pseq & 1) * 8 + (sw ^ 4)] != 0;
+            ++pseq;
+            return all;
+        };
+        auto fail_out = [&]() {
+            raise_abort(abort_flag);
+            bool f;
+            pair_sync(false, true, f);
+        };
         constexpr int DVH = DV / 2;
         uint32_t gm = 0, gi = 0;
         // P V of key tile k is the (k >> 1)-th completion of pv_done(k & 1).  When
@@ -623,10 +645,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // folds gate * O / l of the finished branch into Acc (warp-uniform); in
             // split mode writes this share's O / l and lse for the row instead
             auto correction = [&](int br) {
+                bool fail;
                 xsum[half * BM + r] = l;
-                named_sync_softmax();
+                pair_sync(true, false, fail);
+                if (fail) return false;
                 const float lrow = l + xsum[(half ^ 1) * BM + r];
-                named_sync_softmax();
+                pair_sync(true, false, fail);
+                if (fail) return false;
                 if (split_mode) {
                     const size_t pr = (grow * 3 + br) * a.n_split + split;
                     const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
@@ -646,7 +671,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (row_valid && half == 0)
                         a.split_lse[pr] = lrow > 0.f ? m_ref + __log2f(lrow) : -INFINITY;
                     visited |= 1u << br;
-                    return;
+                    return true;
                 }
                 float wgt = 0.f;
                 if (row_valid && lrow > 0.f) {
@@ -668,11 +693,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 tc::tmem_wait_st();
                 acc_has = true;
+                return true;
             };
 
             while (true) {
                 const int slot = gm % NM;
                 if (!warp_wait(bar.meta_full(slot), (gm / NM) & 1, abort_flag)) {
+                    fail_out();
                     ok = false;
                     break;
                 }
@@ -684,6 +711,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
                 const int sb = gi & 1;
                 if (!warp_wait(bar.s_full(sb), (gi >> 1) & 1, abort_flag)) {
+                    fail_out();
                     ok = false;
                     break;
                 }
@@ -732,7 +760,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // exchange with the other half of the row; after this barrier both
                     // halves have finished reading S, so P may overwrite it
                     xmax[((gi & 1) * 2 + half) * BM + r] = m_half;
-                    named_sync_softmax();
+                    bool fail;
+                    pair_sync(true, false, fail);
+                    if (fail) return false;
                     const float m_raw = fmaxf(m_half, xmax[((gi & 1) * 2 + (half ^ 1)) * BM + r]);
                     // scale > 0, so the scaled max is the max of the scaled scores
                     const float m_tile = m_raw * a.scale_log2;
@@ -759,6 +789,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         sv[k >> 1] = tc::pack_bf16x2(p0, p1);     // packed in place: k/2 < k
                     }
                     psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                    return true;
                 };
                 // Later tiles of a branch try one pass first: the exponentials use the
                 // row's running reference max while the tile's max is taken alongside.
@@ -802,14 +833,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 bool done = false;
                 if (!new_branch) {
                     const bool over = full_warp ? one_pass(std::false_type{}) : one_pass(std::true_type{});
-                    done = tc::named_bar_and(2 + quarter, 64, !over);
+                    bool fail;
+                    done = pair_sync(!over, false, fail);
+                    if (fail) {
+                        ok = false;
+                        break;
+                    }
                     if (done) m_use = m_ref;
                 }
-                if (!done) {
-                    if (full_warp)
-                        half_row(std::false_type{});
-                    else
-                        half_row(std::true_type{});
+                if (!done && !(full_warp ? half_row(std::false_type{}) : half_row(std::true_type{}))) {
+                    ok = false;
+                    break;
                 }
                 tc::tmem_st32(tS0 + sb * 128 + lane_off + half * 32, sv);
                 tc::tmem_wait_st();
@@ -820,13 +854,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const bool touch_o = (new_branch && cur_br >= 0) || __any_sync(0xffffffffu, rescale);
                     if (touch_o) {
                         if (!wait_pv(gi - 1)) {
+                            fail_out();
                             ok = false;
                             break;
                         }
                         tc::fence_after_sync();
                     }
                 }
-                if (new_branch && cur_br >= 0) correction(cur_br);
+                if (new_branch && cur_br >= 0 && !correction(cur_br)) {
+                    ok = false;
+                    break;
+                }
                 if (new_branch) l = 0.f;
                 if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
@@ -854,11 +892,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!ok) break;
             if (have_prev) {
                 if (!wait_pv(gi - 1)) {
+                    fail_out();
                     ok = false;
                     break;
                 }
                 tc::fence_after_sync();
-                correction(cur_br);
+                if (!correction(cur_br)) {
+                    ok = false;
+                    break;
+                }
             }
             if (split_mode) {
                 if (row_valid && half == 0)
@@ -1124,6 +1166,11 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns) {
     __syncwarp();
     const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bar, 0, &abort_flag, limit_ns));
     if (!ok && threadIdx.x == 0) raise_abort(&abort_flag);
+}
+
+cudaError_t set_wait_limit(uint64_t limit_ns) {
+    const uint64_t v = limit_ns ? limit_ns : WAIT_NS;
+    return cudaMemcpyToSymbol(c_wait_ns, &v, sizeof(v));
 }
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st) {

@@ -116,6 +116,8 @@ cudaError_t launch_split_merge(const Shape& s, int n_split, const float* split_o
 int read_and_clear_tc_status();
 // the bounded wait's failure path on a barrier nothing completes (attn_tc.cu)
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st);
+// limit of the tensor-core attention kernel's waits (0: the default of one second)
+cudaError_t set_wait_limit(uint64_t limit_ns);
 // number of invalid rows of a caller-supplied idx into *bad (synchronises st) (sel_index.cu)
 cudaError_t check_idx_rows(const Shape& s, const int32_t* idx, int* bad, cudaStream_t st);
 cudaError_t launch_sel_merge(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,

@@ -611,6 +611,11 @@ nsa_status nsa_check_bounded_wait(uint64_t limit_ns, void* stream) {
     return cuda_status(nsa::launch_wait_selftest(limit_ns, static_cast<cudaStream_t>(stream)));
 }
 
+nsa_status nsa_set_wait_limit_ns(uint64_t limit_ns) {
+    if (limit_ns > 1000000000ull) return NSA_ERR_INVALID_ARG;
+    return cuda_status(nsa::set_wait_limit(limit_ns));
+}
+
 nsa_status nsa_timing_enable(int32_t on) {
     StageTiming& t = g_timing;
     if (on && !t.created) {

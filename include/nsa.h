@@ -329,6 +329,20 @@ nsa_status nsa_get_device_status(int32_t* status);
  */
 nsa_status nsa_check_bounded_wait(uint64_t limit_ns, void* stream);
 
+/*
+ * Test and debug knob (the pages have no counterpart): the limit, in ns, of
+ * every bounded wait of the tensor-core attention kernel launched after this
+ * call (the kernel behind nsa_sparse_attn_fwd's query-major, block-major and
+ * split-K plans); 0 restores the default of one second, values above 1e9 are
+ * refused.  With a limit shorter than the copies and MMAs take, the kernel's
+ * waits give up: it raises NSA_ERR_TIMEOUT in the status word, every role
+ * unwinds (the two warps that share rows leave their barriers together) and
+ * the context stays usable.  The waits that drain in-flight copies and MMAs
+ * before the kernel frees its tensor memory keep one second.  Synchronous;
+ * not for use while another thread launches this library's kernels.
+ */
+nsa_status nsa_set_wait_limit_ns(uint64_t limit_ns);
+
 /* Organisations of nsa_sparse_attn_fwd (same results, different speed). */
 #define NSA_PATH_ROWWISE 0       /* shapes outside the tensor-core kernels' limits */
 #define NSA_PATH_QUERY_MAJOR 1   /* tensor cores; selected branch over each tile's block union */

@@ -201,6 +201,7 @@ def test_append_kv_rejects_bad_arguments_on_host(abi):
 def test_bounded_wait_self_test_rejects_bad_limits_on_host(abi):
     assert abi.lib.nsa_check_bounded_wait(0, None) == 1
     assert abi.lib.nsa_check_bounded_wait(2_000_000_000, None) == 1
+    assert abi.lib.nsa_set_wait_limit_ns(2_000_000_000) == 1
 
 
 def test_score_variant_flags_validated_on_host(abi):

@@ -3,6 +3,10 @@
 * The bounded wait that every tensor-core kernel uses gives up on a barrier
   that nothing completes, records NSA_ERR_TIMEOUT in the device status word,
   and leaves the context usable (a forward right after is still correct).
+* The tensor-core attention kernel itself, with its wait limit cut to 1 ns so
+  that its waits on copies and MMAs give up, unwinds every role (the warps
+  that share rows leave their barriers together), reports NSA_ERR_TIMEOUT,
+  and the same calls with the default limit are correct afterwards.
 * NSA_DEBUG_CHECKS: a caller-supplied idx that breaks the id rules is refused
   with NSA_ERR_INVALID_ARG before any attention kernel runs; out is untouched.
 """
@@ -68,3 +72,35 @@ def test_debug_checks_refuse_bad_ids_before_any_attention_kernel():
         torch.cuda.synchronize()
         assert bool((out == 7.0).all()), f"{name}: out was written"
     assert abi.nsa_get_device_status() == 0
+
+
+def test_attention_kernel_waits_run_out_and_the_next_calls_are_correct():
+    run = GpuRun(TINY)
+    assert abi.nsa_get_device_status() == 0
+    out = torch.empty_like(run.out)
+    ws = torch.empty(abi.nsa_workspace_size(run.cfg), dtype=torch.uint8, device="cuda")
+    abi.nsa_set_wait_limit_ns(1)
+    try:
+        # the query-major plan (ids given, no workspace) and the split-K plan (workspace)
+        st = _forward(run.cfg, run, run.idx, out)
+        torch.cuda.synchronize()
+        status_qm = abi.nsa_get_device_status()
+        abi.forward(run.cfg, run.x["q"], run.x["k"], run.x["v"], run.x["gates"], idx=run.idx,
+                    pooled=run.pooled, workspace=ws, out=out)
+        torch.cuda.synchronize()
+        status_split = abi.nsa_get_device_status()
+    finally:
+        abi.nsa_set_wait_limit_ns(0)
+    assert st == 0
+    assert status_qm == 5 and status_split == 5        # NSA_ERR_TIMEOUT from both launches
+    rows = np.arange(TINY.seqlen_q)
+    ora, _, _ = run.oracle_rows(0, rows, idx=run.idx[0].cpu().numpy())
+    assert _forward(run.cfg, run, run.idx, out) == 0
+    torch.cuda.synchronize()
+    assert abi.nsa_get_device_status() == 0
+    check_out(f64(out[0]), ora, "query-major forward after timed-out launches")
+    out2, _ = abi.forward(run.cfg, run.x["q"], run.x["k"], run.x["v"], run.x["gates"], idx=run.idx,
+                          pooled=run.pooled, workspace=ws)
+    torch.cuda.synchronize()
+    assert abi.nsa_get_device_status() == 0
+    check_out(f64(out2[0]), ora, "split-K forward after timed-out launches")
