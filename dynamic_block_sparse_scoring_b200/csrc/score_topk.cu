@@ -351,9 +351,8 @@ __global__ void __launch_bounds__(SR_NT, 2)
 #pragma unroll
     for (int j = 0; j < NSEG; ++j) qv[j] = *reinterpret_cast<const float2*>(qs + 64 * j + 2 * lane);
     bool ok = true;
-    volatile int no_abort = 0;
     for (int c = 0; c < nchunk; ++c) {
-        ok = tc::mbar_wait(wb + c % SR_NSLOT, (c / SR_NSLOT) & 1, &no_abort, 1000000000ull) && ok;
+        ok = tc::mbar_wait_bounded(wb + c % SR_NSLOT, (c / SR_NSLOT) & 1, 1000000000ull) && ok;
         const float* buf = reinterpret_cast<const float*>(ring + (c % SR_NSLOT) * SR_SLOT);
         const int nr = min(RPS, nw - c * RPS);
         float part[RPS];
