@@ -663,6 +663,89 @@ def run_config(name: str, steps: int, warmup: int, world: int, rank: int):
     return res
 
 
+def _event_ms(fn, steps: int, warmup: int) -> float:
+    """Mean device time of fn() over `steps` calls after `warmup`, each call preceded by a
+    256 MB L2 flush; CUDA events on the current stream."""
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        fn()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for s in range(steps):
+        flush.fill_(float(s))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    return tot / steps
+
+
+def run_backward(steps: int, warmup: int, seqlen: int = 8192):
+    """The backward pass (nsa_sparse_attn_bwd) on the 64k prefill's shapes at `seqlen`
+    queries, for the blocks the forward selected.  Algorithmic work: per visible (query,
+    head, key) 2*(3*d_qk + 2*d_v) FLOP (S recomputed, dP, dV, dQ, dK); the kernel runs on
+    the FP32 FFMA units, so the roofline is their peak."""
+    from dynamic_block_sparse_scoring_b200 import abi
+    wl = WORKLOADS["nsa64k"].with_(name=f"nsa64k_bwd_{seqlen}", seqlen_q=seqlen, seqlen_kv=seqlen)
+    cfg = abi.config(wl)
+    x = make_inputs(wl, device="cuda", seed=0)
+    idx = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, wl.top_k, dtype=torch.int32, device="cuda")
+    pooled = abi.alloc_pooled(cfg, "cuda")
+    abi.nsa_pool_kv(cfg, x["k"], x["v"], pooled["kbar"], pooled["kcmp"], pooled["vcmp"])
+    abi.nsa_topk_select(cfg, x["q"], pooled["kbar"], None, idx)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    d_out = torch.randn(wl.batch, wl.seqlen_q, wl.h_q, wl.d_v, generator=g, device="cuda").to(torch.bfloat16)
+    dq = torch.empty(wl.batch, wl.seqlen_q, wl.h_q, wl.d_qk, device="cuda")
+    dk = torch.empty(wl.batch, wl.h_kv, wl.seqlen_kv, wl.d_qk, device="cuda")
+    dv = torch.empty(wl.batch, wl.h_kv, wl.seqlen_kv, wl.d_v, device="cuda")
+    dg = torch.empty(wl.batch, wl.seqlen_q, wl.h_q, 3, device="cuda")
+    ws = torch.empty(max(abi.nsa_bwd_workspace_size(cfg), 1), dtype=torch.uint8, device="cuda")
+
+    def call():
+        abi.nsa_sparse_attn_bwd(cfg, x["q"], x["k"], x["v"], pooled["kcmp"], pooled["vcmp"], x["gates"],
+                                idx, d_out, dq, dk, dv, dg, ws, ws.numel())
+    ms = _event_ms(call, steps, warmup)
+    keys = sum(float(v.sum()) for v in visible_key_counts(wl).values())
+    flops = keys * wl.h_q * 2 * (3 * wl.d_qk + 2 * wl.d_v) * wl.batch
+    status = abi.nsa_get_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} in the backward: a kernel's bounded wait timed out")
+    return {"workload": wl.name, "seq_len": seqlen, "steps": steps, "ms_per_step": ms,
+            "algorithmic_flops_per_step": flops, "value": flops / ms / 1e9, "unit": "TFLOP/s",
+            "bound": "alu", "peak": ALU_FP32_TFLOPS, "frac": flops / ms / 1e9 / ALU_FP32_TFLOPS,
+            "peak_source": "FP32 FFMA: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz"}
+
+
+def run_selection_variants(steps: int, warmup: int, seqlen: int = 16384):
+    """The block selection alone (nsa_topk_select_ex) on the 64k prefill's shapes at `seqlen`
+    queries, for each score definition: summed scaled dot products (the default, on the
+    tensor cores inside the forward; here the stand-alone FFMA kernel), summed per-head
+    probabilities, compressed-branch weights, and the default with two forced sink blocks.
+    Reported as ms per call and (query, selection unit) rows per second."""
+    from dynamic_block_sparse_scoring_b200 import abi
+    from dynamic_block_sparse_scoring_b200.workloads import SCORE_CMP, SCORE_PROB, SINK_SHIFT
+    wl = WORKLOADS["nsa64k"].with_(seqlen_q=seqlen, seqlen_kv=seqlen)
+    x = make_inputs(wl, device="cuda", seed=0)
+    base = abi.config(wl)
+    pooled = abi.alloc_pooled(base, "cuda")
+    abi.nsa_pool_kv(base, x["k"], x["v"], pooled["kbar"], pooled["kcmp"], pooled["vcmp"])
+    idx = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, wl.top_k, dtype=torch.int32, device="cuda")
+    out = {}
+    for name, extra in (("dot", 0), ("prob", SCORE_PROB), ("cmp", SCORE_CMP), ("dot_2_sinks", 2 << SINK_SHIFT)):
+        cfg = abi.config(wl, flags=wl.flags | extra)
+        ms = _event_ms(lambda: abi.nsa_topk_select_ex(cfg, x["q"], pooled["kbar"], pooled["kcmp"], None, idx),
+                       steps, warmup)
+        out[name] = {"ms": ms, "rows_per_s": wl.batch * wl.h_sel * wl.seqlen_q / ms * 1e3}
+    status = abi.nsa_get_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} in the selection variants")
+    return {"workload": f"nsa64k shapes at {seqlen} queries", "steps": steps, "variants": out}
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -730,6 +813,11 @@ def run_ours(args):
         for name in ("tiny", "moba32k", "moba32k_full", "nsa128k_planted"):
             if name != wl.name:
                 others[name] = run_config(name, min(args.steps, 5), args.warmup, world, rank)
+    extras = {}
+    if not args.no_configs:
+        extras["backward"] = run_backward(min(args.steps, 3), 1)
+        extras["selection_variants"] = run_selection_variants(min(args.steps, 5), 2)
+        torch.cuda.empty_cache()
     cpu = cpu_baseline(wl, x_cpu) if x_cpu is not None else None
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -742,7 +830,8 @@ def run_ours(args):
                              "attn": float(per[:, 2].mean()) - stage_ms.get("select", 0.0)},
                 "roofline": roof, "roofline_selected": sel_roof, "peaks": src,
                 "cpu_baseline": cpu, "e2e": e2e,
-                "decode": decode, "configs": others, "gpu_launches": launches, "clocks": clk,
+                "decode": decode, "configs": others, "extras": extras, "gpu_launches": launches,
+                "clocks": clk,
                 "wall_s_timed_region": wall}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -14,12 +14,17 @@
 // are collected per token (fp32) and then spread over the token's window with
 // weight 1 / cmp_block, the derivative of the window mean.
 //
-// One CTA (128 threads) per (query row, head, sequence): the branch's scores,
-// then probabilities, then ds live in shared memory (one value per key), the
-// dot products run over the threads, and dk / dv (shared by the heads of a
-// KV group and by many queries) accumulate with fp32 atomic adds.  This is a
-// plain FFMA formulation, written for clarity of the gradient rather than
-// speed.
+// One CTA (256 threads) per (query row, selection unit, sequence) covering
+// the unit's heads (the group's G heads, or one head with per-head selection),
+// which share every key of every branch.  A branch's keys are taken 64 at a
+// time into shared memory (rows padded to an odd number of 32-bit words, so
+// that threads reading the same column of different keys hit different
+// banks) and passed over three times: the softmax statistics of every head,
+// then the branch output (for the gate gradient and D), then ds with the
+// gradients.  dk and dv of a key receive one fp32 atomic add per column and
+// row, summed over the CTA's heads first and issued by consecutive threads on
+// consecutive columns; dq stays in registers over all branches.  A plain
+// FFMA formulation of the gradient.
 #include <math.h>
 
 #include <algorithm>
@@ -30,8 +35,11 @@ namespace nsa {
 
 namespace {
 
-constexpr int BW_NT = 128;
-constexpr int BW_MAXK = 16384;          // keys of one branch held in shared memory
+constexpr int BG_NT = 256;
+constexpr int BG_KC = 64;               // keys per chunk
+constexpr int BG_MAXH = 16;             // heads per CTA
+constexpr int BG_MAXD = 256;            // d_qk, d_v
+constexpr int BG_RO = BG_MAXH * BG_MAXD / BG_NT;   // per-thread outputs of o / dq
 constexpr int BW_MAXB = 32;             // kept blocks per row
 
 struct BwdArgs {
@@ -42,58 +50,78 @@ struct BwdArgs {
     float *dq, *dk, *dv, *dgates, *dkc, *dvc;
 };
 
-__device__ __forceinline__ float block_sum(float x, float* red) {
-    x = warp_sum(x);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __syncthreads();
-    if (lane == 0) red[warp] = x;
-    __syncthreads();
-    float t = 0.f;
-    for (int w = 0; w < BW_NT / 32; ++w) t += red[w];
-    return t;
-}
+// shared-memory layout (in 4-byte words) for a shape
+struct BgLayout {
+    int hb, dqk, dv, ks, vs;   // heads, dims, padded key / value row strides (bf16)
+    int q, dos, dob, ps, ds, stat, red, krow, blk, kc, vc, total;
+    __host__ __device__ BgLayout(const Shape& s) {
+        hb = s.per_head ? 1 : s.G;
+        dqk = s.dqk;
+        dv = s.dv;
+        ks = dqk + 2;                 // (dqk / 2 + 1) words: odd
+        vs = dv + 2;
+        q = 0;                        // [hb][dqk] fp32
+        dos = q + hb * dqk;           // [hb][dv] d_out
+        dob = dos + hb * dv;          // [hb][dv] gate * d_out
+        ps = dob + hb * dv;           // [hb][KC] P
+        ds = ps + hb * BG_KC;         // [hb][KC] ds
+        stat = ds + hb * BG_KC;       // m, l, D, g, dgate: [5][BG_MAXH]
+        red = stat + 5 * BG_MAXH;     // [2 warps][4][BG_MAXH / 4] reduction scratch, x2
+        krow = red + 4 * BG_MAXH;     // [KC] key rows (int64: 2 words each)
+        blk = krow + 2 * BG_KC;       // [BW_MAXB + 1] starts, [BW_MAXB] ids, [1] count
+        kc = blk + 2 * BW_MAXB + 2;   // [KC][ks] bf16
+        vc = kc + BG_KC * ks / 2;     // [KC][vs] bf16
+        total = vc + BG_KC * vs / 2;
+    }
+};
 
-__device__ __forceinline__ float block_max(float x, float* red) {
-    x = warp_max(x);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __syncthreads();
-    if (lane == 0) red[warp] = x;
-    __syncthreads();
-    float t = -INFINITY;
-    for (int w = 0; w < BW_NT / 32; ++w) t = fmaxf(t, red[w]);
-    return t;
-}
-
-__global__ void __launch_bounds__(BW_NT) bwd_rows_kernel(BwdArgs a) {
-    extern __shared__ float bw_smem[];
+__global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
+    extern __shared__ float sm[];
     const Shape& s = a.s;
-    const int dqk = s.dqk, dv = s.dv;
-    float* qs = bw_smem;                  // [dqk] the query row
-    float* dos = qs + dqk;                // [dv] d_out of the row
-    float* dob = dos + dv;                // [dv] gate * d_out
-    float* os = dob + dv;                 // [dv] branch output
-    float* red = os + dv;                 // [4] reductions
-    int* blk_start = reinterpret_cast<int*>(red + 4);   // [BW_MAXB + 1] kept blocks' key offsets
-    int* blk_id = blk_start + BW_MAXB + 1;               // [BW_MAXB]
-    float* pe = reinterpret_cast<float*>(blk_id + BW_MAXB);   // [BW_MAXK] scores -> P -> ds
-    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x;
+    const BgLayout L(s);
+    const int hb = L.hb, dqk = s.dqk, dv = s.dv;
+    float* qs = sm + L.q;
+    float* dos = sm + L.dos;
+    float* dob = sm + L.dob;
+    float* ps = sm + L.ps;
+    float* dss = sm + L.ds;
+    float* st_m = sm + L.stat;
+    float* st_l = st_m + BG_MAXH;
+    float* st_D = st_l + BG_MAXH;
+    float* st_g = st_D + BG_MAXH;
+    float* st_dg = st_g + BG_MAXH;
+    float* red = sm + L.red;                                   // [2][4][4]
+    long long* krow = reinterpret_cast<long long*>(sm + L.krow);
+    int* blk_start = reinterpret_cast<int*>(sm + L.blk);
+    int* blk_id = blk_start + BW_MAXB + 1;
+    int* blk_n = blk_id + BW_MAXB;
+    __nv_bfloat16* kcs = reinterpret_cast<__nv_bfloat16*>(sm + L.kc);
+    __nv_bfloat16* vcs = reinterpret_cast<__nv_bfloat16*>(sm + L.vc);
+
+    const int i = blockIdx.x, unit = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t = s.q0 + i;
-    const int kvh = h / s.G;
-    const size_t row = ((size_t)b * s.Tq + i) * s.Hq + h;
-    for (int c = tid; c < dqk; c += BW_NT) qs[c] = bf2f(a.q[row * dqk + c]);
-    for (int c = tid; c < dv; c += BW_NT) dos[c] = bf2f(a.d_out[row * dv + c]);
-    __syncthreads();
-    float dq_acc[2] = {0.f, 0.f};         // columns tid and tid + 128 of dq (dqk <= 256)
+    const int h0 = s.per_head ? unit : unit * s.G;
+    const int kvh = s.per_head ? unit / s.G : unit;
+    const size_t row0 = ((size_t)b * s.Tq + i) * s.Hq + h0;        // row of head h0; heads follow
     const size_t plane = (size_t)b * s.Hkv + kvh;
+    for (int x = tid; x < hb * dqk; x += BG_NT) qs[x] = bf2f(a.q[row0 * dqk + x]);
+    for (int x = tid; x < hb * dv; x += BG_NT) dos[x] = bf2f(a.d_out[row0 * dv + x]);
+    // score thread: key e_s of the chunk, heads 4 hq .. 4 hq + 3
+    const int e_s = tid % BG_KC, hq = tid / BG_KC;
+    const bool score_thread = 4 * hq < hb;
+    float dq_acc[BG_RO];
+#pragma unroll
+    for (int r = 0; r < BG_RO; ++r) dq_acc[r] = 0.f;
+    __syncthreads();
+
     for (int br = 0; br < 3; ++br) {
         if (!(s.flags & (1u << br))) {
             // the output does not depend on a disabled branch's gate
-            if (tid == 0 && a.dgates) a.dgates[row * 3 + br] = 0.f;
+            if (tid < hb && a.dgates) a.dgates[(row0 + tid) * 3 + br] = 0.f;
             continue;
         }
-        // the branch's keys: e -> (key row, whether it is a compressed token)
-        int nkeys = 0, win_lo = 0, nblk = 0;
+        int nkeys = 0, win_lo = 0;
         if (br == 0) {
             nkeys = t >= s.lc - 1 ? min(s.n_cmp, (t - s.lc + 1) / s.sc + 1) : 0;
         } else if (br == 2) {
@@ -101,8 +129,7 @@ __global__ void __launch_bounds__(BW_NT) bwd_rows_kernel(BwdArgs a) {
             nkeys = t - win_lo + 1;
         } else {
             if (tid == 0) {
-                const int u = s.per_head ? h : kvh;
-                const int32_t* r = a.idx + (((size_t)b * s.Hsel + u) * s.Tq + i) * s.topk;
+                const int32_t* r = a.idx + (((size_t)b * s.Hsel + unit) * s.Tq + i) * s.topk;
                 int n = 0, tot = 0;
                 for (int e = 0; e < s.topk && n < BW_MAXB; ++e) {
                     const int j = r[e];
@@ -113,96 +140,209 @@ __global__ void __launch_bounds__(BW_NT) bwd_rows_kernel(BwdArgs a) {
                     ++n;
                 }
                 blk_start[n] = tot;
-                red[3] = __int_as_float(n);
+                *blk_n = n;
             }
             __syncthreads();
-            nblk = __float_as_int(red[3]);
-            nkeys = blk_start[nblk];
+            nkeys = blk_start[*blk_n];
         }
-        nkeys = min(nkeys, BW_MAXK);
-        const float g = a.gates ? a.gates[row * 3 + br] : 1.f;
-        auto key_row = [&](int e) -> size_t {         // row of k / v (or of kcmp / vcmp)
-            if (br == 0) return plane * s.n_cmp + e;
-            if (br == 2) return plane * s.Tk + win_lo + e;
-            int lo = 0;
-            while (lo + 1 < nblk && blk_start[lo + 1] <= e) ++lo;
-            return plane * s.Tk + (size_t)blk_id[lo] * s.bs + (e - blk_start[lo]);
-        };
+        if (tid < hb) {
+            st_g[tid] = a.gates ? a.gates[(row0 + tid) * 3 + br] : 1.f;
+            st_m[tid] = -INFINITY;
+            st_l[tid] = 0.f;
+            st_dg[tid] = 0.f;
+        }
+        __syncthreads();
+        for (int x = tid; x < hb * dv; x += BG_NT) dob[x] = st_g[x / dv] * dos[x];
         const __nv_bfloat16* K = br == 0 ? a.kcmp : a.k;
         const __nv_bfloat16* V = br == 0 ? a.vcmp : a.v;
-        // scores, max, probabilities
-        float mloc = -INFINITY;
-        for (int e = tid; e < nkeys; e += BW_NT) {
-            const __nv_bfloat16* kr = K + key_row(e) * dqk;
-            float acc = 0.f;
-            for (int c = 0; c < dqk; c += 8) {
-                float f[8];
-                unpack8(*reinterpret_cast<const uint4*>(kr + c), f);
+        float* dK = br == 0 ? a.dkc : a.dk;
+        float* dV = br == 0 ? a.dvc : a.dv;
+        const int nchunk = (nkeys + BG_KC - 1) / BG_KC;
+        float o_acc[BG_RO];
 #pragma unroll
-                for (int x = 0; x < 8; ++x) acc = fmaf(qs[c + x], f[x], acc);
+        for (int r = 0; r < BG_RO; ++r) o_acc[r] = 0.f;
+
+        // one chunk: key rows, K (and V) rows into shared memory, then the four heads'
+        // scores of this thread's key (scaled; -inf past the last key)
+        auto load_chunk = [&](int c0, bool with_v, float* sc4) {
+            const int nk = min(BG_KC, nkeys - c0);
+            __syncthreads();                                   // the previous chunk is consumed
+            if (tid < nk) {
+                const int e = c0 + tid;
+                long long r;
+                if (br == 0) {
+                    r = (long long)(plane * s.n_cmp + e);
+                } else if (br == 2) {
+                    r = (long long)(plane * s.Tk + win_lo + e);
+                } else {
+                    int lo = 0;
+                    while (lo + 1 < *blk_n && blk_start[lo + 1] <= e) ++lo;
+                    r = (long long)(plane * s.Tk + (size_t)blk_id[lo] * s.bs + (e - blk_start[lo]));
+                }
+                krow[tid] = r;
             }
-            pe[e] = s.scale * acc;
-            mloc = fmaxf(mloc, pe[e]);
-        }
-        const float m = block_max(mloc, red);
-        float lloc = 0.f;
-        for (int e = tid; e < nkeys; e += BW_NT) {
-            const float p = expf(pe[e] - m);
-            pe[e] = p;
-            lloc += p;
-        }
-        const float l = block_sum(lloc, red);
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        for (int e = tid; e < nkeys; e += BW_NT) pe[e] *= inv;
-        __syncthreads();
-        // branch output, gate gradient, D
-        for (int c = tid; c < dv; c += BW_NT) {
-            float acc = 0.f;
-            for (int e = 0; e < nkeys; ++e) acc = fmaf(pe[e], bf2f(V[key_row(e) * dv + c]), acc);
-            os[c] = acc;
-            dob[c] = g * dos[c];
-        }
-        __syncthreads();
-        float part = 0.f;
-        for (int c = tid; c < dv; c += BW_NT) part += dos[c] * os[c];
-        const float dgate = block_sum(part, red);
-        if (tid == 0 && a.dgates) a.dgates[row * 3 + br] = dgate;
-        const float D = g * dgate;
-        // ds_e = P_e (d_o . v_e - D); dv_e += P_e d_o
-        for (int e = tid; e < nkeys; e += BW_NT) {
-            const size_t kr = key_row(e);
-            const __nv_bfloat16* vr = V + kr * dv;
-            float dp = 0.f;
-            for (int c = 0; c < dv; c += 8) {
-                float f[8];
-                unpack8(*reinterpret_cast<const uint4*>(vr + c), f);
+            __syncthreads();
+            const int kv8 = dqk / 8, vv8 = dv / 8;
+            for (int x = tid; x < nk * kv8; x += BG_NT) {
+                const int e = x / kv8, c = (x % kv8) * 8;
+                const uint4 u = *reinterpret_cast<const uint4*>(K + krow[e] * dqk + c);
+                uint32_t* d = reinterpret_cast<uint32_t*>(kcs + e * L.ks + c);
+                d[0] = u.x; d[1] = u.y; d[2] = u.z; d[3] = u.w;
+            }
+            if (with_v)
+                for (int x = tid; x < nk * vv8; x += BG_NT) {
+                    const int e = x / vv8, c = (x % vv8) * 8;
+                    const uint4 u = *reinterpret_cast<const uint4*>(V + krow[e] * dv + c);
+                    uint32_t* d = reinterpret_cast<uint32_t*>(vcs + e * L.vs + c);
+                    d[0] = u.x; d[1] = u.y; d[2] = u.z; d[3] = u.w;
+                }
+            __syncthreads();
 #pragma unroll
-                for (int x = 0; x < 8; ++x) dp = fmaf(dob[c + x], f[x], dp);
+            for (int j = 0; j < 4; ++j) sc4[j] = -INFINITY;
+            if (score_thread && e_s < nk) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(kcs + e_s * L.ks);
+                for (int c = 0; c < dqk; c += 2) {
+                    const float2 kf = __bfloat1622float2(kr[c / 2]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int h = min(4 * hq + j, hb - 1);
+                        acc[j] = fmaf(qs[h * dqk + c], kf.x, fmaf(qs[h * dqk + c + 1], kf.y, acc[j]));
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (4 * hq + j < hb) sc4[j] = s.scale * acc[j];
             }
-            const float p = pe[e];
-            float* dvr = (br == 0 ? a.dvc : a.dv) + kr * dv;
-            for (int c = 0; c < dv; ++c) atomicAdd(dvr + c, p * dob[c]);
-            pe[e] = p * (dp - D);
+            return nk;
+        };
+
+        // pass 1: per-head max and sum of exponentials (online over chunks)
+        for (int ch = 0; ch < nchunk; ++ch) {
+            float sc4[4];
+            load_chunk(ch * BG_KC, false, sc4);
+            // the two warps of each head quad reduce their 32 keys, then combine
+            float cm[4], cl[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                cm[j] = warp_max(sc4[j]);
+                cl[j] = warp_sum(sc4[j] == -INFINITY ? 0.f : expf(sc4[j] - cm[j]));
+            }
+            if (lane == 0)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    red[(warp * 4 + j) * 2 + 0] = cm[j];
+                    red[(warp * 4 + j) * 2 + 1] = cl[j];
+                }
+            __syncthreads();
+            if (tid < hb) {
+                const int qd = tid / 4, j = tid % 4;
+                const int w0 = 2 * qd, w1 = 2 * qd + 1;              // the quad's two warps
+                const float m0 = red[(w0 * 4 + j) * 2], l0 = red[(w0 * 4 + j) * 2 + 1];
+                const float m1 = red[(w1 * 4 + j) * 2], l1 = red[(w1 * 4 + j) * 2 + 1];
+                const float mc = fmaxf(m0, m1);
+                if (mc != -INFINITY) {
+                    const float lc = (m0 == -INFINITY ? 0.f : l0 * expf(m0 - mc)) +
+                                     (m1 == -INFINITY ? 0.f : l1 * expf(m1 - mc));
+                    const float mo = st_m[tid], mn = fmaxf(mo, mc);
+                    st_l[tid] = (mo == -INFINITY ? 0.f : st_l[tid] * expf(mo - mn)) + lc * expf(mc - mn);
+                    st_m[tid] = mn;
+                }
+            }
         }
         __syncthreads();
-        // dq += scale sum_e ds_e k_e;  dk_e += scale ds_e q
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = tid + cc * BW_NT;
-            if (c >= dqk) break;
-            float acc = 0.f;
-            for (int e = 0; e < nkeys; ++e) acc = fmaf(pe[e], bf2f(K[key_row(e) * dqk + c]), acc);
-            dq_acc[cc] += s.scale * acc;
+        if (tid < hb) st_l[tid] = st_l[tid] > 0.f ? 1.f / st_l[tid] : 0.f;    // now 1 / l
+
+        // pass 2: branch output o = sum_e P_e v_e (this thread's outputs)
+        for (int ch = 0; ch < nchunk; ++ch) {
+            float sc4[4];
+            const int nk = load_chunk(ch * BG_KC, true, sc4);
+            if (score_thread)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int h = 4 * hq + j;
+                    if (h < hb) ps[h * BG_KC + e_s] = sc4[j] == -INFINITY ? 0.f : expf(sc4[j] - st_m[h]) * st_l[h];
+                }
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < BG_RO; ++r) {
+                const int x = tid + r * BG_NT;
+                if (x < hb * dv) {
+                    const int h = x / dv, c = x % dv;
+                    float acc = o_acc[r];
+                    for (int e = 0; e < nk; ++e) acc = fmaf(ps[h * BG_KC + e], bf2f(vcs[e * L.vs + c]), acc);
+                    o_acc[r] = acc;
+                }
+            }
         }
-        for (int e = tid; e < nkeys; e += BW_NT) {
-            float* dkr = (br == 0 ? a.dkc : a.dk) + key_row(e) * dqk;
-            const float w = s.scale * pe[e];
-            for (int c = 0; c < dqk; ++c) atomicAdd(dkr + c, w * qs[c]);
+        // gate gradient d_out . o and D = g d_out . o per head
+#pragma unroll
+        for (int r = 0; r < BG_RO; ++r) {
+            const int x = tid + r * BG_NT;
+            if (x < hb * dv) atomicAdd(&st_dg[x / dv], dos[x] * o_acc[r]);
+        }
+        __syncthreads();
+        if (tid < hb) {
+            if (a.dgates) a.dgates[(row0 + tid) * 3 + br] = st_dg[tid];
+            st_D[tid] = st_g[tid] * st_dg[tid];
+        }
+
+        // pass 3: ds_e = P_e (d_o . v_e - D); dv_e += sum_h P_e d_o; dk_e += scale sum_h ds_e q;
+        // dq += scale sum_e ds_e k_e
+        for (int ch = 0; ch < nchunk; ++ch) {
+            float sc4[4];
+            const int nk = load_chunk(ch * BG_KC, true, sc4);
+            if (score_thread && e_s < nk) {
+                float dp[4] = {0.f, 0.f, 0.f, 0.f};
+                const __nv_bfloat162* vr = reinterpret_cast<const __nv_bfloat162*>(vcs + e_s * L.vs);
+                for (int c = 0; c < dv; c += 2) {
+                    const float2 vf = __bfloat1622float2(vr[c / 2]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int h = min(4 * hq + j, hb - 1);
+                        dp[j] = fmaf(dob[h * dv + c], vf.x, fmaf(dob[h * dv + c + 1], vf.y, dp[j]));
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int h = 4 * hq + j;
+                    if (h < hb) {
+                        const float p = sc4[j] == -INFINITY ? 0.f : expf(sc4[j] - st_m[h]) * st_l[h];
+                        ps[h * BG_KC + e_s] = p;
+                        dss[h * BG_KC + e_s] = p * (dp[j] - st_D[h]);
+                    }
+                }
+            }
+            __syncthreads();
+            for (int x = tid; x < nk * dv; x += BG_NT) {
+                const int e = x / dv, c = x % dv;
+                float acc = 0.f;
+                for (int h = 0; h < hb; ++h) acc = fmaf(ps[h * BG_KC + e], dob[h * dv + c], acc);
+                atomicAdd(dV + krow[e] * dv + c, acc);
+            }
+            for (int x = tid; x < nk * dqk; x += BG_NT) {
+                const int e = x / dqk, c = x % dqk;
+                float acc = 0.f;
+                for (int h = 0; h < hb; ++h) acc = fmaf(dss[h * BG_KC + e], qs[h * dqk + c], acc);
+                atomicAdd(dK + krow[e] * dqk + c, s.scale * acc);
+            }
+#pragma unroll
+            for (int r = 0; r < BG_RO; ++r) {
+                const int x = tid + r * BG_NT;
+                if (x < hb * dqk) {
+                    const int h = x / dqk, c = x % dqk;
+                    float acc = 0.f;
+                    for (int e = 0; e < nk; ++e) acc = fmaf(dss[h * BG_KC + e], bf2f(kcs[e * L.ks + c]), acc);
+                    dq_acc[r] = fmaf(s.scale, acc, dq_acc[r]);
+                }
+            }
         }
         __syncthreads();
     }
-    for (int cc = 0; cc < 2; ++cc) {
-        const int c = tid + cc * BW_NT;
-        if (c < dqk) a.dq[row * dqk + c] = dq_acc[cc];
+#pragma unroll
+    for (int r = 0; r < BG_RO; ++r) {
+        const int x = tid + r * BG_NT;
+        if (x < hb * dqk) a.dq[row0 * dqk + x] = dq_acc[r];
     }
 }
 
@@ -233,16 +373,13 @@ __global__ void bwd_spread_kernel(const float* __restrict__ dkc, const float* __
 
 }  // namespace
 
-size_t bwd_smem_bytes(const Shape& s) {
-    return (size_t)(s.dqk + 3 * s.dv + 4) * 4 + (2 * BW_MAXB + 1) * 4 + (size_t)BW_MAXK * 4;
-}
+size_t bwd_smem_bytes(const Shape& s) { return (size_t)BgLayout(s).total * 4; }
 
 bool bwd_supported(const Shape& s) {
-    if (s.dqk % 8 || s.dv % 8 || s.dqk > 2 * BW_NT) return false;
-    if ((s.flags & NSA_BR_SEL) && (s.topk > BW_MAXB || (size_t)s.topk * s.bs > BW_MAXK)) return false;
-    if ((s.flags & NSA_BR_WIN) && s.win > BW_MAXK) return false;
-    if ((s.flags & NSA_BR_CMP) && s.n_cmp > BW_MAXK) return false;
-    return true;
+    if (s.dqk % 8 || s.dv % 8 || s.dqk > BG_MAXD || s.dv > BG_MAXD) return false;
+    if ((s.per_head ? 1 : s.G) > BG_MAXH) return false;
+    if ((s.flags & NSA_BR_SEL) && s.topk > BW_MAXB) return false;
+    return bwd_smem_bytes(s) <= 200 * 1024;
 }
 
 cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
@@ -257,9 +394,9 @@ cudaError_t launch_attn_bwd(const Shape& s, const __nv_bfloat16* q, const __nv_b
     if (e != cudaSuccess) return e;
     BwdArgs a{s, q, k, v, kcmp, vcmp, d_out, gates, idx, dq, dk, dv, dgates, dkc, dvc};
     const size_t smem = bwd_smem_bytes(s);
-    e = cudaFuncSetAttribute(bwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(bwd_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_rows_kernel<<<dim3(s.Tq, s.Hq, s.B), BW_NT, smem, st>>>(a);
+    bwd_group_kernel<<<dim3(s.Tq, s.per_head ? s.Hq : s.Hkv, s.B), BG_NT, smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess || !cmp) return e;
     const size_t n = (size_t)s.B * s.Hkv * s.Tk * (s.dqk + s.dv);
