@@ -39,7 +39,7 @@ constexpr int BG_NT = 256;
 constexpr int BG_KC = 64;               // keys per chunk
 constexpr int BG_MAXH = 16;             // heads per CTA
 constexpr int BG_MAXD = 256;            // d_qk, d_v
-constexpr int BG_RO = BG_MAXH * BG_MAXD / BG_NT;   // per-thread outputs of o / dq
+constexpr int BG_RO4 = BG_MAXH * BG_MAXD / 4 / BG_NT;   // per-thread column quads of o / dq
 constexpr int BW_MAXB = 32;             // kept blocks per row
 
 struct BwdArgs {
@@ -74,6 +74,32 @@ struct BgLayout {
         total = vc + BG_KC * vs / 2;
     }
 };
+
+// acc += w * sum_e p[e] * rows[e][0..3] for e < n (rows of `stride` bf16, four
+// columns at a time; p four keys at a time)
+__device__ __forceinline__ float4 fma_rows(const float* p, const __nv_bfloat16* rows, int stride, int n,
+                                           float4 acc, float w = 1.f) {
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    int e = 0;
+    for (; e + 4 <= n; e += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(p + e);
+        const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat162* r = reinterpret_cast<const __nv_bfloat162*>(rows + (e + u) * stride);
+            const float2 a0 = __bfloat1622float2(r[0]), a1 = __bfloat1622float2(r[1]);
+            t.x = fmaf(pv[u], a0.x, t.x); t.y = fmaf(pv[u], a0.y, t.y);
+            t.z = fmaf(pv[u], a1.x, t.z); t.w = fmaf(pv[u], a1.y, t.w);
+        }
+    }
+    for (; e < n; ++e) {
+        const __nv_bfloat162* r = reinterpret_cast<const __nv_bfloat162*>(rows + e * stride);
+        const float2 a0 = __bfloat1622float2(r[0]), a1 = __bfloat1622float2(r[1]);
+        t.x = fmaf(p[e], a0.x, t.x); t.y = fmaf(p[e], a0.y, t.y);
+        t.z = fmaf(p[e], a1.x, t.z); t.w = fmaf(p[e], a1.y, t.w);
+    }
+    return make_float4(fmaf(w, t.x, acc.x), fmaf(w, t.y, acc.y), fmaf(w, t.z, acc.z), fmaf(w, t.w, acc.w));
+}
 
 __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
     extern __shared__ float sm[];
@@ -110,9 +136,9 @@ __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
     // score thread: key e_s of the chunk, heads 4 hq .. 4 hq + 3
     const int e_s = tid % BG_KC, hq = tid / BG_KC;
     const bool score_thread = 4 * hq < hb;
-    float dq_acc[BG_RO];
+    float4 dq_acc[BG_RO4];
 #pragma unroll
-    for (int r = 0; r < BG_RO; ++r) dq_acc[r] = 0.f;
+    for (int r = 0; r < BG_RO4; ++r) dq_acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
 
     for (int br = 0; br < 3; ++br) {
@@ -158,9 +184,9 @@ __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
         float* dK = br == 0 ? a.dkc : a.dk;
         float* dV = br == 0 ? a.dvc : a.dv;
         const int nchunk = (nkeys + BG_KC - 1) / BG_KC;
-        float o_acc[BG_RO];
+        float4 o_acc[BG_RO4];
 #pragma unroll
-        for (int r = 0; r < BG_RO; ++r) o_acc[r] = 0.f;
+        for (int r = 0; r < BG_RO4; ++r) o_acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
 
         // one chunk: key rows, K (and V) rows into shared memory, then the four heads'
         // scores of this thread's key (scaled; -inf past the last key)
@@ -202,12 +228,13 @@ __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
             if (score_thread && e_s < nk) {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(kcs + e_s * L.ks);
-                for (int c = 0; c < dqk; c += 2) {
-                    const float2 kf = __bfloat1622float2(kr[c / 2]);
+                for (int c = 0; c < dqk; c += 4) {
+                    const float2 k0 = __bfloat1622float2(kr[c / 2]), k1 = __bfloat1622float2(kr[c / 2 + 1]);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int h = min(4 * hq + j, hb - 1);
-                        acc[j] = fmaf(qs[h * dqk + c], kf.x, fmaf(qs[h * dqk + c + 1], kf.y, acc[j]));
+                        const float4 qv = *reinterpret_cast<const float4*>(qs + h * dqk + c);
+                        acc[j] = fmaf(qv.w, k1.y, fmaf(qv.z, k1.x, fmaf(qv.y, k0.y, fmaf(qv.x, k0.x, acc[j]))));
                     }
                 }
 #pragma unroll
@@ -265,21 +292,22 @@ __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
                 }
             __syncthreads();
 #pragma unroll
-            for (int r = 0; r < BG_RO; ++r) {
-                const int x = tid + r * BG_NT;
-                if (x < hb * dv) {
-                    const int h = x / dv, c = x % dv;
-                    float acc = o_acc[r];
-                    for (int e = 0; e < nk; ++e) acc = fmaf(ps[h * BG_KC + e], bf2f(vcs[e * L.vs + c]), acc);
-                    o_acc[r] = acc;
+            for (int r = 0; r < BG_RO4; ++r) {
+                const int x = tid + r * BG_NT;                 // column quad of o
+                if (x < hb * dv / 4) {
+                    const int h = 4 * x / dv, c = 4 * x % dv;
+                    o_acc[r] = fma_rows(ps + h * BG_KC, vcs + c, L.vs, nk, o_acc[r]);
                 }
             }
         }
         // gate gradient d_out . o and D = g d_out . o per head
 #pragma unroll
-        for (int r = 0; r < BG_RO; ++r) {
+        for (int r = 0; r < BG_RO4; ++r) {
             const int x = tid + r * BG_NT;
-            if (x < hb * dv) atomicAdd(&st_dg[x / dv], dos[x] * o_acc[r]);
+            if (x < hb * dv / 4) {
+                const float4 d = *reinterpret_cast<const float4*>(dos + 4 * x);
+                atomicAdd(&st_dg[4 * x / dv], d.x * o_acc[r].x + d.y * o_acc[r].y + d.z * o_acc[r].z + d.w * o_acc[r].w);
+            }
         }
         __syncthreads();
         if (tid < hb) {
@@ -295,12 +323,13 @@ __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
             if (score_thread && e_s < nk) {
                 float dp[4] = {0.f, 0.f, 0.f, 0.f};
                 const __nv_bfloat162* vr = reinterpret_cast<const __nv_bfloat162*>(vcs + e_s * L.vs);
-                for (int c = 0; c < dv; c += 2) {
-                    const float2 vf = __bfloat1622float2(vr[c / 2]);
+                for (int c = 0; c < dv; c += 4) {
+                    const float2 v0 = __bfloat1622float2(vr[c / 2]), v1 = __bfloat1622float2(vr[c / 2 + 1]);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int h = min(4 * hq + j, hb - 1);
-                        dp[j] = fmaf(dob[h * dv + c], vf.x, fmaf(dob[h * dv + c + 1], vf.y, dp[j]));
+                        const float4 dv4 = *reinterpret_cast<const float4*>(dob + h * dv + c);
+                        dp[j] = fmaf(dv4.w, v1.y, fmaf(dv4.z, v1.x, fmaf(dv4.y, v0.y, fmaf(dv4.x, v0.x, dp[j]))));
                     }
                 }
 #pragma unroll
@@ -314,35 +343,44 @@ __global__ void __launch_bounds__(BG_NT) bwd_group_kernel(BwdArgs a) {
                 }
             }
             __syncthreads();
-            for (int x = tid; x < nk * dv; x += BG_NT) {
-                const int e = x / dv, c = x % dv;
-                float acc = 0.f;
-                for (int h = 0; h < hb; ++h) acc = fmaf(ps[h * BG_KC + e], dob[h * dv + c], acc);
-                atomicAdd(dV + krow[e] * dv + c, acc);
+            // dv and dk of the chunk's keys: four columns per thread and atomic add
+            for (int x = tid; x < nk * dv / 4; x += BG_NT) {
+                const int e = 4 * x / dv, c = 4 * x % dv;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int h = 0; h < hb; ++h) {
+                    const float p = ps[h * BG_KC + e];
+                    const float4 d = *reinterpret_cast<const float4*>(dob + h * dv + c);
+                    acc.x = fmaf(p, d.x, acc.x); acc.y = fmaf(p, d.y, acc.y);
+                    acc.z = fmaf(p, d.z, acc.z); acc.w = fmaf(p, d.w, acc.w);
+                }
+                atomicAdd(reinterpret_cast<float4*>(dV + krow[e] * dv + c), acc);
             }
-            for (int x = tid; x < nk * dqk; x += BG_NT) {
-                const int e = x / dqk, c = x % dqk;
-                float acc = 0.f;
-                for (int h = 0; h < hb; ++h) acc = fmaf(dss[h * BG_KC + e], qs[h * dqk + c], acc);
-                atomicAdd(dK + krow[e] * dqk + c, s.scale * acc);
+            for (int x = tid; x < nk * dqk / 4; x += BG_NT) {
+                const int e = 4 * x / dqk, c = 4 * x % dqk;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int h = 0; h < hb; ++h) {
+                    const float d = s.scale * dss[h * BG_KC + e];
+                    const float4 qv = *reinterpret_cast<const float4*>(qs + h * dqk + c);
+                    acc.x = fmaf(d, qv.x, acc.x); acc.y = fmaf(d, qv.y, acc.y);
+                    acc.z = fmaf(d, qv.z, acc.z); acc.w = fmaf(d, qv.w, acc.w);
+                }
+                atomicAdd(reinterpret_cast<float4*>(dK + krow[e] * dqk + c), acc);
             }
 #pragma unroll
-            for (int r = 0; r < BG_RO; ++r) {
-                const int x = tid + r * BG_NT;
-                if (x < hb * dqk) {
-                    const int h = x / dqk, c = x % dqk;
-                    float acc = 0.f;
-                    for (int e = 0; e < nk; ++e) acc = fmaf(dss[h * BG_KC + e], bf2f(kcs[e * L.ks + c]), acc);
-                    dq_acc[r] = fmaf(s.scale, acc, dq_acc[r]);
+            for (int r = 0; r < BG_RO4; ++r) {
+                const int x = tid + r * BG_NT;                 // column quad of dq
+                if (x < hb * dqk / 4) {
+                    const int h = 4 * x / dqk, c = 4 * x % dqk;
+                    dq_acc[r] = fma_rows(dss + h * BG_KC, kcs + c, L.ks, nk, dq_acc[r], s.scale);
                 }
             }
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int r = 0; r < BG_RO; ++r) {
+    for (int r = 0; r < BG_RO4; ++r) {
         const int x = tid + r * BG_NT;
-        if (x < hb * dqk) a.dq[row0 * dqk + x] = dq_acc[r];
+        if (x < hb * dqk / 4) *reinterpret_cast<float4*>(a.dq + row0 * dqk + 4 * x) = dq_acc[r];
     }
 }
 
