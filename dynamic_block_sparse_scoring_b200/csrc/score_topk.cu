@@ -439,6 +439,10 @@ constexpr int SV_NW = SV_NT / 32;
 constexpr int SV_MAXH = 16;
 constexpr int SV_MAXC = 16384;          // candidate blocks / visible compressed tokens per row
 
+// shared-memory entries kept for n candidates (a multiple of 4 floats, so the
+// arrays after them stay 16-byte aligned)
+__host__ __device__ __forceinline__ int sv_cap(int n) { return (n + 3) & ~3; }
+
 template <int VMODE, int D>
 __global__ void __launch_bounds__(SV_NT) score_variant_kernel(Shape s, const __nv_bfloat16* __restrict__ q,
                                                               const float* __restrict__ kbar,
@@ -451,9 +455,10 @@ __global__ void __launch_bounds__(SV_NT) score_variant_kernel(Shape s, const __n
     float* red_l = red_m + SV_NW * SV_MAXH;       // [NW][MAXH]
     float* hm = red_l + SV_NW * SV_MAXH;          // [MAXH] per-head max
     float* hl = hm + SV_MAXH;                     // [MAXH] per-head 1 / sum
-    float* sc = hl + SV_MAXH;                     // [SV_MAXC] block scores
-    float* pj = sc + SV_MAXC;                     // [SV_MAXC] compressed-token weights (VMODE 2)
-    unsigned long long* lists = reinterpret_cast<unsigned long long*>(pj + (VMODE == 2 ? SV_MAXC : 0));
+    // (sized to this shape's candidates, so that several CTAs share an SM)
+    float* sc = hl + SV_MAXH;                     // [nb_full] block scores
+    float* pj = sc + sv_cap(s.nb_full);           // [n_cmp] compressed-token weights (VMODE 2)
+    unsigned long long* lists = reinterpret_cast<unsigned long long*>(pj + (VMODE == 2 ? sv_cap(s.n_cmp) : 0));
     const int i = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kvh = s.per_head ? u / s.G : u;
@@ -621,8 +626,8 @@ __global__ void __launch_bounds__(SV_NT) score_variant_kernel(Shape s, const __n
 template <int VMODE, int D>
 void launch_variant(const Shape& s, const __nv_bfloat16* q, const float* kbar, const __nv_bfloat16* kcmp,
                     float* scores_out, int32_t* idx, cudaStream_t st) {
-    const int smem = (SV_MAXH * D + 2 * SV_NW * SV_MAXH + 2 * SV_MAXH + SV_MAXC * (VMODE == 2 ? 2 : 1)) * 4 +
-                     SV_NW * 32 * 8;
+    const int smem = (SV_MAXH * D + 2 * SV_NW * SV_MAXH + 2 * SV_MAXH + sv_cap(s.nb_full) +
+                      (VMODE == 2 ? sv_cap(s.n_cmp) : 0)) * 4 + SV_NW * 32 * 8;
     cudaFuncSetAttribute(score_variant_kernel<VMODE, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     score_variant_kernel<VMODE, D><<<dim3(s.Tq, s.Hsel, s.B), SV_NT, smem, st>>>(s, q, kbar, kcmp, scores_out,
                                                                                idx);
