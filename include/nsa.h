@@ -302,8 +302,8 @@ nsa_status nsa_sparse_attn_fwd_noalloc(const nsa_config* cfg, const void* q, con
  * with NSA_BR_SEL); kcmp/vcmp as nsa_pool_kv writes them (with NSA_BR_CMP).
  * Needs nsa_bwd_workspace_size() bytes of workspace (the compressed tokens'
  * gradients).  Plain fp32 CUDA-core arithmetic with atomic accumulation of
- * dk / dv (summation order varies between runs).  Limits: d_qk <= 256, at
- * most 16384 keys per branch and row (NSA_ERR_UNSUPPORTED otherwise).
+ * dk / dv (summation order varies between runs).  Limits: d_qk, d_v <= 256,
+ * <= 16 heads per selection unit, top_k <= 32 (NSA_ERR_UNSUPPORTED otherwise).
  */
 nsa_status nsa_bwd_workspace_size(const nsa_config* cfg, size_t* bytes);
 nsa_status nsa_sparse_attn_bwd(const nsa_config* cfg, const void* q, const void* k,

@@ -242,3 +242,16 @@ def test_backward_validates_on_host(abi):
     assert L.nsa_sparse_attn_bwd(ctypes.byref(cfg), *a, fake, n.value, None) == 1
     # workspace too small
     assert L.nsa_sparse_attn_bwd(ctypes.byref(cfg), *args, fake, n.value - 256, None) == 3
+
+
+def test_backward_limits_refused_on_host(abi):
+    from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS
+    fake = 1 << 20
+    args = [fake] * 12
+    for over in (dict(h_q=32, h_kv=1),                       # 32 heads share a unit
+                 dict(d_qk=320),                             # wider than 256
+                 dict(top_k=40)):                            # more kept blocks than the kernel holds
+        cfg = abi.config(WORKLOADS["tiny"].with_(seqlen_q=256, seqlen_kv=256, **over))
+        n = ctypes.c_size_t(0)
+        abi.lib.nsa_bwd_workspace_size(ctypes.byref(cfg), ctypes.byref(n))
+        assert abi.lib.nsa_sparse_attn_bwd(ctypes.byref(cfg), *args, fake, max(n.value, 1 << 20), None) == 2, over
