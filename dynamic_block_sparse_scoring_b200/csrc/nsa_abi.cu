@@ -9,6 +9,7 @@
 
 #include <algorithm>
 
+#include <nvtx3/nvToolsExt.h>
 #include "common.cuh"
 #include "sel_index.cuh"
 
@@ -207,8 +208,12 @@ nsa_status cuda_status(cudaError_t e) {
     return NSA_ERR_CUDA;
 }
 
-// Per-host-thread stage events for nsa_timing_enable / nsa_timing_read.
+// Per-host-thread stage events for nsa_timing_enable / nsa_timing_read.  The
+// same stage boundaries open and close NVTX ranges (one per stage inside one
+// per call), which a profiler attached to the process shows on its timeline;
+// without one the NVTX calls return at once.
 struct StageTiming {
+    bool nvtx_open = false;  // a stage range is open
     bool on = false;
     bool created = false;
     int dev = -1;
@@ -227,6 +232,9 @@ struct StageTiming {
         active = cudaGetDevice(&d) == cudaSuccess && d == dev;
     }
     void mark(const char* name, cudaStream_t st) {
+        if (nvtx_open) nvtxRangePop();
+        nvtxRangePushA(name);
+        nvtx_open = true;
         if (!active || n >= NSA_TIMING_MAX_STAGES) return;
         if (cudaEventRecord(ev[n], st) != cudaSuccess) {
             active = false;
@@ -236,6 +244,8 @@ struct StageTiming {
         names[n++] = name;
     }
     void end(cudaStream_t st) {
+        if (nvtx_open) nvtxRangePop();
+        nvtx_open = false;
         if (!active) return;
         closed = n > 0 && cudaEventRecord(ev[n], st) == cudaSuccess;
         if (!closed) n = 0;
@@ -247,8 +257,14 @@ thread_local StageTiming g_timing;
 // Records the end of the timed call on every return path of nsa_sparse_attn_fwd.
 struct TimingScope {
     cudaStream_t st;
-    explicit TimingScope(cudaStream_t s) : st(s) { g_timing.begin(); }
-    ~TimingScope() { g_timing.end(st); }
+    explicit TimingScope(cudaStream_t s) : st(s) {
+        nvtxRangePushA("nsa_sparse_attn_fwd");
+        g_timing.begin();
+    }
+    ~TimingScope() {
+        g_timing.end(st);
+        nvtxRangePop();
+    }
 };
 
 }  // namespace
