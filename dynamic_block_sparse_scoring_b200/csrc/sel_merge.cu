@@ -18,7 +18,7 @@ namespace {
 constexpr int MG_MAXK = 16;   // slots per query handled here (the block-major path needs top_k <= 16)
 constexpr int MG_BATCH = 8;
 
-__global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
+__global__ void __launch_bounds__(256, 4) sel_merge_kernel(Shape s, const int32_t* __restrict__ idx,
                                                         const __nv_bfloat16* __restrict__ part_o,
                                                         const float* __restrict__ part_lse,
                                                         __nv_bfloat16* __restrict__ o_sel) {
@@ -48,9 +48,9 @@ __global__ void __launch_bounds__(256, 3) sel_merge_kernel(Shape s, const int32_
         if (sl < nvalid) m = fmaxf(m, lse_s[sl * hpt + h]);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     float wsum = 0.f;
-    // slots in batches of MG_BATCH whose loads are issued together (three CTAs of
-    // 256 threads per SM keep enough bytes in flight with half the row at a time,
-    // and the 80-register budget holds a batch without spilling)
+    // slots in batches of MG_BATCH whose loads are issued together: a batch fits the
+    // 64 registers that four CTAs of 256 threads per SM leave each thread, and four
+    // CTAs keep more bytes in flight than three with the whole row at once
 #pragma unroll
     for (int b0 = 0; b0 < MG_MAXK; b0 += MG_BATCH) {
         if (b0 >= nvalid) break;
