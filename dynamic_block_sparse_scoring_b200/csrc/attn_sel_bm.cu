@@ -21,12 +21,13 @@
 // queries); every CTA takes a contiguous share of each chunk, so consecutive
 // items of a CTA share their K/V block.
 //
-// Roles (448 threads): warp 0 TMA producer (K/V once per run of items on the
-// same block, Q rows per item), warp 1 MMA lane + TMEM owner, warps 2-5 and
-// 6-9 two softmax warpgroups taking alternate items (S/P double-buffered in
-// TMEM), warps 10-13 the epilogue warpgroup (O double-buffered in TMEM,
-// drained to the partial buffers while the next items' softmax runs).  All waits are
-// bounded; a timeout records NSA_ERR_TIMEOUT in g_bm_status and unwinds.
+// Roles (480 threads): warp 0 TMA producer (item descriptors, K/V once per run
+// of items on the same block; with one head per unit also the Q rows), warp 1
+// MMA lane + TMEM owner, warps 2-5 and 6-9 two softmax warpgroups taking
+// alternate items (S/P double-buffered in TMEM), warps 10-13 the epilogue
+// warpgroup (O double-buffered in TMEM, drained to the partial buffers while the
+// next items' softmax runs), warp 14 the Q-row loader (groups of heads).  All
+// waits are bounded; a timeout records NSA_ERR_TIMEOUT in g_bm_status and unwinds.
 #include <cudaTypedefs.h>
 #include <math.h>
 
