@@ -82,68 +82,71 @@ __global__ void __launch_bounds__(256, 4) sel_merge_kernel(Shape s, const int32_
 // Zhang Xiaojun #94 transcript (bidclub.ai), §7: every head keeps its own
 // blocks and the output is that branch alone).  A kept block reaches here as
 // its 64-key sub-blocks, each one slot with its own partial; the merge is the
-// same normaliser-weighted sum, taken in batches of MO_BATCH slots whose loads
-// are issued together (running maximum rescaled between batches), and the
-// result is written to out with the branch's gate.  One thread per 8 output
-// columns of a (query, head).
+// same normaliser-weighted sum, written to out with the branch's gate.  One
+// CTA per (query, group of MO_NT / (d_v / 8) heads): the heads' block ids and
+// log-sum-exps are staged in shared memory with one coalesced pass, so every
+// thread (8 output columns of one head) knows its slot count and maximum
+// before it issues its 16-byte partial loads, eight slots at a time.
+constexpr int MO_NT = 256;
+constexpr int MO_MAXK = 64;    // slots per (query, head): kept 64-key sub-blocks
+constexpr int MO_MAXH = 32;    // heads per CTA (d_v = 64)
 constexpr int MO_BATCH = 8;
 
-__global__ void __launch_bounds__(256) sel_merge_out_kernel(Shape s, const int32_t* __restrict__ idx,
-                                                            const __nv_bfloat16* __restrict__ part_o,
-                                                            const float* __restrict__ part_lse,
-                                                            const float* __restrict__ gates,
-                                                            __nv_bfloat16* __restrict__ out) {
-    const int c8n = s.dv / 8;
-    const size_t total = (size_t)s.B * s.Tq * s.Hq * c8n;
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-         e += (size_t)gridDim.x * blockDim.x) {
-        const int c8 = (int)(e % c8n);
-        const size_t row = e / c8n;                     // (b, query, head) of out
-        const int hq = (int)(row % s.Hq);
-        const int qi = (int)((row / s.Hq) % s.Tq);
-        const int b = (int)(row / ((size_t)s.Hq * s.Tq));
-        const size_t prow0 = ((size_t)(b * s.Hsel + hq) * s.Tq + qi) * s.topk;   // unit = head
-        // the kept sub-blocks fill the first slots (-1 padded)
-        int nvalid = 0;
-        while (nvalid < s.topk && idx[prow0 + nvalid] >= 0) ++nvalid;
-        float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f, m = -INFINITY;
-        for (int kb = 0; kb < nvalid; kb += MO_BATCH) {
-            float lse[MO_BATCH];
-            uint4 raw[MO_BATCH];
-#pragma unroll
-            for (int k = 0; k < MO_BATCH; ++k) {
-                lse[k] = -INFINITY;
-                if (kb + k < nvalid) {
-                    lse[k] = __ldcs(part_lse + prow0 + kb + k);
-                    raw[k] = __ldcs(reinterpret_cast<const uint4*>(part_o + (prow0 + kb + k) * s.dv + c8 * 8));
-                }
-            }
-            float mb = m;
-#pragma unroll
-            for (int k = 0; k < MO_BATCH; ++k) mb = fmaxf(mb, lse[k]);
-            if (mb == -INFINITY) continue;             // nothing visible so far
-            const float sc = m == -INFINITY ? 0.f : exp2f(m - mb);
-            wsum *= sc;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) o[q] *= sc;
-            m = mb;
-#pragma unroll
-            for (int k = 0; k < MO_BATCH; ++k) {
-                if (kb + k >= nvalid) break;
-                const float w = exp2f(lse[k] - m);
-                wsum += w;
-                float f[8];
-                unpack8(raw[k], f);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) o[q] = fmaf(w, f[q], o[q]);
-            }
-        }
-        const float g = gates ? gates[row * 3 + 1] : 1.f;
-        const float scale = wsum > 0.f ? g / wsum : 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) o[q] *= scale;
-        *reinterpret_cast<uint4*>(out + row * s.dv + c8 * 8) = pack8(o);
+__global__ void __launch_bounds__(MO_NT, 3) sel_merge_out_kernel(Shape s, const int32_t* __restrict__ idx,
+                                                               const __nv_bfloat16* __restrict__ part_o,
+                                                               const float* __restrict__ part_lse,
+                                                               const float* __restrict__ gates,
+                                                               __nv_bfloat16* __restrict__ out) {
+    __shared__ float lse_s[MO_MAXH * MO_MAXK];
+    __shared__ int nvalid_s[MO_MAXH];
+    const int c8n = s.dv / 8, hpc = MO_NT / c8n;
+    const int qi = blockIdx.x, b = blockIdx.z;
+    const int h0 = blockIdx.y * hpc;
+    const int nh = min(hpc, s.Hq - h0);
+    if (threadIdx.x < MO_MAXH) nvalid_s[threadIdx.x] = 0;
+    __syncthreads();
+    // unit = head: the partial rows of (b, head, query) are ((b * Hsel + head) * Tq + qi) * topk + slot
+    for (int e = threadIdx.x; e < nh * s.topk; e += MO_NT) {
+        const int hl = e / s.topk, sl = e % s.topk;
+        const size_t pr = ((size_t)(b * s.Hsel + h0 + hl) * s.Tq + qi) * s.topk + sl;
+        const int blk = idx[pr];
+        const float lse = __ldcs(part_lse + pr);
+        lse_s[hl * MO_MAXK + sl] = blk >= 0 ? lse : -INFINITY;
+        if (blk >= 0) atomicAdd(&nvalid_s[hl], 1);       // the kept sub-blocks fill the first slots
     }
+    __syncthreads();
+    const int hl = threadIdx.x / c8n, c8 = threadIdx.x % c8n;
+    if (hl >= nh) return;
+    const int h = h0 + hl;
+    const int nvalid = nvalid_s[hl];
+    const float* lrow = lse_s + hl * MO_MAXK;
+    float m = -INFINITY;
+    for (int k = 0; k < nvalid; ++k) m = fmaxf(m, lrow[k]);
+    const size_t prow0 = ((size_t)(b * s.Hsel + h) * s.Tq + qi) * s.topk;
+    float o[8] = {0, 0, 0, 0, 0, 0, 0, 0}, wsum = 0.f;
+    for (int kb = 0; kb < nvalid; kb += MO_BATCH) {
+        uint4 raw[MO_BATCH];
+#pragma unroll
+        for (int k = 0; k < MO_BATCH; ++k)
+            if (kb + k < nvalid)
+                raw[k] = __ldcs(reinterpret_cast<const uint4*>(part_o + (prow0 + kb + k) * s.dv + c8 * 8));
+#pragma unroll
+        for (int k = 0; k < MO_BATCH; ++k) {
+            if (kb + k >= nvalid) break;
+            const float w = exp2f(lrow[kb + k] - m);
+            wsum += w;
+            float f[8];
+            unpack8(raw[k], f);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) o[q] = fmaf(w, f[q], o[q]);
+        }
+    }
+    const size_t row = ((size_t)b * s.Tq + qi) * s.Hq + h;      // (b, query, head) of out
+    const float g = gates ? gates[row * 3 + 1] : 1.f;
+    const float scale = wsum > 0.f ? g / wsum : 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) o[q] *= scale;
+    *reinterpret_cast<uint4*>(out + row * s.dv + c8 * 8) = pack8(o);
 }
 
 }  // namespace
@@ -151,10 +154,11 @@ __global__ void __launch_bounds__(256) sel_merge_out_kernel(Shape s, const int32
 cudaError_t launch_sel_merge_out(const Shape& s, const int32_t* idx, const __nv_bfloat16* part_o,
                                  const float* part_lse, const float* gates, __nv_bfloat16* out,
                                  cudaStream_t st) {
-    const size_t total = (size_t)s.B * s.Tq * s.Hq * (s.dv / 8);
-    if (total == 0) return cudaSuccess;
-    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
-    sel_merge_out_kernel<<<grid, 256, 0, st>>>(s, idx, part_o, part_lse, gates, out);
+    if ((size_t)s.B * s.Tq * s.Hq == 0) return cudaSuccess;
+    if (s.topk > MO_MAXK || (s.dv != 64 && s.dv != 128)) return cudaErrorInvalidValue;
+    const int hpc = MO_NT / (s.dv / 8);
+    dim3 grid(s.Tq, (s.Hq + hpc - 1) / hpc, s.B);
+    sel_merge_out_kernel<<<grid, MO_NT, 0, st>>>(s, idx, part_o, part_lse, gates, out);
     return cudaGetLastError();
 }
 
