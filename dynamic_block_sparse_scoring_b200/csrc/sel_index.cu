@@ -19,22 +19,38 @@ namespace nsa {
 
 namespace {
 
-// list id of pair e (flat index into idx) holding block blk
-__device__ __forceinline__ size_t list_of(size_t e, int blk, int BHsel, int Tq, int topk,
-                                          int nb_all) {
-    const size_t bu = e / ((size_t)Tq * topk);                  // b * Hsel + u
-    const int qi = (int)((e % ((size_t)Tq * topk)) / topk);
-    const size_t chunk = qi / SEL_CHUNK;
-    return (chunk * BHsel + bu) * nb_all + blk;
+// One thread per row of idx (a (sequence, unit, query)): the row's pairs all
+// fall in lists of one chunk and unit, so the list base is one division per
+// row.  A warp's 32 rows are consecutive queries, which mostly keep the same
+// blocks in the same slots (the own block above all, and with per-head
+// selection whole runs of sub-blocks), so at every slot the lanes that hit the
+// same list are combined into one atomic (warp-aggregated, __match_any_sync).
+// All 32 lanes run every slot (rows past the end take no part), so the warp
+// stays converged at the collectives.
+__device__ __forceinline__ size_t warp_row0() {
+    return ((size_t)blockIdx.x * blockDim.x + threadIdx.x) & ~size_t(31);
 }
 
 __global__ void count_pairs_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
-                                   int BHsel, int Tq, int topk, int nb_all, size_t total) {
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-         e += (size_t)gridDim.x * blockDim.x) {
-        const int blk = idx[e];
-        if (blk < 0) continue;
-        atomicAdd(&cnt[list_of(e, blk, BHsel, Tq, topk, nb_all)], 1);
+                                   int BHsel, int Tq, int topk, int nb_all, size_t rows) {
+    const int lane = threadIdx.x & 31;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t r0 = warp_row0(); r0 < rows; r0 += stride) {
+        const size_t r = r0 + lane;
+        const bool in = r < rows;
+        const size_t bu = in ? r / Tq : 0;
+        const int qi = in ? (int)(r - bu * Tq) : 0;
+        const int lbase = (int)(((size_t)(qi / SEL_CHUNK) * BHsel + bu) * nb_all);
+        const int32_t* row = idx + r * topk;
+        for (int k = 0; k < topk; ++k) {
+            const int blk = in ? row[k] : -1;
+            const unsigned valid = __ballot_sync(0xffffffffu, blk >= 0);
+            if (blk >= 0) {
+                const int lid = lbase + blk;
+                const unsigned peers = __match_any_sync(valid, lid);
+                if (lane == __ffs(peers) - 1) atomicAdd(&cnt[lid], __popc(peers));
+            }
+        }
     }
 }
 
@@ -105,15 +121,29 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 
 __global__ void fill_pairs_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ cursor,
                                   int32_t* __restrict__ list, int BHsel, int Tq, int topk,
-                                  int nb_all, size_t total) {
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-         e += (size_t)gridDim.x * blockDim.x) {
-        const int blk = idx[e];
-        if (blk < 0) continue;
-        const int rem = (int)(e % ((size_t)Tq * topk));
-        const int qi = rem / topk, slot = rem % topk;
-        const int pos = atomicAdd(&cursor[list_of(e, blk, BHsel, Tq, topk, nb_all)], 1);
-        list[pos] = qi * SEL_SLOTS + slot;
+                                  int nb_all, size_t rows) {
+    const int lane = threadIdx.x & 31;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t r0 = warp_row0(); r0 < rows; r0 += stride) {
+        const size_t r = r0 + lane;
+        const bool in = r < rows;
+        const size_t bu = in ? r / Tq : 0;
+        const int qi = in ? (int)(r - bu * Tq) : 0;
+        const int lbase = (int)(((size_t)(qi / SEL_CHUNK) * BHsel + bu) * nb_all);
+        const int32_t* row = idx + r * topk;
+        for (int k = 0; k < topk; ++k) {
+            const int blk = in ? row[k] : -1;
+            const unsigned valid = __ballot_sync(0xffffffffu, blk >= 0);
+            if (blk >= 0) {
+                const int lid = lbase + blk;
+                const unsigned peers = __match_any_sync(valid, lid);
+                const int leader = __ffs(peers) - 1;
+                int pos = 0;
+                if (lane == leader) pos = atomicAdd(&cursor[lid], __popc(peers));
+                pos = __shfl_sync(peers, pos, leader) + __popc(peers & ((1u << lane) - 1u));
+                list[pos] = qi * SEL_SLOTS + k;
+            }
+        }
     }
 }
 
@@ -207,14 +237,14 @@ cudaError_t launch_sel_index(const Shape& s, const int32_t* idx, const SelIndex&
                              cudaStream_t st) {
     const int L = (int)sel_lists(s);
     const int BHsel = s.B * s.Hsel;
-    const size_t total = (size_t)s.B * s.Hsel * s.Tq * s.topk;
+    const size_t rows = (size_t)s.B * s.Hsel * s.Tq;
     cudaError_t e = cudaMemsetAsync(x.cnt, 0, sizeof(int32_t) * L, st);
     if (e != cudaSuccess) return e;
-    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 16);
-    count_pairs_kernel<<<grid, 256, 0, st>>>(idx, x.cnt, BHsel, s.Tq, s.topk, s.nb_all, total);
+    const int grid = (int)std::min<size_t>((rows + 255) / 256, 148 * 16);
+    count_pairs_kernel<<<grid, 256, 0, st>>>(idx, x.cnt, BHsel, s.Tq, s.topk, s.nb_all, rows);
     scan_kernel<<<1, 1024, 0, st>>>(x.cnt, x.off, x.item_off, x.cursor, L, tok);
     fill_pairs_kernel<<<grid, 256, 0, st>>>(idx, x.cursor, x.list, BHsel, s.Tq, s.topk, s.nb_all,
-                                            total);
+                                            rows);
     make_items_kernel<<<(L + 255) / 256, 256, 0, st>>>(x.off, x.item_off, x.items, L, tok);
     return cudaGetLastError();
 }
