@@ -54,7 +54,7 @@ def oracle_selection(wl: Workload, q: np.ndarray, pos: np.ndarray, K: np.ndarray
     return s, idx, gap
 
 
-class GpuRun:
+class GpuCase:
     """Inputs for a workload on cuda:0 and the library's outputs for them."""
 
     def __init__(self, wl: Workload, seed=None):
@@ -149,7 +149,7 @@ def check_out(gpu: np.ndarray, ora: np.ndarray, what=""):
     return float(err.max()), float(err.mean())
 
 
-def check_selection_all_rows(run: "GpuRun", chunk: int = 2048):
+def check_selection_all_rows(run: "GpuCase", chunk: int = 2048):
     """Both GPU selections (stand-alone and inside the forward call) against the
     oracle's selection on every query row of every sequence, in row chunks.
 

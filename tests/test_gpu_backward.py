@@ -12,7 +12,7 @@ import torch
 from dynamic_block_sparse_scoring_b200 import abi
 from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS, BR_CMP, BR_SEL, BR_WIN
 from oracle import nsa_oracle as O
-from tests.parity import GpuRun, f64, oracle_cfg
+from tests.parity import GpuCase, f64, oracle_cfg
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,7 @@ def _close(got, ref, what):
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_backward_matches_oracle(name):
     wl = CASES[name]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     cfg = run.cfg
     g = torch.Generator(device="cuda")
     g.manual_seed(77)

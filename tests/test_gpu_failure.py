@@ -16,7 +16,7 @@ import torch
 
 from dynamic_block_sparse_scoring_b200 import abi
 from dynamic_block_sparse_scoring_b200.workloads import WORKLOADS, make_inputs
-from tests.parity import GpuRun, check_out, f64
+from tests.parity import GpuCase, check_out, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +29,7 @@ def test_bounded_wait_times_out_and_the_context_stays_usable():
     torch.cuda.synchronize()
     assert abi.nsa_get_device_status() == 5          # NSA_ERR_TIMEOUT ...
     assert abi.nsa_get_device_status() == 0          # ... read once, then cleared
-    run = GpuRun(TINY)                               # a full forward afterwards
+    run = GpuCase(TINY)                               # a full forward afterwards
     rows = np.arange(TINY.seqlen_q)
     ora, _, _ = run.oracle_rows(0, rows, idx=run.idx_fwd[0].cpu().numpy())
     check_out(f64(run.out[0]), ora, "forward after a timed-out wait")
@@ -44,7 +44,7 @@ def _forward(cfg, run, idx, out):
 
 
 def test_debug_checks_refuse_bad_ids_before_any_attention_kernel():
-    run = GpuRun(TINY)
+    run = GpuCase(TINY)
     checked = abi.config(TINY, flags=TINY.flags | abi.NSA_DEBUG_CHECKS)
     good = run.idx.clone()
     # valid ids pass and give the same bits as the unchecked call
@@ -75,7 +75,7 @@ def test_debug_checks_refuse_bad_ids_before_any_attention_kernel():
 
 
 def test_attention_kernel_waits_run_out_and_the_next_calls_are_correct():
-    run = GpuRun(TINY)
+    run = GpuCase(TINY)
     assert abi.nsa_get_device_status() == 0
     out = torch.empty_like(run.out)
     ws = torch.empty(abi.nsa_workspace_size(run.cfg), dtype=torch.uint8, device="cuda")

@@ -16,7 +16,7 @@ from oracle import nsa_oracle as O
 pytestmark = pytest.mark.gpu
 
 from dynamic_block_sparse_scoring_b200 import abi
-from tests.parity import (GpuRun, check_idx, check_out, check_selection_all_rows, f64,
+from tests.parity import (GpuCase, check_idx, check_out, check_selection_all_rows, f64,
                           oracle_cfg, oracle_selection, OUT_MAX_ABS, OUT_MEAN_ABS, SCORE_ATOL,
                           SCORE_RTOL)
 
@@ -128,7 +128,7 @@ EDGE = {
 }
 
 
-def compare_run(run: GpuRun, rows_per_seq, seqs=None):
+def compare_run(run: GpuCase, rows_per_seq, seqs=None):
     wl = run.wl
     seqs = range(wl.batch) if seqs is None else seqs
     for b in seqs:
@@ -157,13 +157,13 @@ def compare_run(run: GpuRun, rows_per_seq, seqs=None):
 @pytest.mark.parametrize("name", sorted(EDGE))
 def test_small_problem_all_rows(name):
     wl = EDGE[name]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     compare_run(run, np.arange(wl.seqlen_q))
 
 
 def test_pool_kv_matches_oracle():
     for wl in [TINY, EDGE["ragged_77"], WORKLOADS["nsa64k"], WORKLOADS["moba32k"]]:
-        run = GpuRun(wl) if wl.seqlen_q <= 4096 else None
+        run = GpuCase(wl) if wl.seqlen_q <= 4096 else None
         if run is None:
             cfg = abi.config(wl)
             from dynamic_block_sparse_scoring_b200.workloads import make_inputs
@@ -189,7 +189,7 @@ def test_pool_kv_matches_oracle():
                                   "prob_sinks_nsa_small"])
 def test_materialised_scores_and_select_from_scores(name):
     wl = EDGE[name]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     cfg = run.cfg
     nb_all = -(-wl.seqlen_kv // wl.sel_block)
     scores = torch.empty(wl.batch, wl.h_sel, wl.seqlen_q, nb_all, device="cuda")
@@ -218,7 +218,7 @@ def test_materialised_scores_and_select_from_scores(name):
 def test_full_attention_layer_is_dense_causal_attention():
     """MoBA's full-attention layers (a window covering the cache) against library SDPA (fp32)."""
     wl = EDGE["full_attn_mha"]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     assert abi.nsa_attn_plan(run.cfg, False, abi.nsa_workspace_size(run.cfg))[0] in ("query-major", "split-k")
     q = run.x["q"][0].float().permute(1, 0, 2)
     ref = F.scaled_dot_product_attention(q, run.x["k"][0].float(), run.x["v"][0].float(),
@@ -229,7 +229,7 @@ def test_full_attention_layer_is_dense_causal_attention():
 def test_every_block_kept_is_dense_causal_attention():
     """Library SDPA (fp32) as an independent check of the special case."""
     wl = EDGE["every_block"].with_(h_q=8, h_kv=2)
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     q = run.x["q"][0].float().permute(1, 0, 2)
     k = run.x["k"][0].float().repeat_interleave(4, dim=0)
     v = run.x["v"][0].float().repeat_interleave(4, dim=0)
@@ -247,7 +247,7 @@ SAMPLED["bm_two_chunks"] = WORKLOADS["nsa64k"].with_(name="bm_two_chunks", seqle
 def test_full_size_prefill_sampled_rows(name):
     """Selected ids on every row against the oracle; outputs on sampled rows."""
     wl = SAMPLED[name]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     if wl.branches & BR_SEL:
         check_selection_all_rows(run)
     T = wl.seqlen_q
@@ -273,7 +273,7 @@ def test_full_size_prefill_sampled_rows(name):
 
 def test_decode_every_sequence():
     wl = WORKLOADS["decode64x64k"]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     compare_run(run, [0], seqs=range(wl.batch))
 
 
@@ -281,7 +281,7 @@ def test_decode_every_sequence():
 def test_minimal_workspace_path_matches_oracle(name):
     """With only nsa_workspace_size_min() bytes the selected branch runs query-major."""
     wl = EDGE[name]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     cfg = run.cfg
     wmin = abi.nsa_workspace_size_min(cfg)
     assert wmin < abi.nsa_workspace_size(cfg)
@@ -314,7 +314,7 @@ def test_block_major_rounding_budget(name):
     tolerance), and against the query-major plan (one rounding) within the extra term
     plus one bf16 ulp (2^-7 relative) of the output."""
     wl = EDGE[name]
-    run = GpuRun(wl)
+    run = GpuCase(wl)
     assert abi.nsa_attn_plan(run.cfg, True, abi.nsa_workspace_size(run.cfg))[0] == "block-major"
     rows = np.arange(wl.seqlen_q)
     ora, _, _ = run.oracle_rows(0, rows, idx=run.idx_fwd[0].cpu().numpy())
